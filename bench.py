@@ -1,0 +1,416 @@
+"""Benchmark of one paged decode step: paged_kv_append of one new token per
+sequence, then paged_attention_decode over the whole batch.
+
+Default workload: the Llama-3-8B-shaped layer (batch 64, 32 q / 8 kv heads,
+head_dim 128, bf16, 16-token blocks, context lengths uniform in [128, 4096],
+blocks shuffled in a pool 10% larger than needed), seeded synthetic data.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is the KV-read throughput of the
+step in GB/s: the K and V bytes of every (block, kv head) tile the step reads
+(the algorithmic bytes; tail blocks count whole) divided by the device time
+of the step, measured with CUDA events on the launching stream.  Between
+timed steps a 256 MiB buffer is written (untimed) so that every step starts
+with a cold L2.  With N GPUs each rank runs its own replica (the path needs
+no exchange between GPUs) and ``value`` sums the replicas over the slowest
+rank's time.  ``--impl reference`` times the CPU oracle instead, on a bounded
+sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import workloads as W  # noqa: E402
+from paged_kv_cache_386_b200 import layout  # noqa: E402
+
+METRIC = "paged decode attention: KV-read GB/s (fraction of HBM peak); tokens/s per layer"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = ROOT / "profiles" / "ncu_traffic.json"
+KERNEL_SOURCES = ["paged_kv_cache_386_b200/csrc/pkv_kernels.cuh", "paged_kv_cache_386_b200/csrc/pkv_device.cuh",
+                  "paged_kv_cache_386_b200/csrc/pkv_api.cu"]
+
+WORKLOADS = {
+    "llama3_8b_gqa": (lambda seed: W.uniform_gqa(seed=seed),
+                      "llama3_8b_gqa: batch 64, 32 q / 8 kv heads, head_dim 128, bf16, block 16, "
+                      "context U[128,4096], shuffled pool +10%"),
+    "llama2_7b_mha": (lambda seed: W.lognormal_mha(seed=seed),
+                      "llama2_7b_mha: batch 256, 32 q = 32 kv heads, head_dim 128, fp16, block 16, "
+                      "context round(clip(lognormal(ln 300, 1), 1, 2048)), shuffled pool +10%"),
+    "shared_prefix_70b": (lambda seed: W.shared_prefix(seed=seed),
+                          "shared_prefix_70b: 128 seqs, 64 q / 8 kv heads, head_dim 128, bf16, one shared "
+                          "2048-token prefix + private suffix U[16,512]"),
+    "best_of_8": (lambda seed: W.best_of_n(seed=seed),
+                  "best_of_8: 16 prompts x 8 samples, 2000-token shared prompt + 100 private tokens, "
+                  "64 q / 8 kv heads, head_dim 128, bf16"),
+    "long_ctx_128k": (lambda seed: W.long_context(seed=seed),
+                      "long_ctx_128k: batch 4 x 131072 tokens, 64 q / 8 kv heads, head_dim 128, bf16, "
+                      "4 sink keys x4"),
+}
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update((ROOT / rel).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def measured_hbm_peak() -> tuple[float, str]:
+    p = ROOT / "MEASURED_PEAKS.json"
+    try:
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons sampled through NVML every
+    millisecond in a background thread during the timed region (read-only
+    queries; no GPU setting is changed)."""
+
+    def __init__(self, device: torch.device, period_s: float = 0.001):
+        self.device = device
+        self.period = period_s
+        self.samples: list[tuple[int, int, int]] = []
+        self.error = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def _run(self):
+        try:
+            nv, h = self._handle()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            while not self._stop.is_set():
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx,
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                self._stop.wait(self.period)
+        except Exception as e:  # NVML missing: report no samples
+            self.error = repr(e)
+
+    def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._thread.join(timeout=5)
+
+    def summary(self) -> dict:
+        names = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+                 0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+        reasons = set()
+        for _, _, r in self.samples:
+            for bit, n in names.items():
+                if r & bit:
+                    reasons.add(n)
+        sm = [c for c, _, _ in self.samples]
+        out = {"sm_mhz": statistics.median(sm) if sm else None,
+               "sm_max_mhz": self.samples[0][1] if self.samples else None,
+               "reasons": sorted(reasons), "samples": len(sm), "source": "nvml"}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units: float, max_seconds: float, world: int) -> float:
+    """Whole-job throughput: the units every replica processed over the slowest
+    rank's time (replicas process the same amount of work)."""
+    return per_rank_units * world / max_seconds
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args) -> None:
+    import paged_kv_cache_386_b200 as pkv
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    make, desc = WORKLOADS[args.workload]
+    w = make(args.seed)
+    es = w.k_cache.element_size()
+    tr = layout.decode_traffic(w.block_tables, w.context_lens, w.n_q_heads, w.n_kv_heads, w.head_dim, es)
+    kv_bytes = tr["kv_unique"]
+    decode_bytes = tr["total_unique"]
+
+    # Device copies of the whole problem.
+    kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
+    q, k_new, v_new = w.q.to(dev), w.k_new.to(dev), w.v_new.to(dev)
+    slots, bt, cl = w.slot_mapping.to(dev), w.block_tables.to(dev), w.context_lens.to(dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
+                                                        w.dtype), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
+        pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream)
+
+    # Warm-up: W steps, continued until 0.3 s have passed so that the SM
+    # clock has left its idle state before timing.
+    t_warm, warm_steps = time.perf_counter(), 0
+    while warm_steps < args.warmup or time.perf_counter() - t_warm < 0.3:
+        flush.fill_(1)
+        step()
+        warm_steps += 1
+        if warm_steps % 16 == 0:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    if pkv.pkv_get_device_error(stream) != 0:
+        raise RuntimeError("device error flag set during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clocks:
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
+            ev[i][1].record(stream)
+            pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - t0
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    decode_ms = [b.elapsed_time(c) for _, b, c in ev]
+    step_s = sum(step_ms) / 1e3
+    max_step_s = reduce_max(step_s, world, dev)
+    value = aggregate(kv_bytes, max_step_s / args.steps, world) / 1e9
+    tokens_per_s = aggregate(w.batch, max_step_s / args.steps, world)
+    dec_avg_s = sum(decode_ms) / len(decode_ms) / 1e3
+    achieved = decode_bytes / dec_avg_s / 1e9
+    peak, peak_kind = measured_hbm_peak()
+
+    # End to end through the public API with host buffers: pinned host ->
+    # device copies of this step's inputs, append + decode, device -> host read
+    # of the output, all inside the timed region.
+    h_in = [t.pin_memory() for t in (w.q, w.k_new, w.v_new, w.slot_mapping, w.block_tables, w.context_lens)]
+    d_in = [q, k_new, v_new, slots, bt, cl]
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        for d, h in zip(d_in, h_in):
+            d.copy_(h, non_blocking=True)
+        pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
+        pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_s = reduce_max(sum(e2e_ms) / 1e3, world, dev)
+    e2e_value = aggregate(kv_bytes, e2e_s / args.steps, world) / 1e9
+    if pkv.pkv_get_device_error(stream) != 0:
+        raise RuntimeError("device error flag set during the timed run")
+
+    traffic = None
+    try:
+        prof = json.loads(PROFILE_TRAFFIC.read_text())
+        if prof.get("kernel_hash") == kernel_hash() and prof.get("workload") == args.workload:
+            traffic = prof.get("dram_bytes_per_launch")
+    except Exception:
+        traffic = None
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline(w, kv_bytes, budget_s=args.cpu_budget) if (world == 1 and not args.no_cpu) else None
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(max_step_s / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": W.DTYPE_NAMES[w.dtype], "data": "synthetic (seeded N(0,1) q/K/V, random block placement)",
+            "config": {"workload": desc, "global_batch": w.batch * world, "seq_len": "ragged",
+                       "mean_context": round(tr["tokens"] / w.batch, 1), "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps (256 MiB write, untimed)", "seed": args.seed,
+                       "warmup_steps_run": warm_steps},
+            "tokens_per_s_per_layer": round(tokens_per_s, 1),
+            "kv_bytes_per_step": kv_bytes,
+            "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (decode + merge kernels)",
+                         "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "algorithmic_bytes_per_launch": decode_bytes,
+                         "avg_launch_us": round(dec_avg_s * 1e6, 2)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_s / args.steps * 1e3, 4)},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks.summary(),
+            "wall_s_timed_loop": round(wall, 4),
+        }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+
+
+def cpu_baseline(w, kv_bytes: int, budget_s: float = 20.0) -> dict:
+    """The oracle (append + fp64 decode) on the host cores, on whole sequences
+    of the same workload, for about ``budget_s`` seconds or one full pass."""
+    import oracle
+
+    cores = oracle.cpu_cores()
+    lens = w.lens()
+    n_kv, d, es = w.n_kv_heads, w.head_dim, w.k_cache.element_size()
+    order = list(range(w.batch))
+    done_bytes, done_seqs, t_total = 0, 0, 0.0
+    kc, vc = w.k_cache.clone(), w.v_cache.clone()
+    t0 = time.perf_counter()
+    oracle.kv_append(w.k_new, w.v_new, w.slot_mapping, kc, vc, w.block_size)
+    t_total += time.perf_counter() - t0
+    chunk = 8
+    for s in range(0, len(order), chunk):
+        seqs = order[s:s + chunk]
+        rows = [(b, h) for b in seqs for h in range(w.n_q_heads)]
+        t0 = time.perf_counter()
+        oracle.paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=rows, n_threads=cores)
+        t_total += time.perf_counter() - t0
+        done_seqs += len(seqs)
+        done_bytes += sum(layout.blocks_for(lens[b]) for b in seqs) * n_kv * 16 * d * es * 2
+        if t_total > budget_s:
+            break
+    return {"value": round(done_bytes / t_total / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"append + fp64 decode of {done_seqs} of {w.batch} sequences (all q heads), "
+                      f"{t_total:.1f} s on {cores} threads"}
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the CPU oracle, as it stands, on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args) -> None:
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+
+    make, desc = WORKLOADS[args.workload]
+    w = make(args.seed)
+    cores = oracle.cpu_cores()
+    es = w.k_cache.element_size()
+    # Each step: append of every new token + decode of a fixed sample of
+    # sequences (all q heads), sized to keep the whole run within minutes.
+    n_seq = w.batch if args.ref_seqs <= 0 else min(args.ref_seqs, w.batch)
+    sample = list(range(0, w.batch, max(1, w.batch // n_seq)))[:n_seq]
+    rows = [(b, h) for b in sample for h in range(w.n_q_heads)]
+    kv_bytes = sum(layout.blocks_for(w.lens()[b]) for b in sample) * w.n_kv_heads * 16 * w.head_dim * es * 2
+
+    def step():
+        kc, vc = w.k_cache, w.v_cache
+        oracle.kv_append(w.k_new, w.v_new, w.slot_mapping, kc, vc, w.block_size)
+        oracle.paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=rows, n_threads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = kv_bytes * args.steps / dt / 1e9
+    sample_desc = (f"append of all {w.batch} new tokens + fp64 decode of {len(sample)} of {w.batch} "
+                   f"sequences (all q heads) per step")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) q/K/V, random block placement)",
+        "config": {"workload": desc, "global_batch": w.batch, "seq_len": "ragged", "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample_desc},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="llama3_8b_gqa")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
+    ap.add_argument("--ref-seqs", type=int, default=0, help="sequences per reference-arm step (0: all)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

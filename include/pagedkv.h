@@ -1,0 +1,182 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: paged KV-cache append and paged
+ * single-query (decode) attention on NVIDIA B200 (sm_100a).
+ *
+ * The KV cache of one attention layer is a flat pool of fixed-size physical
+ * blocks of `block_size` tokens; a sequence reaches its tokens through a block
+ * table whose entry i names the physical block that holds its logical block i
+ * ("Transformer anatomy", ch. 15 §15.5, PagedAttention: blocks of typically 16
+ * tokens, per-sequence block table, append into the current block;
+ * "LLM Primer VI", ch. 8 §8.1: a flat physical pool, the attention kernel takes
+ * the block table as an extra input and fetches K and V indirectly by index).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tensors are dense, row-major, and live in device memory of the current CUDA
+ * device unless stated otherwise.  The caller owns every buffer; the library
+ * keeps no pointer after a call returns.
+ *
+ *   k_cache, v_cache : [num_blocks][n_kv_heads][block_size][head_dim]
+ *                      (within a block, one contiguous block_size x head_dim
+ *                      tile per kv head)
+ *   block_tables     : int32 [batch][max_blocks_per_seq]; entries past a
+ *                      sequence's last block are never read
+ *   context_lens     : int32 [batch]; tokens of each sequence, counting the
+ *                      token appended in this step
+ *   q, out           : [batch][n_q_heads][head_dim], same dtype as the caches
+ *   slot_mapping     : int64 [num_tokens]; slot = block * block_size + offset
+ *
+ * Query head h reads kv head h / (n_q_heads / n_kv_heads) (grouped-query
+ * attention with contiguous groups, "Transformer anatomy" ch. 15 §15.2 and
+ * §15.7: h_kv < h_q).
+ *
+ * Supported: block_size == 16; head_dim in {64, 128}; n_q_heads a multiple of
+ * n_kv_heads; dtype f32, f16 or bf16 (the same for q, caches and out); all
+ * pointers 16-byte aligned; batch <= PKV_MAX_BATCH.
+ *
+ * Calls are asynchronous: they enqueue work on `stream` (a cudaStream_t; NULL
+ * is the legacy default stream) and return.  Work enqueued on one stream runs
+ * in order, so an append followed by a decode on the same stream sees the
+ * appended token.
+ *
+ * Errors: arguments are checked on the host before anything is enqueued; a
+ * failed check returns a status and enqueues nothing.  Values that only the
+ * device sees (block ids, context lengths, slots) are range-checked by the
+ * kernels: a bad value sets a bit in a per-device error word (read and cleared
+ * by pkv_get_device_error), the offending access is skipped or reads zeros,
+ * and the kernel never traps.  No entry point aborts the process.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PKV_MAX_BATCH 4096
+
+typedef enum pkv_dtype {
+  PKV_F32 = 0,
+  PKV_F16 = 1,
+  PKV_BF16 = 2
+} pkv_dtype;
+
+typedef enum pkv_status {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned pointer, n_q % n_kv != 0 */
+  PKV_ERR_UNSUPPORTED = 2,   /* block_size, head_dim, dtype or batch outside the supported set */
+  PKV_ERR_OUT_OF_RANGE = 3,  /* a kernel saw a bad block id, context length or slot */
+  PKV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  PKV_ERR_WORKSPACE = 5      /* workspace too small */
+} pkv_status;
+
+/* Bits of the device error word (pkv_get_device_error). */
+#define PKV_DEVERR_BLOCK_ID 0x1u   /* block table entry outside [0, num_blocks): zeros were read */
+#define PKV_DEVERR_CONTEXT 0x2u    /* context length < 0 or > max_blocks_per_seq * block_size: clamped */
+#define PKV_DEVERR_SLOT 0x4u       /* slot >= num_blocks * block_size: the token was not written */
+#define PKV_DEVERR_TIMEOUT 0x8u    /* a bounded in-kernel wait (2 s) gave up: that launch wrote no result */
+
+/*
+ * paged_kv_append -- write the K/V of new tokens into their cache slots.
+ *
+ * For each token i with s = slot_mapping[i] >= 0 and every kv head h:
+ *   k_cache[s / block_size][h][s % block_size][:] = k[i][h][:]
+ *   v_cache[s / block_size][h][s % block_size][:] = v[i][h][:]
+ * ("Transformer anatomy" ch. 15 §15.5: a new token goes into the current
+ * block; §15.1: its K and V are concatenated onto the cache).  A negative slot
+ * marks a padding token and is skipped.  A slot >= num_blocks * block_size is
+ * skipped and sets PKV_DEVERR_SLOT.  The copy is bit-exact.  Two tokens with
+ * the same slot race (one of them wins).
+ *
+ *   k, v          : device, [num_tokens][n_kv_heads][head_dim], dtype
+ *   slot_mapping  : device, int64 [num_tokens]
+ *   k_cache, v_cache : device, layout above; written in place
+ *   stream        : cudaStream_t
+ */
+pkv_status paged_kv_append(const void* k, const void* v, const int64_t* slot_mapping,
+                           int32_t num_tokens, void* k_cache, void* v_cache,
+                           int32_t num_blocks, int32_t block_size, int32_t n_kv_heads,
+                           int32_t head_dim, pkv_dtype dtype, void* stream);
+
+/*
+ * paged_attention_workspace_size -- device scratch bytes that
+ * paged_attention_decode needs on the current device for this shape (the
+ * partial softmax states of split contexts and their merge metadata).  The
+ * result depends on the device's SM count, not on context lengths.
+ */
+pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                          int32_t head_dim, pkv_dtype dtype, size_t* bytes);
+
+/*
+ * paged_attention_decode -- single-query attention through the block table.
+ *
+ * For every sequence b and query head h, with kv = h / (n_q_heads / n_kv_heads),
+ * n = context_lens[b], and K_j, V_j the rows of logical token j found at
+ * block_tables[b][j / block_size], slot j % block_size, kv head kv:
+ *   s_j = scale * <q[b][h], K_j>,  out[b][h] = sum_j softmax(s)_j V_j
+ * ("KV Cache and PagedAttention" (gyaansetu): dot Q with all K, weights,
+ * weighted sum of V; "PagedAttention: KV cache memory management" (yfxerp)
+ * §3.2: the per-page loop, read as one softmax over the whole context).
+ * n == 0 gives a zero row.  Scores, softmax and accumulation are fp32; the
+ * result is rounded to the dtype (round to nearest even).
+ *
+ * Long contexts are split across work units (split-KV) and merged with a
+ * log-sum-exp reduction.  The result is bit-for-bit independent of where the
+ * blocks sit in the pool and of whether blocks are shared between sequences;
+ * it depends, within rounding, on the split chosen for the device.
+ *
+ *   workspace     : device scratch of at least paged_attention_workspace_size()
+ *                   bytes, 256-byte aligned, owned by the caller and not
+ *                   shared by two calls in flight at once; NULL makes the
+ *                   library take a stream-ordered allocation for this call
+ *                   (cudaMallocAsync / cudaFreeAsync on `stream`)
+ *   workspace_bytes : size of `workspace`
+ */
+pkv_status paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t batch, int32_t num_blocks,
+                                  float scale, int32_t n_q_heads, int32_t n_kv_heads,
+                                  int32_t head_dim, int32_t block_size, void* out, pkv_dtype dtype,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Tuning and test hooks for paged_attention_decode_ex. Zero-initialise. */
+typedef struct pkv_decode_options {
+  int32_t num_units;   /* 0: default split (one work unit per consumer warp on every SM);
+                          n > 0: use at most n work units (n = 1 computes every row in one
+                          unit, with no split and no merge) */
+  int32_t force_simt;  /* 1: CUDA-core path even where the tensor-core path applies */
+  int32_t reserved[6]; /* must be zero */
+} pkv_decode_options;
+
+/* paged_attention_decode with options (NULL options = paged_attention_decode). */
+pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t batch,
+                                     int32_t num_blocks, float scale, int32_t n_q_heads,
+                                     int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
+                                     void* out, pkv_dtype dtype, void* workspace,
+                                     size_t workspace_bytes, void* stream,
+                                     const pkv_decode_options* options);
+
+/*
+ * pkv_get_device_error -- synchronise `stream`, then read and clear the
+ * current device's error word.  *flags receives the PKV_DEVERR_* bits seen
+ * since the last call.  Returns PKV_ERR_OUT_OF_RANGE if any bit was set,
+ * PKV_ERR_CUDA if synchronisation failed, else PKV_OK.
+ */
+pkv_status pkv_get_device_error(void* stream, uint32_t* flags);
+
+/* Static, NUL-terminated description of a status code. */
+const char* pkv_status_string(pkv_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

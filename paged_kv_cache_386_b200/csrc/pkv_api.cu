@@ -1,0 +1,354 @@
+// pkv_api.cu -- C ABI of libpagedkv.so (declared in include/pagedkv.h):
+// argument checks, per-device set-up, tensor-map encoding and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "pagedkv.h"
+#include "pkv_kernels.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int32_t kVersion = 10000;  // 1.0.0
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+  int smem_optin = 0;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+pkv_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    d.ready = true;
+  }
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess || fn == nullptr)
+      return PKV_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *out = d;
+  return PKV_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(pkv_dtype dt) {
+  switch (dt) {
+    case PKV_F32: return 4;
+    case PKV_F16: return 2;
+    case PKV_BF16: return 2;
+    default: return 0;
+  }
+}
+
+// Query heads handled together on one kv head by the tensor-core path: the
+// largest divisor of the group size that is at most 16; 1 selects the
+// CUDA-core path.
+int heads_per_segment(int group, pkv_dtype dt, bool force_simt) {
+  if (dt == PKV_F32 || force_simt || group < 2) return 1;
+  for (int gp = 16; gp >= 2; --gp)
+    if (group % gp == 0) return gp;
+  return 1;
+}
+
+int record_floats(int gp, int head_dim) { return (gp * (head_dim + 2) + 3) & ~3; }
+
+size_t meta_bytes(int units) { return (static_cast<size_t>(units) * sizeof(int4) + 255) & ~static_cast<size_t>(255); }
+
+size_t workspace_for(int units, int gp, int head_dim) {
+  return meta_bytes(units) + static_cast<size_t>(units) * 2 * record_floats(gp, head_dim) * sizeof(float);
+}
+
+struct DecodeShape {
+  int batch, n_q, n_kv, head_dim, group, gp, ng, units;
+  pkv_dtype dtype;
+};
+
+pkv_status check_decode_args(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
+                             int32_t num_blocks, float scale, int32_t n_q_heads, int32_t n_kv_heads,
+                             int32_t head_dim, int32_t block_size, void* out, pkv_dtype dtype) {
+  if (batch < 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 ||
+      head_dim <= 0 || block_size <= 0)
+    return PKV_ERR_INVALID_ARG;
+  if (n_q_heads % n_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+  if (!(scale == scale)) return PKV_ERR_INVALID_ARG;  // NaN scale
+  if (elem_bytes(dtype) == 0) return PKV_ERR_UNSUPPORTED;
+  if (block_size != kBlockTokens) return PKV_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+  if (batch > PKV_MAX_BATCH) return PKV_ERR_UNSUPPORTED;
+  if (max_blocks_per_seq > (1 << 26)) return PKV_ERR_UNSUPPORTED;  // context lengths stay below 2^30
+  if (batch == 0) return PKV_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PKV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PKV_ERR_INVALID_ARG;
+  // Tile counts are 32-bit on the device: bound the worst case.
+  const int64_t worst = static_cast<int64_t>(batch) * max_blocks_per_seq * n_q_heads;
+  if (worst >= (int64_t(1) << 31)) return PKV_ERR_UNSUPPORTED;
+  return PKV_OK;
+}
+
+pkv_status encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dt, int num_blocks, int n_kv,
+                            int head_dim) {
+  const int es = elem_bytes(dt);
+  const CUtensorMapDataType ty = dt == PKV_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // [block][kv head][token][dim], innermost first.
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(kBlockTokens),
+                              static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * es;
+  const cuuint64_t strides[3] = {row, row * kBlockTokens, row * kBlockTokens * n_kv};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(kBlockTokens), 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = g_encode(map, ty, 4, const_cast<void*>(cache), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <int DT, int D, int GPAD>
+pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid, size_t smem,
+                         cudaStream_t stream) {
+  auto kern = pkv_decode_kernel<DT, D, GPAD>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  kern<<<grid, kDecodeThreads, smem, stream>>>(mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <int DT, int D>
+pkv_status launch_merge(const MergeParams& mp, cudaStream_t stream) {
+  const int grid = (mp.num_units + kMergeWarps - 1) / kMergeWarps;
+  pkv_merge_kernel<DT, D><<<grid, kMergeWarps * 32, 0, stream>>>(mp);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <int DT, int D>
+pkv_status dispatch_gpad(int gpad, const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid,
+                         size_t smem, cudaStream_t stream) {
+  if constexpr (DT == kF32) {
+    return launch_decode<DT, D, 0>(mk, mv, p, grid, smem, stream);
+  } else {
+    switch (gpad) {
+      case 0: return launch_decode<DT, D, 0>(mk, mv, p, grid, smem, stream);
+      case 8: return launch_decode<DT, D, 8>(mk, mv, p, grid, smem, stream);
+      default: return launch_decode<DT, D, 16>(mk, mv, p, grid, smem, stream);
+    }
+  }
+}
+
+template <int DT>
+pkv_status dispatch_dim(int head_dim, int gpad, const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p,
+                        const MergeParams& mp, int grid, size_t smem, cudaStream_t stream) {
+  pkv_status st = head_dim == 64 ? dispatch_gpad<DT, 64>(gpad, mk, mv, p, grid, smem, stream)
+                                 : dispatch_gpad<DT, 128>(gpad, mk, mv, p, grid, smem, stream);
+  if (st != PKV_OK) return st;
+  return head_dim == 64 ? launch_merge<DT, 64>(mp, stream) : launch_merge<DT, 128>(mp, stream);
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+int32_t pkv_version(void) { return kVersion; }
+
+const char* pkv_status_string(pkv_status s) {
+  switch (s) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID_ARG: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PKV_ERR_OUT_OF_RANGE: return "a kernel saw an out-of-range block id, context length or slot";
+    case PKV_ERR_CUDA: return "CUDA runtime error";
+    case PKV_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+pkv_status paged_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                           void* k_cache, void* v_cache, int32_t num_blocks, int32_t block_size,
+                           int32_t n_kv_heads, int32_t head_dim, pkv_dtype dtype, void* stream) {
+  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || n_kv_heads <= 0 || head_dim <= 0)
+    return PKV_ERR_INVALID_ARG;
+  const int es = elem_bytes(dtype);
+  if (es == 0 || block_size != kBlockTokens || (head_dim * es) % 16 != 0) return PKV_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PKV_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return PKV_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  AppendParams p;
+  p.k = static_cast<const uint8_t*>(k);
+  p.v = static_cast<const uint8_t*>(v);
+  p.slot_mapping = slot_mapping;
+  p.k_cache = static_cast<uint8_t*>(k_cache);
+  p.v_cache = static_cast<uint8_t*>(v_cache);
+  p.num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  p.n_kv_heads = n_kv_heads;
+  p.row_chunks = head_dim * es / 16;
+  p.total = static_cast<int64_t>(num_tokens) * n_kv_heads * p.row_chunks;
+  const int64_t want = (p.total + 255) / 256;
+  const int grid = static_cast<int>(want < int64_t(di.sm_count) * 8 ? want : int64_t(di.sm_count) * 8);
+  pkv_append_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                          pkv_dtype dtype, size_t* bytes) {
+  if (!bytes || batch < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0 || head_dim <= 0)
+    return PKV_ERR_INVALID_ARG;
+  if (elem_bytes(dtype) == 0 || (head_dim != 64 && head_dim != 128)) return PKV_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  // Sized for the widest head group so that force_simt never needs more.
+  const int gp = heads_per_segment(n_q_heads / n_kv_heads, dtype, false);
+  *bytes = workspace_for(di.sm_count * kConsumerWarps, gp, head_dim);
+  return PKV_OK;
+}
+
+pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t batch, int32_t num_blocks, float scale,
+                                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
+                                     void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream, const pkv_decode_options* options) {
+  pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
+                                    num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
+  if (st != PKV_OK || batch == 0) return st;
+  pkv_decode_options opt = {};
+  if (options) {
+    opt = *options;
+    for (int i = 0; i < 6; ++i)
+      if (opt.reserved[i] != 0) return PKV_ERR_INVALID_ARG;
+    if (opt.num_units < 0 || (opt.force_simt != 0 && opt.force_simt != 1)) return PKV_ERR_INVALID_ARG;
+  }
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const int group = n_q_heads / n_kv_heads;
+  const int gp = heads_per_segment(group, dtype, opt.force_simt == 1);
+  const int gpad = gp == 1 ? 0 : (gp <= 8 ? 8 : 16);
+  const int default_units = di.sm_count * kConsumerWarps;
+  const int units = opt.num_units > 0 ? opt.num_units : default_units;
+  const int grid = (units + kConsumerWarps - 1) / kConsumerWarps;
+
+  // Ring depth: as many 8-slot rounds as shared memory allows (at most 4).
+  const int es = elem_bytes(dtype);
+  const size_t stage_bytes = static_cast<size_t>(2) * (head_dim * es / 128) * kBoxBytes;
+  // 1 KiB alignment slack, abort word, prefix sums and clamped lengths, and
+  // 256 bytes for the kernel's static shared memory.
+  const size_t fixed = 1024 + 16 + static_cast<size_t>(2 * batch + 1) * sizeof(int) + 256;
+  const size_t per_round = kConsumerWarps * (stage_bytes + 2 * sizeof(uint64_t));
+  if (fixed + per_round > static_cast<size_t>(di.smem_optin)) return PKV_ERR_UNSUPPORTED;
+  int stages = static_cast<int>((di.smem_optin - fixed) / per_round);
+  if (stages > 4) stages = 4;
+  const size_t smem = fixed - 256 + stages * per_round;
+
+  const size_t need = workspace_for(units, gp, head_dim);
+  void* ws = workspace;
+  bool own = false;
+  if (ws == nullptr) {
+    if (cudaMallocAsync(&ws, need, s) != cudaSuccess) return PKV_ERR_CUDA;
+    own = true;
+  } else if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
+    return PKV_ERR_WORKSPACE;
+  }
+
+  CUtensorMap mk, mv;
+  st = encode_cache_map(&mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
+  if (st == PKV_OK) st = encode_cache_map(&mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+
+  DecodeParams p;
+  p.q = q;
+  p.out = out;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.meta = static_cast<int4*>(ws);
+  p.records = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + meta_bytes(units));
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.batch = batch;
+  p.num_blocks = num_blocks;
+  p.n_q_heads = n_q_heads;
+  p.group = group;
+  p.gp = gp;
+  p.ng = n_q_heads / gp;
+  p.num_units = units;
+  p.stages = stages;
+  p.rec_floats = record_floats(gp, head_dim);
+  p.scale_log2 = scale * 1.4426950408889634f;
+
+  MergeParams mp;
+  mp.out = out;
+  mp.context_lens = context_lens;
+  mp.records = p.records;
+  mp.meta = p.meta;
+  mp.batch = batch;
+  mp.n_q_heads = n_q_heads;
+  mp.gp = gp;
+  mp.ng = p.ng;
+  mp.num_units = units;
+  mp.rec_floats = p.rec_floats;
+  mp.max_ctx = max_blocks_per_seq * kBlockTokens;
+
+  if (st == PKV_OK) {
+    switch (dtype) {
+      case PKV_F32: st = dispatch_dim<kF32>(head_dim, gpad, mk, mv, p, mp, grid, smem, s); break;
+      case PKV_F16: st = dispatch_dim<kF16>(head_dim, gpad, mk, mv, p, mp, grid, smem, s); break;
+      default: st = dispatch_dim<kBF16>(head_dim, gpad, mk, mv, p, mp, grid, smem, s); break;
+    }
+  }
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == PKV_OK) st = PKV_ERR_CUDA;
+  return st;
+}
+
+pkv_status paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t batch, int32_t num_blocks, float scale,
+                                  int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
+                                  void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  return paged_attention_decode_ex(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
+                                   num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype,
+                                   workspace, workspace_bytes, stream, nullptr);
+}
+
+pkv_status pkv_get_device_error(void* stream, uint32_t* flags) {
+  if (!flags) return PKV_ERR_INVALID_ARG;
+  *flags = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PKV_ERR_CUDA;
+  uint32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return PKV_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) return PKV_ERR_CUDA;
+  *flags = v;
+  return v ? PKV_ERR_OUT_OF_RANGE : PKV_OK;
+}
+
+}  // extern "C"

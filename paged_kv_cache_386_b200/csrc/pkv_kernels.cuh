@@ -1,0 +1,823 @@
+// pkv_kernels.cuh -- sm_100a kernels of the paged KV cache:
+//   pkv_append_kernel   scatter of new K/V rows into their slots
+//   pkv_decode_kernel   persistent split-KV paged decode attention
+//   pkv_merge_kernel    log-sum-exp merge of split contexts
+//
+// Decode design (one launch for every sequence, head group and context split):
+//
+// * Work is counted in tiles: one tile is one 16-token physical block of one kv
+//   head (a contiguous 16 x head_dim run of the pool).  A segment is the whole
+//   context of one sequence for one group of `gp` query heads that share a kv
+//   head; it has ceil(ctx / 16) tiles.  The tiles of all segments, in the order
+//   (sequence, head group, logical block), are split into `num_units` equal
+//   contiguous ranges (stream-K style).  A unit is one consumer warp, so every
+//   warp gets the same number of tiles whatever the length mix; a segment that
+//   straddles unit boundaries is a split context whose partial softmax states
+//   are merged by pkv_merge_kernel.
+// * Each CTA runs 8 consumer warps (units) and one producer warp.  Lane w of
+//   the producer walks unit w's tiles, reads the physical block id from the
+//   block table one tile ahead and issues TMA tensor loads of the K and V tile
+//   into unit w's ring of `stages` shared-memory slots (mbarrier full/empty
+//   pairs).  The tensor map views the pool as [block][kv head][token][dim] and
+//   loads 128-byte-wide boxes with the 128B swizzle, so that the consumers'
+//   shared-memory reads are free of bank conflicts.
+// * Consumers: grouped query heads (2..16 of them on one kv head, 16-bit
+//   data) use mma.sync m16n8k16 with fp32 accumulation: S = Q K^T with the
+//   query heads as the M rows, then O += P V with P taken from the S
+//   registers.  When a group has at most 8 heads the unused M rows 8..15 carry
+//   the rounding residual of P (P - round16(P)), so that P enters the product
+//   with about 16 significant bits.  A single query head per kv head, or fp32
+//   data, runs on CUDA cores (8 tokens x 4 dim-slices per warp).  Both keep an
+//   fp32 online softmax (running max and sum, exp2 with log2(e) folded into
+//   the scale) reduced with warp shuffles.
+// * The reduction order depends only on logical positions and on the split,
+//   never on where blocks sit in the pool, so the result is bit-identical
+//   under any block placement and with shared or private prefix blocks.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr int kBlockTokens = 16;
+constexpr int kConsumerWarps = 8;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kBoxBytes = 16 * 128;  // one TMA box: 16 tokens x 128 bytes
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+enum DType { kF32 = 0, kF16 = 1, kBF16 = 2 };
+
+template <int DT>
+struct DTypeInfo;
+template <>
+struct DTypeInfo<kF32> {
+  using T = float;
+  static constexpr int kBytes = 4;
+};
+template <>
+struct DTypeInfo<kF16> {
+  using T = __half;
+  static constexpr int kBytes = 2;
+};
+template <>
+struct DTypeInfo<kBF16> {
+  using T = __nv_bfloat16;
+  static constexpr int kBytes = 2;
+};
+
+// ---------------------------------------------------------------------------
+// Append
+// ---------------------------------------------------------------------------
+struct AppendParams {
+  const uint8_t* k;
+  const uint8_t* v;
+  const int64_t* slot_mapping;
+  uint8_t* k_cache;
+  uint8_t* v_cache;
+  int64_t num_slots;  // num_blocks * block_size
+  int64_t total;      // num_tokens * n_kv_heads * row_chunks
+  int32_t n_kv_heads;
+  int32_t row_chunks;  // 16-byte chunks per head row
+};
+
+__global__ void __launch_bounds__(256) pkv_append_kernel(const AppendParams p) {
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < p.total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int c = static_cast<int>(idx % p.row_chunks);
+    const int64_t th = idx / p.row_chunks;  // token * n_kv + head
+    const int h = static_cast<int>(th % p.n_kv_heads);
+    const int64_t i = th / p.n_kv_heads;
+    const int64_t s = __ldg(p.slot_mapping + i);
+    if (s < 0) continue;  // padding token
+    if (s >= p.num_slots) {
+      if (h == 0 && c == 0) flag_error(PKV_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t blk = s / kBlockTokens, off = s % kBlockTokens;
+    const int64_t src = (th * p.row_chunks + c) * 16;
+    const int64_t dst = (((blk * p.n_kv_heads + h) * kBlockTokens + off) * p.row_chunks + c) * 16;
+    const int4 kv = __ldg(reinterpret_cast<const int4*>(p.k + src));
+    const int4 vv = __ldg(reinterpret_cast<const int4*>(p.v + src));
+    *reinterpret_cast<int4*>(p.k_cache + dst) = kv;
+    *reinterpret_cast<int4*>(p.v_cache + dst) = vv;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decode
+// ---------------------------------------------------------------------------
+struct DecodeParams {
+  const void* q;
+  void* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* records;  // [num_units][2][rec_floats]
+  int4* meta;      // [num_units]
+  int32_t max_blocks_per_seq;
+  int32_t batch;
+  int32_t num_blocks;
+  int32_t n_q_heads;
+  int32_t group;       // query heads per kv head
+  int32_t gp;          // query heads per segment
+  int32_t ng;          // segments per sequence (n_q_heads / gp)
+  int32_t num_units;
+  int32_t stages;      // ring slots per consumer warp
+  int32_t rec_floats;  // floats per partial record: gp * (head_dim + 2), rounded up to 4
+  float scale_log2;    // scale * log2(e)
+};
+
+// Position of a warp in its unit's tile range.
+struct Walk {
+  int b, hg, j, nb, ctx;
+  int k, k_end;
+};
+
+__device__ __forceinline__ int clamp_ctx(int c, int max_ctx) { return c < 0 ? 0 : (c > max_ctx ? max_ctx : c); }
+
+__device__ __forceinline__ bool walk_begin(Walk& w, const int* prefix, const int* ctxs, int B, int k0, int k1) {
+  w.k = k0;
+  w.k_end = k1;
+  if (k0 >= k1) return false;
+  int lo = 0, hi = B;  // prefix[lo] <= k0 < prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= k0) lo = mid; else hi = mid;
+  }
+  w.b = lo;
+  w.ctx = ctxs[lo];
+  w.nb = (w.ctx + kBlockTokens - 1) / kBlockTokens;
+  const int local = k0 - prefix[lo];
+  w.hg = local / w.nb;
+  w.j = local - w.hg * w.nb;
+  return true;
+}
+
+__device__ __forceinline__ void walk_next(Walk& w, const int* prefix, const int* ctxs, int B, int ng) {
+  ++w.k;
+  if (++w.j == w.nb) {
+    w.j = 0;
+    if (++w.hg == ng) {
+      w.hg = 0;
+      do {
+        ++w.b;
+      } while (w.b < B && prefix[w.b + 1] == prefix[w.b]);
+      if (w.b < B) {
+        w.ctx = ctxs[w.b];
+        w.nb = (w.ctx + kBlockTokens - 1) / kBlockTokens;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int unit_of_tile(int k, int T, int U) {
+  return static_cast<int>(((static_cast<int64_t>(k) + 1) * U - 1) / T);
+}
+
+__device__ __forceinline__ int unit_begin(int u, int T, int U) {
+  return static_cast<int>(static_cast<int64_t>(u) * T / U);
+}
+
+// Byte offset of (token, dim) inside one K or V tile in shared memory: boxes of
+// 16 rows x 128 bytes, one box per 128 bytes of head dim, 16-byte chunks
+// swizzled by row (the TMA 128B swizzle).
+template <int ES>
+__device__ __forceinline__ uint32_t tile_offset(int tok, int dim) {
+  constexpr int X = 128 / ES;
+  const int y = dim / X;
+  const int xb = (dim % X) * ES;
+  return static_cast<uint32_t>(y * kBoxBytes + tok * 128 + ((((xb >> 4) ^ (tok & 7))) << 4) + (xb & 15));
+}
+
+// ---- tensor-core consumer (16-bit data, 2..16 query heads per kv head) ----
+template <int DT, int D, int GPAD>
+struct MmaConsumer {
+  static constexpr bool kBf16 = (DT == kBF16);
+  static constexpr int ES = 2;
+  using T = typename DTypeInfo<DT>::T;
+  static constexpr int KS = D / 16;  // k-steps of QK
+  static constexpr int NT = D / 8;   // n-tiles of PV
+
+  uint32_t qa[KS][4];
+  float o[NT][4];
+  float m[2], l[2];
+
+  __device__ __forceinline__ void begin(const DecodeParams& p, int b, int hg, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const T* qb = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp) * D;
+    const bool r0 = g < p.gp;
+    const bool r1 = (GPAD == 16) && (g + 8 < p.gp);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int c = ks * 16 + 2 * t;
+      qa[ks][0] = r0 ? __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + c)) : 0u;
+      qa[ks][2] = r0 ? __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + c + 8)) : 0u;
+      qa[ks][1] = r1 ? __ldg(reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + c)) : 0u;
+      qa[ks][3] = r1 ? __ldg(reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + c + 8)) : 0u;
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ void tile(uint32_t kbase, int nv, float scale_log2, int lane) {
+    const uint32_t vbase = kbase + (D / (128 / ES)) * kBoxBytes;
+    const int t = lane & 3;
+    const int mi = lane >> 3, rr = lane & 7;
+
+    // S = Q K^T: rows = query heads (g, g + 8), columns = tokens.
+    float s[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 32; ++kk) {
+      const int dim = (2 * kk + (mi >> 1)) * 16 + (mi & 1) * 8;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kbase + tile_offset<ES>(nt * 8 + rr, dim), b0, b1, b2, b3);
+        mma_16816<kBf16>(s[nt], qa[2 * kk][0], qa[2 * kk][1], qa[2 * kk][2], qa[2 * kk][3], b0, b1);
+        mma_16816<kBf16>(s[nt], qa[2 * kk + 1][0], qa[2 * kk + 1][1], qa[2 * kk + 1][2], qa[2 * kk + 1][3],
+                         b2, b3);
+      }
+    }
+
+    // Online softmax.  Thread holds tokens nt*8 + 2t + e for rows g (s[.][0..1])
+    // and g + 8 (s[.][2..3]).
+    constexpr int kRows = (GPAD == 16) ? 2 : 1;
+    float pr[2][2][2];  // [row][nt][e]
+    bool grow = false;
+    float alpha[2] = {1.f, 1.f};
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      float x[2][2];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tok = nt * 8 + 2 * t + e;
+          x[nt][e] = (tok < nv) ? s[nt][2 * r + e] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[nt][e]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mn = fmaxf(m[r], mx);
+      if (mn > m[r]) {
+        grow = true;
+        alpha[r] = exp2f(m[r] - mn);
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          pr[r][nt][e] = exp2f(x[nt][e] - mn);
+          sum += pr[r][nt][e];
+        }
+      l[r] = l[r] * alpha[r] + sum;
+      m[r] = mn;
+    }
+    if (__any_sync(0xffffffffu, grow)) {
+      const float a_lo = alpha[0];
+      const float a_hi = (GPAD == 16) ? alpha[1] : alpha[0];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] *= a_lo;
+        o[n][1] *= a_lo;
+        o[n][2] *= a_hi;
+        o[n][3] *= a_hi;
+      }
+    }
+
+    // P as the A operand of P V: a0/a2 = row g, tokens 2t.. / 8+2t..; a1/a3 =
+    // row g + 8 (the next 8 heads, or the residual of row g).
+    uint32_t pa0 = pack2<kBf16>(pr[0][0][0], pr[0][0][1]);
+    uint32_t pa2 = pack2<kBf16>(pr[0][1][0], pr[0][1][1]);
+    uint32_t pa1, pa3;
+    if constexpr (GPAD == 16) {
+      pa1 = pack2<kBf16>(pr[1][0][0], pr[1][0][1]);
+      pa3 = pack2<kBf16>(pr[1][1][0], pr[1][1][1]);
+    } else {
+      float h00, h01, h10, h11;
+      unpack2<kBf16>(pa0, h00, h01);
+      unpack2<kBf16>(pa2, h10, h11);
+      pa1 = pack2<kBf16>(pr[0][0][0] - h00, pr[0][0][1] - h01);
+      pa3 = pack2<kBf16>(pr[0][1][0] - h10, pr[0][1][1] - h11);
+    }
+
+    // Rows of V past the context may hold anything (NaN included): zero them.
+    uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+    if (nv < kBlockTokens) {
+      vm0 = ((2 * t < nv) ? 0x0000ffffu : 0u) | ((2 * t + 1 < nv) ? 0xffff0000u : 0u);
+      vm1 = ((2 * t + 8 < nv) ? 0x0000ffffu : 0u) | ((2 * t + 9 < nv) ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int nd2 = 0; nd2 < D / 16; ++nd2) {
+      const int tok = (mi & 1) * 8 + rr;
+      const int dim = (2 * nd2 + (mi >> 1)) * 8;
+      uint32_t v0, v1, v2, v3;
+      ldsm_x4_trans(vbase + tile_offset<ES>(tok, dim), v0, v1, v2, v3);
+      v0 &= vm0;
+      v2 &= vm0;
+      v1 &= vm1;
+      v3 &= vm1;
+      mma_16816<kBf16>(o[2 * nd2], pa0, pa1, pa2, pa3, v0, v1);
+      mma_16816<kBf16>(o[2 * nd2 + 1], pa0, pa1, pa2, pa3, v2, v3);
+    }
+  }
+
+  // Write either the normalised output rows or an unnormalised partial record.
+  __device__ __forceinline__ void finish(const DecodeParams& p, int b, int hg, float* rec, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float lt[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float x = l[r];
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      lt[r] = x;
+    }
+    constexpr int kRows = (GPAD == 16) ? 2 : 1;
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      const int row = g + 8 * r;
+      if (row >= p.gp) continue;
+      if (rec == nullptr) {
+        T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + row) * D;
+        const float inv = 1.f / lt[r];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          float a0, a1;
+          if constexpr (GPAD == 16) {
+            a0 = o[n][2 * r];
+            a1 = o[n][2 * r + 1];
+          } else {
+            a0 = o[n][0] + o[n][2];
+            a1 = o[n][1] + o[n][3];
+          }
+          *reinterpret_cast<uint32_t*>(ob + n * 8 + 2 * t) = pack2<kBf16>(a0 * inv, a1 * inv);
+        }
+      } else {
+        if (t == 0) {
+          rec[row] = m[r];
+          rec[p.gp + row] = lt[r];
+        }
+        float* ro = rec + 2 * p.gp + row * D;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          float a0, a1;
+          if constexpr (GPAD == 16) {
+            a0 = o[n][2 * r];
+            a1 = o[n][2 * r + 1];
+          } else {
+            a0 = o[n][0] + o[n][2];
+            a1 = o[n][1] + o[n][3];
+          }
+          *reinterpret_cast<float2*>(ro + n * 8 + 2 * t) = make_float2(a0, a1);
+        }
+      }
+    }
+  }
+};
+
+// ---- CUDA-core consumer (one query head per segment; any dtype) ----
+template <int DT, int D>
+struct SimtConsumer {
+  static constexpr int ES = DTypeInfo<DT>::kBytes;
+  using T = typename DTypeInfo<DT>::T;
+  static constexpr int DL = D / 4;        // dims per lane
+  static constexpr int EPC = 16 / ES;     // elements per 16-byte chunk
+  static constexpr int NCH = DL / EPC;    // chunks per lane row slice
+  static constexpr int DO = DL / 8;       // output dims per lane after the reduce-scatter
+
+  float qs[DL];
+  float o[DL];
+  float m, l;
+
+  __device__ __forceinline__ static void widen16(const uint4& c, float* f) {
+    if constexpr (DT == kF32) {
+      f[0] = __uint_as_float(c.x);
+      f[1] = __uint_as_float(c.y);
+      f[2] = __uint_as_float(c.z);
+      f[3] = __uint_as_float(c.w);
+    } else {
+      constexpr bool kB = (DT == kBF16);
+      unpack2<kB>(c.x, f[0], f[1]);
+      unpack2<kB>(c.y, f[2], f[3]);
+      unpack2<kB>(c.z, f[4], f[5]);
+      unpack2<kB>(c.w, f[6], f[7]);
+    }
+  }
+
+  __device__ __forceinline__ void begin(const DecodeParams& p, int b, int hg, int lane) {
+    const int sub = lane >> 3;
+    const T* qb = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.n_q_heads + hg) * D + sub * DL;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qb) + c);
+      widen16(raw, qs + c * EPC);
+    }
+#pragma unroll
+    for (int i = 0; i < DL; ++i) o[i] = 0.f;
+    m = -INFINITY;
+    l = 0.f;
+  }
+
+  __device__ __forceinline__ void tile(uint32_t kbase, int nv, float scale_log2, int lane) {
+    const uint32_t vbase = kbase + (D / (128 / ES)) * kBoxBytes;
+    const int tp = lane & 7, sub = lane >> 3;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int dim = sub * DL + c * EPC;
+      uint4 k0, k1;
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(k0.x), "=r"(k0.y), "=r"(k0.z), "=r"(k0.w)
+                   : "r"(kbase + tile_offset<ES>(tp, dim)));
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(k1.x), "=r"(k1.y), "=r"(k1.z), "=r"(k1.w)
+                   : "r"(kbase + tile_offset<ES>(tp + 8, dim)));
+      float f0[EPC], f1[EPC];
+      widen16(k0, f0);
+      widen16(k1, f1);
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) {
+        s0 = fmaf(qs[c * EPC + e], f0[e], s0);
+        s1 = fmaf(qs[c * EPC + e], f1[e], s1);
+      }
+    }
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 8);
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 8);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    const bool ok0 = tp < nv, ok1 = tp + 8 < nv;
+    const float x0 = ok0 ? s0 * scale_log2 : -INFINITY;
+    const float x1 = ok1 ? s1 * scale_log2 : -INFINITY;
+    float mx = fmaxf(x0, x1);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    const float mn = fmaxf(m, mx);
+    if (mn > m) {  // warp-uniform: m and mx are the same in every lane
+      const float alpha = exp2f(m - mn);
+      l *= alpha;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) o[i] *= alpha;
+      m = mn;
+    }
+    const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn);
+    l += p0 + p1;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int dim = sub * DL + c * EPC;
+      float f[EPC];
+      if (ok0) {
+        uint4 v0;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v0.x), "=r"(v0.y), "=r"(v0.z), "=r"(v0.w)
+                     : "r"(vbase + tile_offset<ES>(tp, dim)));
+        widen16(v0, f);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) o[c * EPC + e] = fmaf(p0, f[e], o[c * EPC + e]);
+      }
+      if (ok1) {
+        uint4 v1;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v1.x), "=r"(v1.y), "=r"(v1.z), "=r"(v1.w)
+                     : "r"(vbase + tile_offset<ES>(tp + 8, dim)));
+        widen16(v1, f);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) o[c * EPC + e] = fmaf(p1, f[e], o[c * EPC + e]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void finish(const DecodeParams& p, int b, int hg, float* rec, int lane) {
+    const int tp = lane & 7, sub = lane >> 3;
+    float lt = l;
+    lt += __shfl_xor_sync(0xffffffffu, lt, 1);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 4);
+    // Reduce-scatter of o over the 8 token lanes: after the three steps lane
+    // tp holds dims [tp * DO, tp * DO + DO) of its slice, summed.
+#pragma unroll
+    for (int step = 0; step < 3; ++step) {
+      const int mask = 4 >> step;
+      const int half = DL >> (step + 1);
+      const bool upper = (tp & mask) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? o[i] : o[i + half];
+        const float keep = upper ? o[i + half] : o[i];
+        o[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+      }
+    }
+    const int d0 = sub * DL + tp * DO;
+    if (rec == nullptr) {
+      T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg) * D + d0;
+      const float inv = 1.f / lt;
+      if constexpr (DT == kF32) {
+#pragma unroll
+        for (int i = 0; i < DO; ++i) ob[i] = o[i] * inv;
+      } else {
+#pragma unroll
+        for (int i = 0; i < DO; i += 2)
+          *reinterpret_cast<uint32_t*>(ob + i) = pack2<DT == kBF16>(o[i] * inv, o[i + 1] * inv);
+      }
+    } else {
+      if (lane == 0) {
+        rec[0] = m;
+        rec[1] = lt;
+      }
+#pragma unroll
+      for (int i = 0; i < DO; ++i) rec[2 + d0 + i] = o[i];
+    }
+  }
+};
+
+template <int DT, int D, int GPAD>
+struct ConsumerFor {
+  using type = MmaConsumer<DT, D, GPAD>;
+};
+template <int DT, int D>
+struct ConsumerFor<DT, D, 0> {
+  using type = SimtConsumer<DT, D>;
+};
+
+// GPAD: 0 = CUDA-core consumer (gp == 1); 8 or 16 = tensor-core consumer.
+template <int DT, int D, int GPAD>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    pkv_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const DecodeParams p) {
+  constexpr int ES = DTypeInfo<DT>::kBytes;
+  constexpr int X = 128 / ES;                      // elements per swizzle row
+  constexpr int Y = D / X;                         // boxes per tile
+  constexpr int kTileBytes = Y * kBoxBytes;
+  constexpr int kStageBytes = 2 * kTileBytes;
+  using Consumer = typename ConsumerFor<DT, D, GPAD>::type;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const int n_slots = kConsumerWarps * p.stages;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(ring + static_cast<size_t>(n_slots) * kStageBytes);
+  uint64_t* empty_bar = full_bar + n_slots;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty_bar + n_slots);
+  int* prefix = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 4));  // [batch + 1]
+  int* ctxs = prefix + p.batch + 1;                                                    // [batch]
+  __shared__ int warp_sums[kConsumerWarps + 1];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int B = p.batch;
+  const int max_ctx = p.max_blocks_per_seq * kBlockTokens;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < n_slots; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kConsumerWarps && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+
+  // Tiles per sequence -> exclusive prefix sums (block-wide scan).
+  {
+    const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
+    const int lo = min(B, threadIdx.x * per), hi = min(B, lo + per);
+    int local = 0;
+    for (int b = lo; b < hi; ++b) {
+      const int c0 = __ldg(p.context_lens + b);
+      const int c = clamp_ctx(c0, max_ctx);
+      if (c != c0) flag_error(PKV_DEVERR_CONTEXT);
+      ctxs[b] = c;
+      local += ((c + kBlockTokens - 1) / kBlockTokens) * p.ng;
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_sums[w];
+    int run = base + incl - local;
+    for (int b = lo; b < hi; ++b) {
+      prefix[b] = run;
+      run += ((ctxs[b] + kBlockTokens - 1) / kBlockTokens) * p.ng;
+    }
+    if (threadIdx.x == kDecodeThreads - 1) prefix[B] = base + incl;
+  }
+  __syncthreads();
+
+  const int T = prefix[B];
+  const int U = p.num_units;
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer ----------------
+    const int u = blockIdx.x * kConsumerWarps + lane;
+    Walk wk;
+    bool active = false;
+    if (lane < kConsumerWarps && u < U) active = walk_begin(wk, prefix, ctxs, B, unit_begin(u, T, U), unit_begin(u + 1, T, U));
+    auto load_phys = [&](const Walk& w) -> int {
+      int ph = __ldg(p.block_tables + static_cast<size_t>(w.b) * p.max_blocks_per_seq + w.j);
+      if (ph < 0 || ph >= p.num_blocks) {
+        flag_error(PKV_DEVERR_BLOCK_ID);
+        ph = 0;
+      }
+      return ph;
+    };
+    int next_phys = active ? load_phys(wk) : 0;
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    while (__any_sync(0xffffffffu, active)) {
+      if (active) {
+        const int phys = next_phys;
+        const int kvh = (wk.hg * p.gp) / p.group;
+        const bool more = wk.k + 1 < wk.k_end;
+        if (more) {
+          walk_next(wk, prefix, ctxs, B, p.ng);
+          next_phys = load_phys(wk);
+        }
+        const int slot = lane * p.stages + stage;
+        if (!mbar_wait_bounded(&empty_bar[slot], phase ^ 1u, abort_flag, kWaitLimitNs)) {
+          active = false;
+        } else {
+          mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
+          uint8_t* sk = ring + static_cast<size_t>(slot) * kStageBytes;
+#pragma unroll
+          for (int y = 0; y < Y; ++y) tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, kvh, phys);
+#pragma unroll
+          for (int y = 0; y < Y; ++y)
+            tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, kvh, phys);
+          ++issued;
+          if (++stage == p.stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          active = more;
+        }
+      }
+    }
+    // Do not leave while copies issued by this lane may still be landing.
+    if (lane < kConsumerWarps) {
+      for (int s = 0; s < p.stages && s < issued; ++s) {
+        const int cnt = (issued - s + p.stages - 1) / p.stages;
+        const uint32_t par = static_cast<uint32_t>((cnt - 1) & 1);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(&full_bar[lane * p.stages + s], par)) {
+          if (global_timer_ns() - t0 > kWaitLimitNs) {
+            flag_error(kDevErrTimeout);
+            break;
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int u = blockIdx.x * kConsumerWarps + warp;
+  if (u >= U) return;
+  const int k0 = unit_begin(u, T, U), k1 = unit_begin(u + 1, T, U);
+  Walk wk;
+  bool have = walk_begin(wk, prefix, ctxs, B, k0, k1);
+  int4 my_meta = make_int4(-1, 0, 0, T);
+  Consumer cs;
+  int first_seg = -1, cur_seg = -1, cur_b = 0, cur_hg = 0, seg_start = 0, seg_end = 0;
+  int stage = 0;
+  uint32_t phase = 0;
+  bool aborted = false;
+
+  auto finish_segment = [&]() {
+    const bool starts_here = seg_start >= k0, ends_here = seg_end <= k1;
+    if (starts_here && ends_here) {
+      cs.finish(p, cur_b, cur_hg, nullptr, lane);
+    } else {
+      const int slot_idx = (cur_seg == first_seg) ? 0 : 1;
+      float* rec = p.records + (static_cast<size_t>(u) * 2 + slot_idx) * p.rec_floats;
+      cs.finish(p, cur_b, cur_hg, rec, lane);
+      if (starts_here) my_meta = make_int4(cur_seg, unit_of_tile(seg_end - 1, T, U), slot_idx, T);
+    }
+  };
+
+  while (have) {
+    const int seg = wk.b * p.ng + wk.hg;
+    if (seg != cur_seg) {
+      if (cur_seg >= 0) finish_segment();
+      cur_seg = seg;
+      if (first_seg < 0) first_seg = seg;
+      cur_b = wk.b;
+      cur_hg = wk.hg;
+      seg_start = prefix[wk.b] + wk.hg * wk.nb;
+      seg_end = seg_start + wk.nb;
+      cs.begin(p, wk.b, wk.hg, lane);
+    }
+    const int slot = warp * p.stages + stage;
+    if (!mbar_wait_bounded(&full_bar[slot], phase, abort_flag, kWaitLimitNs)) {
+      aborted = true;
+      break;
+    }
+    const int nv = min(kBlockTokens, wk.ctx - wk.j * kBlockTokens);
+    cs.tile(smem_u32(ring + static_cast<size_t>(slot) * kStageBytes), nv, p.scale_log2, lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[slot]);
+    if (++stage == p.stages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+    if (wk.k + 1 < wk.k_end) walk_next(wk, prefix, ctxs, B, p.ng);
+    else have = false;
+  }
+  if (!aborted && cur_seg >= 0) finish_segment();
+  if (aborted) my_meta = make_int4(-1, 0, 0, T);
+  if (lane == 0) p.meta[u] = my_meta;
+}
+
+// ---------------------------------------------------------------------------
+// Merge: one warp per unit.  The unit that holds the first piece of a split
+// segment combines the pieces in unit order:
+//   M = max_i m_i,  w_i = 2^(m_i - M),  out = sum_i w_i O_i / sum_i w_i l_i
+// and every warp zero-fills the rows of its share of empty sequences.
+// ---------------------------------------------------------------------------
+struct MergeParams {
+  void* out;
+  const int32_t* context_lens;
+  const float* records;
+  const int4* meta;
+  int32_t batch;
+  int32_t n_q_heads;
+  int32_t gp;
+  int32_t ng;
+  int32_t num_units;
+  int32_t rec_floats;
+  int32_t max_ctx;
+};
+
+constexpr int kMergeWarps = 4;
+
+template <int DT, int D>
+__global__ void __launch_bounds__(kMergeWarps * 32) pkv_merge_kernel(const MergeParams p) {
+  using T = typename DTypeInfo<DT>::T;
+  constexpr int DPL = D / 32;  // dims per lane
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x * kMergeWarps + warp;
+  if (u >= p.num_units) return;
+  const int U = p.num_units;
+  const int4 mt = p.meta[u];
+  if (mt.x >= 0) {
+    const int seg = mt.x, b = seg / p.ng, hg = seg % p.ng, u_hi = mt.y, n_tiles = mt.w;
+    for (int g = 0; g < p.gp; ++g) {
+      float M = -INFINITY;
+      for (int v = u; v <= u_hi; ++v) {
+        if (v > u && unit_begin(v, n_tiles, U) == unit_begin(v + 1, n_tiles, U)) continue;  // empty unit
+        const float* rec = p.records + (static_cast<size_t>(v) * 2 + (v == u ? mt.z : 0)) * p.rec_floats;
+        M = fmaxf(M, rec[g]);
+      }
+      float L = 0.f, acc[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+      for (int v = u; v <= u_hi; ++v) {
+        if (v > u && unit_begin(v, n_tiles, U) == unit_begin(v + 1, n_tiles, U)) continue;
+        const float* rec = p.records + (static_cast<size_t>(v) * 2 + (v == u ? mt.z : 0)) * p.rec_floats;
+        const float w = exp2f(rec[g] - M);
+        L = fmaf(w, rec[p.gp + g], L);
+        const float* ro = rec + 2 * p.gp + g * D + lane * DPL;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, ro[i], acc[i]);
+      }
+      const float inv = 1.f / L;
+      T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
+      if constexpr (DT == kF32) {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) ob[i] = acc[i] * inv;
+      } else {
+#pragma unroll
+        for (int i = 0; i < DPL; i += 2)
+          *reinterpret_cast<uint32_t*>(ob + i) = pack2<DT == kBF16>(acc[i] * inv, acc[i + 1] * inv);
+      }
+    }
+  }
+  // Sequences with no tokens get a zero output row.
+  const int total = p.batch * p.ng;
+  for (int s = u; s < total; s += U) {
+    const int b = s / p.ng, hg = s % p.ng;
+    if (clamp_ctx(__ldg(p.context_lens + b), p.max_ctx) != 0) continue;
+    for (int g = 0; g < p.gp; ++g) {
+      T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) ob[i] = T(0.f);
+    }
+  }
+}
+
+}  // namespace pkv

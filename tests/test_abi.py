@@ -1,0 +1,116 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/pagedkv.h declares, and rejects bad arguments on the host before
+touching CUDA (no compute call is made here)."""
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import paged_kv_cache_386_b200 as pkv
+from paged_kv_cache_386_b200 import build as pkv_build
+
+HEADER = Path(__file__).resolve().parents[1] / "include" / "pagedkv.h"
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pkv_build.build()
+    return pkv._load()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_expected_entry_points():
+    names = set(declared_functions())
+    assert {"paged_kv_append", "paged_attention_decode", "paged_attention_decode_ex",
+            "paged_attention_workspace_size", "pkv_get_device_error", "pkv_status_string",
+            "pkv_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert pkv.pkv_status_string(s)
+    assert pkv.pkv_status_string(99) == "unknown status"
+    assert pkv.pkv_version() >= 10000
+
+
+def _decode(lib, **over):
+    args = dict(q=None, k=None, v=None, bt=None, maxb=4, cl=None, batch=2, nblocks=8, scale=0.125,
+                nq=8, nkv=2, d=128, bs=16, out=None, dtype=2, ws=None, wsb=0, stream=None)
+    args.update(over)
+    a = args
+    return lib.paged_attention_decode(a["q"], a["k"], a["v"], a["bt"], a["maxb"], a["cl"], a["batch"],
+                                      a["nblocks"], a["scale"], a["nq"], a["nkv"], a["d"], a["bs"],
+                                      a["out"], a["dtype"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_decode_host_validation(lib):
+    assert _decode(lib) == INVALID                      # null pointers
+    assert _decode(lib, nq=6, nkv=4) == INVALID          # n_q % n_kv != 0
+    assert _decode(lib, batch=-1) == INVALID
+    assert _decode(lib, nblocks=0) == INVALID
+    assert _decode(lib, scale=float("nan")) == INVALID
+    assert _decode(lib, d=96) == UNSUPPORTED
+    assert _decode(lib, bs=32) == UNSUPPORTED
+    assert _decode(lib, dtype=7) == UNSUPPORTED
+    assert _decode(lib, batch=4097) == UNSUPPORTED
+    assert _decode(lib, batch=0) == 0                    # nothing to do, nothing enqueued
+    # misaligned q (pointers are never dereferenced on the host)
+    assert _decode(lib, q=8, k=256, v=512, bt=1024, cl=2048, out=4096) == INVALID
+    # tile count beyond 32 bits
+    assert _decode(lib, q=256, k=256, v=256, bt=256, cl=256, out=256, batch=4096, maxb=1 << 20) == UNSUPPORTED
+
+
+def test_decode_ex_rejects_bad_options(lib):
+    opts = pkv._Options(num_units=-1)
+    st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
+                                       None, 0, None, ctypes.byref(opts))
+    assert st == INVALID
+    opts = pkv._Options()
+    opts.reserved[2] = 1
+    st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
+                                       None, 0, None, ctypes.byref(opts))
+    assert st == INVALID
+
+
+def test_append_host_validation(lib):
+    f = lib.paged_kv_append
+    assert f(None, None, None, -1, None, None, 8, 16, 2, 128, 2, None) == INVALID
+    assert f(None, None, None, 4, None, None, 8, 32, 2, 128, 2, None) == UNSUPPORTED
+    assert f(None, None, None, 4, None, None, 8, 16, 2, 128, 9, None) == UNSUPPORTED
+    assert f(None, None, None, 0, None, None, 8, 16, 2, 128, 2, None) == 0
+    assert f(None, None, None, 4, None, None, 8, 16, 2, 128, 2, None) == INVALID
+    assert f(16, 32, 4, 4, 64, 128, 8, 16, 2, 128, 2, None) == INVALID   # slot_mapping misaligned
+
+
+def test_workspace_size_validation(lib):
+    out = ctypes.c_size_t()
+    assert lib.paged_attention_workspace_size(4, 6, 4, 128, 2, ctypes.byref(out)) == INVALID
+    assert lib.paged_attention_workspace_size(4, 8, 2, 96, 2, ctypes.byref(out)) == UNSUPPORTED
+    assert lib.paged_attention_workspace_size(4, 8, 2, 128, 2, None) == INVALID
+
+
+def test_device_error_needs_flags(lib):
+    assert lib.pkv_get_device_error(None, None) == INVALID
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    t = torch.zeros(1, 8, 128, dtype=torch.bfloat16)
+    cache = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        pkv.paged_attention_decode(t, cache, cache, torch.zeros(1, 1, dtype=torch.int32),
+                                   torch.ones(1, dtype=torch.int32), 0.1, out=t.clone())
