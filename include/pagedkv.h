@@ -162,6 +162,43 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
                                      const pkv_decode_options* options);
 
 /*
+ * paged_attention_decode_noalloc -- paged_attention_decode for callers that
+ * cannot allocate device memory.  (The pages have no counterpart: this entry
+ * point is an addition of this library.)
+ *
+ * Some callers cannot call cudaMalloc or any allocator: a plugin whose host
+ * framework owns all device memory and hands it no allocator, a serving loop
+ * that must never allocate on its hot path (an allocation can synchronise the
+ * device and stall every stream), or a process that has already given all
+ * free memory to its KV-cache pool.  This entry point takes the same inputs
+ * and outputs as paged_attention_decode, minus the workspace, and allocates
+ * nothing: the scratch for split contexts lives in one file-scope device array
+ * of PKV_STATIC_WORKSPACE_BYTES (20 MiB), which every GPU that loads the
+ * library holds until the process exits.
+ *
+ * - Sizes whose scratch (paged_attention_workspace_size) exceeds the array are
+ *   rejected with PKV_ERR_WORKSPACE before anything is enqueued.  On a 148-SM
+ *   B200 every supported shape fits.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current and caches it; make that
+ *   first call before any stream capture.
+ * - Every call on a device shares the one array and it keeps the last call's
+ *   contents.  Nothing in it has to start at zero: each call rewrites the
+ *   per-unit metadata before its merge reads any record.  Calls whose work
+ *   overlaps on the GPU (on different streams, or from several host threads
+ *   without ordering) race on the array and give wrong results: order them.
+ * Results are bit-identical to paged_attention_decode with its default split.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (20u * 1024u * 1024u)
+
+pkv_status paged_attention_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                          const int32_t* context_lens, int32_t batch, int32_t num_blocks,
+                                          float scale, int32_t n_q_heads, int32_t n_kv_heads,
+                                          int32_t head_dim, int32_t block_size, void* out,
+                                          pkv_dtype dtype, void* stream);
+
+/*
  * pkv_get_device_error -- synchronise `stream`, then read and clear the
  * current device's error word.  *flags receives the PKV_DEVERR_* bits seen
  * since the last call.  Returns PKV_ERR_OUT_OF_RANGE if any bit was set,

@@ -22,7 +22,8 @@ from pathlib import Path
 import torch
 
 __all__ = [
-    "paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
+    "paged_kv_append", "paged_attention_decode", "paged_attention_decode_noalloc",
+    "paged_attention_workspace_size",
     "pkv_get_device_error", "pkv_status_string", "pkv_version", "PagedKVError", "library_path",
     "DEVERR_BLOCK_ID", "DEVERR_CONTEXT", "DEVERR_SLOT", "DEVERR_TIMEOUT",
 ]
@@ -72,6 +73,8 @@ def _load() -> ctypes.CDLL:
     lib.paged_attention_decode.restype = ctypes.c_int
     lib.paged_attention_decode_ex.argtypes = dec + [ctypes.POINTER(_Options)]
     lib.paged_attention_decode_ex.restype = ctypes.c_int
+    lib.paged_attention_decode_noalloc.argtypes = dec[:15] + [p]
+    lib.paged_attention_decode_noalloc.restype = ctypes.c_int
     lib.pkv_get_device_error.argtypes = [p, ctypes.POINTER(ctypes.c_uint32)]
     lib.pkv_get_device_error.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]
@@ -154,6 +157,28 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
         B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
         ws_ptr, ws_bytes, _stream(stream), ctypes.byref(opts)), "paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale: float, out=None,
+                                   block_size: int = 16, stream=None):
+    """paged_attention_decode for callers that cannot allocate device memory:
+    the split-context scratch is the library's static device array (shared by
+    every call on the device, so calls must not overlap on the GPU)."""
+    lib = _load()
+    B, n_q, d = q.shape
+    num_blocks, n_kv, bs, d2 = k_cache.shape
+    if d2 != d or bs != block_size or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.paged_attention_decode_noalloc(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+        B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
+        _stream(stream)), "paged_attention_decode_noalloc")
     return out
 
 

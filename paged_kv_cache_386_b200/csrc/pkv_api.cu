@@ -340,6 +340,53 @@ pkv_status paged_attention_decode(const void* q, const void* k_cache, const void
                                    workspace, workspace_bytes, stream, nullptr);
 }
 
+// ---------------------------------------------------------------------------
+// Decode without any allocation: the split-context scratch lives in a
+// file-scope device array instead of caller or library allocations.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_pkv_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
+
+namespace {
+std::mutex g_static_mutex;
+void* g_static_workspace_ptr[kMaxDevices] = {};
+
+// Device address of the static array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+pkv_status static_workspace(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (g_static_workspace_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_pkv_static_workspace) != cudaSuccess || ptr == nullptr) return PKV_ERR_CUDA;
+    g_static_workspace_ptr[dev] = ptr;
+  }
+  *out = g_static_workspace_ptr[dev];
+  return PKV_OK;
+}
+}  // namespace
+
+pkv_status paged_attention_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                          const int32_t* context_lens, int32_t batch, int32_t num_blocks,
+                                          float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                          int32_t block_size, void* out, pkv_dtype dtype, void* stream) {
+  pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
+                                    num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
+  if (st != PKV_OK || batch == 0) return st;
+  size_t need = 0;
+  st = paged_attention_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, dtype, &need);
+  if (st != PKV_OK) return st;
+  if (need > PKV_STATIC_WORKSPACE_BYTES) return PKV_ERR_WORKSPACE;  // beyond the static maximum
+  void* ws = nullptr;
+  st = static_workspace(&ws);
+  if (st != PKV_OK) return st;
+  return paged_attention_decode_ex(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
+                                   num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, ws,
+                                   PKV_STATIC_WORKSPACE_BYTES, stream, nullptr);
+}
+
 pkv_status pkv_get_device_error(void* stream, uint32_t* flags) {
   if (!flags) return PKV_ERR_INVALID_ARG;
   *flags = 0;
