@@ -76,6 +76,8 @@ int record_floats(int gp, int head_dim) { return (gp * (head_dim + 2) + 3) & ~3;
 
 size_t meta_bytes(int units) { return (static_cast<size_t>(units) * sizeof(int4) + 255) & ~static_cast<size_t>(255); }
 
+// Per work unit: one metadata entry and two partial-softmax records (its
+// first and last segment).
 size_t workspace_for(int units, int gp, int head_dim) {
   return meta_bytes(units) + static_cast<size_t>(units) * 2 * record_floats(gp, head_dim) * sizeof(float);
 }
@@ -129,20 +131,35 @@ pkv_status encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dt, i
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// The decode kernel is launched cooperatively: its CTAs (at most one per SM)
+// are guaranteed to be co-resident, which its grid-wide barrier needs.
 template <int DT, int D, int GPAD>
 pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid, size_t smem,
                          cudaStream_t stream) {
   auto kern = pkv_decode_kernel<DT, D, GPAD>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-    return PKV_ERR_CUDA;
-  kern<<<grid, kDecodeThreads, smem, stream>>>(mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
-}
-
-template <int DT, int D>
-pkv_status launch_merge(const MergeParams& mp, cudaStream_t stream) {
-  const int grid = (mp.num_units + kMergeWarps - 1) / kMergeWarps;
-  pkv_merge_kernel<DT, D><<<grid, kMergeWarps * 32, 0, stream>>>(mp);
+  // Opt in to the largest dynamic shared memory once per device (the launch
+  // itself passes the size it needs).
+  static bool opted_in[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  if (!opted_in[dev]) {
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - 256) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    opted_in[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mk, mv, p) != cudaSuccess) return PKV_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -162,11 +179,9 @@ pkv_status dispatch_gpad(int gpad, const CUtensorMap& mk, const CUtensorMap& mv,
 
 template <int DT>
 pkv_status dispatch_dim(int head_dim, int gpad, const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p,
-                        const MergeParams& mp, int grid, size_t smem, cudaStream_t stream) {
-  pkv_status st = head_dim == 64 ? dispatch_gpad<DT, 64>(gpad, mk, mv, p, grid, smem, stream)
-                                 : dispatch_gpad<DT, 128>(gpad, mk, mv, p, grid, smem, stream);
-  if (st != PKV_OK) return st;
-  return head_dim == 64 ? launch_merge<DT, 64>(mp, stream) : launch_merge<DT, 128>(mp, stream);
+                        int grid, size_t smem, cudaStream_t stream) {
+  return head_dim == 64 ? dispatch_gpad<DT, 64>(gpad, mk, mv, p, grid, smem, stream)
+                        : dispatch_gpad<DT, 128>(gpad, mk, mv, p, grid, smem, stream);
 }
 
 }  // namespace
@@ -256,8 +271,10 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
   const int group = n_q_heads / n_kv_heads;
   const int gp = heads_per_segment(group, dtype, opt.force_simt == 1);
   const int gpad = gp == 1 ? 0 : (gp <= 8 ? 8 : 16);
+  // One CTA per SM at most (the kernel's grid barrier needs every CTA
+  // resident), so the unit count is capped at 8 per SM.
   const int default_units = di.sm_count * kConsumerWarps;
-  const int units = opt.num_units > 0 ? opt.num_units : default_units;
+  const int units = (opt.num_units > 0 && opt.num_units < default_units) ? opt.num_units : default_units;
   const int grid = (units + kConsumerWarps - 1) / kConsumerWarps;
 
   // Ring depth: as many 8-slot rounds as shared memory allows (at most 4).
@@ -265,7 +282,9 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
   const size_t stage_bytes = static_cast<size_t>(2) * (head_dim * es / 128) * kBoxBytes;
   // 1 KiB alignment slack, abort word, prefix sums and clamped lengths, and
   // 256 bytes for the kernel's static shared memory.
-  const size_t fixed = 1024 + 16 + static_cast<size_t>(2 * batch + 1) * sizeof(int) + 256;
+  const size_t qbuf_bytes = static_cast<size_t>(gpad == 0 ? 1 : gpad) * head_dim * es;
+  const size_t fixed =
+      1024 + kConsumerWarps * qbuf_bytes + 16 + static_cast<size_t>(2 * batch + 1) * sizeof(int) + 256;
   const size_t per_round = kConsumerWarps * (stage_bytes + 2 * sizeof(uint64_t));
   if (fixed + per_round > static_cast<size_t>(di.smem_optin)) return PKV_ERR_UNSUPPORTED;
   int stages = static_cast<int>((di.smem_optin - fixed) / per_round);
@@ -303,26 +322,14 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
   p.num_units = units;
   p.stages = stages;
   p.rec_floats = record_floats(gp, head_dim);
+  p.head_dim = head_dim;
   p.scale_log2 = scale * 1.4426950408889634f;
-
-  MergeParams mp;
-  mp.out = out;
-  mp.context_lens = context_lens;
-  mp.records = p.records;
-  mp.meta = p.meta;
-  mp.batch = batch;
-  mp.n_q_heads = n_q_heads;
-  mp.gp = gp;
-  mp.ng = p.ng;
-  mp.num_units = units;
-  mp.rec_floats = p.rec_floats;
-  mp.max_ctx = max_blocks_per_seq * kBlockTokens;
 
   if (st == PKV_OK) {
     switch (dtype) {
-      case PKV_F32: st = dispatch_dim<kF32>(head_dim, gpad, mk, mv, p, mp, grid, smem, s); break;
-      case PKV_F16: st = dispatch_dim<kF16>(head_dim, gpad, mk, mv, p, mp, grid, smem, s); break;
-      default: st = dispatch_dim<kBF16>(head_dim, gpad, mk, mv, p, mp, grid, smem, s); break;
+      case PKV_F32: st = dispatch_dim<kF32>(head_dim, gpad, mk, mv, p, grid, smem, s); break;
+      case PKV_F16: st = dispatch_dim<kF16>(head_dim, gpad, mk, mv, p, grid, smem, s); break;
+      default: st = dispatch_dim<kBF16>(head_dim, gpad, mk, mv, p, grid, smem, s); break;
     }
   }
   if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == PKV_OK) st = PKV_ERR_CUDA;

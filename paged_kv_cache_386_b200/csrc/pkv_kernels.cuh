@@ -1,7 +1,8 @@
 // pkv_kernels.cuh -- sm_100a kernels of the paged KV cache:
 //   pkv_append_kernel   scatter of new K/V rows into their slots
-//   pkv_decode_kernel   persistent split-KV paged decode attention
-//   pkv_merge_kernel    log-sum-exp merge of split contexts
+//   pkv_decode_kernel   persistent split-KV paged decode attention, with the
+//                       log-sum-exp merge of split contexts after a grid-wide
+//                       barrier
 //
 // Decode design (one launch for every sequence, head group and context split):
 //
@@ -13,7 +14,8 @@
 //   contiguous ranges (stream-K style).  A unit is one consumer warp, so every
 //   warp gets the same number of tiles whatever the length mix; a segment that
 //   straddles unit boundaries is a split context whose partial softmax states
-//   are merged by pkv_merge_kernel.
+//   are merged, after a grid-wide barrier of the cooperative launch, by the
+//   unit that holds its first piece.
 // * Each CTA runs 8 consumer warps (units) and one producer warp.  Lane w of
 //   the producer walks unit w's tiles, reads the physical block id from the
 //   block table one tile ahead and issues TMA tensor loads of the K and V tile
@@ -35,6 +37,7 @@
 //   under any block placement and with shared or private prefix blocks.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -114,8 +117,8 @@ struct DecodeParams {
   void* out;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  float* records;  // [num_units][2][rec_floats]
-  int4* meta;      // [num_units]
+  float* records;  // [num_units][2][rec_floats]: O[gp][D], m[gp], l[gp]
+  int4* meta;      // [num_units]: split segment whose first piece the unit holds
   int32_t max_blocks_per_seq;
   int32_t batch;
   int32_t num_blocks;
@@ -126,6 +129,7 @@ struct DecodeParams {
   int32_t num_units;
   int32_t stages;      // ring slots per consumer warp
   int32_t rec_floats;  // floats per partial record: gp * (head_dim + 2), rounded up to 4
+  int32_t head_dim;
   float scale_log2;    // scale * log2(e)
 };
 
@@ -204,18 +208,19 @@ struct MmaConsumer {
   float o[NT][4];
   float m[2], l[2];
 
-  __device__ __forceinline__ void begin(const DecodeParams& p, int b, int hg, int lane) {
+  // Q of the segment's gp heads from the warp's shared buffer ([gp][D]).
+  __device__ __forceinline__ void begin(const uint8_t* qbuf, int gp, int lane) {
     const int g = lane >> 2, t = lane & 3;
-    const T* qb = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp) * D;
-    const bool r0 = g < p.gp;
-    const bool r1 = (GPAD == 16) && (g + 8 < p.gp);
+    const T* qb = reinterpret_cast<const T*>(qbuf);
+    const bool r0 = g < gp;
+    const bool r1 = (GPAD == 16) && (g + 8 < gp);
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       const int c = ks * 16 + 2 * t;
-      qa[ks][0] = r0 ? __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + c)) : 0u;
-      qa[ks][2] = r0 ? __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + c + 8)) : 0u;
-      qa[ks][1] = r1 ? __ldg(reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + c)) : 0u;
-      qa[ks][3] = r1 ? __ldg(reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + c + 8)) : 0u;
+      qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t*>(qb + g * D + c) : 0u;
+      qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t*>(qb + g * D + c + 8) : 0u;
+      qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + c) : 0u;
+      qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + c + 8) : 0u;
     }
 #pragma unroll
     for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -363,10 +368,10 @@ struct MmaConsumer {
         }
       } else {
         if (t == 0) {
-          rec[row] = m[r];
-          rec[p.gp + row] = lt[r];
+          rec[p.gp * D + row] = m[r];
+          rec[p.gp * D + p.gp + row] = lt[r];
         }
-        float* ro = rec + 2 * p.gp + row * D;
+        float* ro = rec + row * D;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           float a0, a1;
@@ -413,14 +418,13 @@ struct SimtConsumer {
     }
   }
 
-  __device__ __forceinline__ void begin(const DecodeParams& p, int b, int hg, int lane) {
+  // This lane's dim slice of the segment's one query head, from the warp's
+  // shared buffer.
+  __device__ __forceinline__ void begin(const uint8_t* qbuf, int /*gp*/, int lane) {
     const int sub = lane >> 3;
-    const T* qb = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.n_q_heads + hg) * D + sub * DL;
+    const uint4* qb = reinterpret_cast<const uint4*>(qbuf + sub * DL * ES);
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qb) + c);
-      widen16(raw, qs + c * EPC);
-    }
+    for (int c = 0; c < NCH; ++c) widen16(qb[c], qs + c * EPC);
 #pragma unroll
     for (int i = 0; i < DL; ++i) o[i] = 0.f;
     m = -INFINITY;
@@ -530,11 +534,11 @@ struct SimtConsumer {
       }
     } else {
       if (lane == 0) {
-        rec[0] = m;
-        rec[1] = lt;
+        rec[D] = m;
+        rec[D + 1] = lt;
       }
 #pragma unroll
-      for (int i = 0; i < DO; ++i) rec[2 + d0 + i] = o[i];
+      for (int i = 0; i < DO; ++i) rec[d0 + i] = o[i];
     }
   }
 };
@@ -548,7 +552,114 @@ struct ConsumerFor<DT, D, 0> {
   using type = SimtConsumer<DT, D>;
 };
 
+// Four fp32 values rounded to the output dtype and stored together.
+template <int DT>
+__device__ __forceinline__ void store4(typename DTypeInfo<DT>::T* dst, float a, float b, float c, float d) {
+  if constexpr (DT == kF32) {
+    *reinterpret_cast<float4*>(dst) = make_float4(a, b, c, d);
+  } else {
+    uint2 v;
+    v.x = pack2<DT == kBF16>(a, b);
+    v.y = pack2<DT == kBF16>(c, d);
+    *reinterpret_cast<uint2*>(dst) = v;
+  }
+}
+
+// Copy the gp x head_dim Q rows of segment (b, hg) into a warp's shared
+// buffer with 16-byte cp.async (completion: cp_async_wait_all + __syncwarp).
+template <int ES, int D>
+__device__ __forceinline__ void q_fetch(uint8_t* qbuf, const void* q, int n_q_heads, int b, int hg, int gp,
+                                        int lane) {
+  const uint8_t* src =
+      static_cast<const uint8_t*>(q) + (static_cast<size_t>(b) * n_q_heads + static_cast<size_t>(hg) * gp) * D * ES;
+  const int chunks = gp * D * ES / 16;
+  for (int c = lane; c < chunks; c += 32) cp_async_16(qbuf + c * 16, src + c * 16);
+  cp_async_commit();
+}
+
+// Phase 2 of the decode kernel: one warp merges query head g of the split
+// segment whose first piece unit u holds (mt = meta[u]); the pieces are held
+// by units u..u_hi (units are never empty: their count is capped at the tile
+// count) and are combined in unit order as
+//   M = max_i m_i,  w_i = 2^(m_i - M),  out = sum_i w_i O_i / sum_i w_i l_i.
+// Lane j holds the scalars of pieces j and j + 32; each lane owns D/32 dims
+// of the numerator and walks the pieces eight loads at a time, the weights
+// broadcast by shuffles.  Reads go to L2 (ld.global.cg): the records were
+// written by other SMs before the grid barrier.
+template <int DT, int D>
+__device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt, int g, int lane) {
+  using T = typename DTypeInfo<DT>::T;
+  constexpr int DPL = D / 32;
+  const int seg = mt.x, b = seg / p.ng, hg = seg % p.ng, n = mt.y - u + 1;
+  const int mo = p.gp * D + g, lo = p.gp * D + p.gp + g, oo = g * D + lane * DPL;
+  auto rec_of = [&](int j) -> const float* {  // record of piece j (unit u + j)
+    return p.records + (static_cast<size_t>(u + j) * 2 + (j == 0 ? mt.z : 0)) * p.rec_floats;
+  };
+  // Scalars of pieces lane and lane + 32; pieces beyond 64 (rare) are folded
+  // in by a plain loop.
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  if (lane < n) {
+    m0 = __ldcg(rec_of(lane) + mo);
+    l0 = __ldcg(rec_of(lane) + lo);
+  }
+  if (lane + 32 < n) {
+    m1 = __ldcg(rec_of(lane + 32) + mo);
+    l1 = __ldcg(rec_of(lane + 32) + lo);
+  }
+  float M = fmaxf(m0, m1);
+  for (int j = 64 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(rec_of(j) + mo));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float w0 = exp2f(m0 - M), w1 = exp2f(m1 - M);
+  float L = w0 * l0 + w1 * l1;
+  for (int j = 64 + lane; j < n; j += 32) L = fmaf(exp2f(__ldcg(rec_of(j) + mo) - M), __ldcg(rec_of(j) + lo), L);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+
+  float acc[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+  for (int j0 = 0; j0 < n; j0 += 8) {
+    float o[8][DPL];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = min(j0 + jj, n - 1);
+      const float* r = rec_of(j) + oo;
+      if constexpr (DPL == 4) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(r));
+        o[jj][0] = x.x; o[jj][1] = x.y; o[jj][2] = x.z; o[jj][3] = x.w;
+      } else {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(r));
+        o[jj][0] = x.x; o[jj][1] = x.y;
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = j0 + jj;
+      float wj = __shfl_sync(0xffffffffu, (j & 32) ? w1 : w0, j & 31);
+      if (j >= 64 && j < n) wj = exp2f(__ldcg(rec_of(j) + mo) - M);
+      if (j >= n) wj = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wj, o[jj][i], acc[i]);
+    }
+  }
+  const float inv = 1.f / L;
+  T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
+  if constexpr (DPL == 4) {
+    store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  } else if constexpr (DT == kF32) {
+    *reinterpret_cast<float2*>(ob) = make_float2(acc[0] * inv, acc[1] * inv);
+  } else {
+    *reinterpret_cast<uint32_t*>(ob) = pack2<DT == kBF16>(acc[0] * inv, acc[1] * inv);
+  }
+}
+
 // GPAD: 0 = CUDA-core consumer (gp == 1); 8 or 16 = tensor-core consumer.
+//
+// Launched cooperatively (all CTAs co-resident, one per SM): phase 1 runs the
+// producer/consumer pipeline; a grid-wide barrier follows (every wait before
+// it is bounded, so every thread reaches it); phase 2 merges split segments
+// and zero-fills the rows of empty sequences.
 template <int DT, int D, int GPAD>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     pkv_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -558,13 +669,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   constexpr int Y = D / X;                         // boxes per tile
   constexpr int kTileBytes = Y * kBoxBytes;
   constexpr int kStageBytes = 2 * kTileBytes;
+  constexpr int kQBufBytes = (GPAD == 0 ? 1 : GPAD) * D * ES;
   using Consumer = typename ConsumerFor<DT, D, GPAD>::type;
+  using OutT = typename DTypeInfo<DT>::T;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const int n_slots = kConsumerWarps * p.stages;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(ring + static_cast<size_t>(n_slots) * kStageBytes);
+  uint8_t* qbufs = ring + static_cast<size_t>(n_slots) * kStageBytes;  // [warps][kQBufBytes]
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(qbufs + kConsumerWarps * kQBufBytes);
   uint64_t* empty_bar = full_bar + n_slots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty_bar + n_slots);
   int* prefix = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 4));  // [batch + 1]
@@ -582,6 +696,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     *abort_flag = 0;
     mbar_fence_init();
+    // Bring this CTA's slice of q into L2 ahead of the consumers' copies.
+    const size_t q_bytes = static_cast<size_t>(B) * p.n_q_heads * D * ES;
+    const size_t slice = ((q_bytes / gridDim.x) + 15) & ~static_cast<size_t>(15);
+    const size_t off = slice * blockIdx.x;
+    if (slice > 0 && off < q_bytes) {
+      const size_t n = q_bytes - off < slice ? q_bytes - off : slice;
+      bulk_prefetch_l2(static_cast<const uint8_t*>(p.q) + off, static_cast<uint32_t>(n));
+    }
   }
   if (warp == kConsumerWarps && lane == 0) {
     tma_prefetch_desc(&tm_k);
@@ -620,14 +742,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __syncthreads();
 
   const int T = prefix[B];
-  const int U = p.num_units;
+  // At most one unit per tile, so that no unit is empty.
+  const int U = min(p.num_units, max(T, 1));
+  int4 my_meta = make_int4(-1, 0, 0, T);  // consumer warps: split segment this unit merges
 
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
+    // Lane w feeds unit w.  Lanes never wait for each other: each polls its
+    // own next ring slot (non-blocking test of the empty barrier) and issues
+    // the TMA loads when the slot is free.  The physical block ids of a lane's
+    // next two tiles are kept in registers, loaded two tiles ahead.
     const int u = blockIdx.x * kConsumerWarps + lane;
-    Walk wk;
-    bool active = false;
-    if (lane < kConsumerWarps && u < U) active = walk_begin(wk, prefix, ctxs, B, unit_begin(u, T, U), unit_begin(u + 1, T, U));
+    int pending = 0;
+    Walk wn;
+    if (lane < kConsumerWarps && u < U) {
+      const int k0 = unit_begin(u, T, U), k1 = unit_begin(u + 1, T, U);
+      if (walk_begin(wn, prefix, ctxs, B, k0, k1)) pending = k1 - k0;
+    }
     auto load_phys = [&](const Walk& w) -> int {
       int ph = __ldg(p.block_tables + static_cast<size_t>(w.b) * p.max_blocks_per_seq + w.j);
       if (ph < 0 || ph >= p.num_blocks) {
@@ -636,35 +767,66 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       return ph;
     };
-    int next_phys = active ? load_phys(wk) : 0;
+    auto advance = [&](Walk& w) {
+      if (w.k + 1 < w.k_end) walk_next(w, prefix, ctxs, B, p.ng);
+      else w.k = w.k_end;
+    };
+    int q0_phys = 0, q0_kvh = 0, q1_phys = 0, q1_kvh = 0;
+    if (pending > 0) {
+      q0_phys = load_phys(wn);
+      q0_kvh = (wn.hg * p.gp) / p.group;
+      advance(wn);
+      if (wn.k < wn.k_end) {
+        q1_phys = load_phys(wn);
+        q1_kvh = (wn.hg * p.gp) / p.group;
+        advance(wn);
+      }
+    }
     int stage = 0, issued = 0;
     uint32_t phase = 0;
-    while (__any_sync(0xffffffffu, active)) {
-      if (active) {
-        const int phys = next_phys;
-        const int kvh = (wk.hg * p.gp) / p.group;
-        const bool more = wk.k + 1 < wk.k_end;
-        if (more) {
-          walk_next(wk, prefix, ctxs, B, p.ng);
-          next_phys = load_phys(wk);
-        }
+    uint64_t idle_since = 0;
+    while (__any_sync(0xffffffffu, pending > 0)) {
+      bool progressed = false;
+      if (pending > 0) {
         const int slot = lane * p.stages + stage;
-        if (!mbar_wait_bounded(&empty_bar[slot], phase ^ 1u, abort_flag, kWaitLimitNs)) {
-          active = false;
-        } else {
+        if (mbar_test_wait(&empty_bar[slot], phase ^ 1u)) {
           mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
           uint8_t* sk = ring + static_cast<size_t>(slot) * kStageBytes;
 #pragma unroll
-          for (int y = 0; y < Y; ++y) tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, kvh, phys);
+          for (int y = 0; y < Y; ++y)
+            tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, q0_kvh, q0_phys);
 #pragma unroll
           for (int y = 0; y < Y; ++y)
-            tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, kvh, phys);
+            tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, q0_kvh, q0_phys);
           ++issued;
+          --pending;
           if (++stage == p.stages) {
             stage = 0;
             phase ^= 1u;
           }
-          active = more;
+          q0_phys = q1_phys;
+          q0_kvh = q1_kvh;
+          if (wn.k < wn.k_end) {
+            q1_phys = load_phys(wn);
+            q1_kvh = (wn.hg * p.gp) / p.group;
+            advance(wn);
+          }
+          progressed = true;
+        }
+      }
+      // Bounded: give up (warp-uniformly) after kWaitLimitNs without progress.
+      if (__any_sync(0xffffffffu, progressed)) {
+        idle_since = 0;
+      } else {
+        const uint64_t now = global_timer_ns();
+        if (idle_since == 0) idle_since = now;
+        const bool give_up = __shfl_sync(0xffffffffu, (*abort_flag != 0) || (now - idle_since > kWaitLimitNs), 0);
+        if (give_up) {
+          if (lane == 0 && *abort_flag == 0) {
+            *abort_flag = 1;
+            flag_error(kDevErrTimeout);
+          }
+          break;
         }
       }
     }
@@ -682,140 +844,115 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
       }
     }
-    return;
+  } else {
+    // ---------------- consumers ----------------
+    const int u = blockIdx.x * kConsumerWarps + warp;
+    if (u < U) {
+      uint8_t* qbuf = qbufs + warp * kQBufBytes;
+      const int k0 = unit_begin(u, T, U), k1 = unit_begin(u + 1, T, U);
+      Walk wk;
+      bool have = walk_begin(wk, prefix, ctxs, B, k0, k1);
+      Consumer cs;
+      int first_seg = -1, cur_seg = -1, cur_b = 0, cur_hg = 0, seg_start = 0, seg_end = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool aborted = false;
+      bool q_ready = false;  // qbuf holds the next segment's Q (copy in flight)
+
+      auto finish_segment = [&]() {
+        const bool starts_here = seg_start >= k0, ends_here = seg_end <= k1;
+        if (starts_here && ends_here) {
+          cs.finish(p, cur_b, cur_hg, nullptr, lane);
+        } else {
+          const int slot_idx = (cur_seg == first_seg) ? 0 : 1;
+          float* rec = p.records + (static_cast<size_t>(u) * 2 + slot_idx) * p.rec_floats;
+          cs.finish(p, cur_b, cur_hg, rec, lane);
+          if (starts_here) my_meta = make_int4(cur_seg, unit_of_tile(seg_end - 1, T, U), slot_idx, T);
+        }
+      };
+
+      while (have) {
+        const int seg = wk.b * p.ng + wk.hg;
+        if (seg != cur_seg) {
+          if (cur_seg >= 0) finish_segment();
+          cur_seg = seg;
+          if (first_seg < 0) first_seg = seg;
+          cur_b = wk.b;
+          cur_hg = wk.hg;
+          seg_start = prefix[wk.b] + wk.hg * wk.nb;
+          seg_end = seg_start + wk.nb;
+          if (!q_ready) q_fetch<ES, D>(qbuf, p.q, p.n_q_heads, wk.b, wk.hg, p.gp, lane);
+          cp_async_wait_all();
+          __syncwarp();
+          cs.begin(qbuf, p.gp, lane);
+          __syncwarp();
+          q_ready = false;
+        }
+        // The last tile of a segment, with more tiles to come: start copying
+        // the next segment's Q now, so that it is in place when it is needed.
+        if (wk.j == wk.nb - 1 && wk.k + 1 < wk.k_end) {
+          Walk nx = wk;
+          walk_next(nx, prefix, ctxs, B, p.ng);
+          q_fetch<ES, D>(qbuf, p.q, p.n_q_heads, nx.b, nx.hg, p.gp, lane);
+          q_ready = true;
+        }
+        const int slot = warp * p.stages + stage;
+        if (!mbar_wait_bounded(&full_bar[slot], phase, abort_flag, kWaitLimitNs)) {
+          aborted = true;
+          break;
+        }
+        const int nv = min(kBlockTokens, wk.ctx - wk.j * kBlockTokens);
+        cs.tile(smem_u32(ring + static_cast<size_t>(slot) * kStageBytes), nv, p.scale_log2, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[slot]);
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (wk.k + 1 < wk.k_end) walk_next(wk, prefix, ctxs, B, p.ng);
+        else have = false;
+      }
+      cp_async_wait_all();
+      if (!aborted && cur_seg >= 0) finish_segment();
+      if (aborted) my_meta = make_int4(-1, 0, 0, T);
+      if (lane == 0) p.meta[u] = my_meta;
+    }
   }
 
-  // ---------------- consumers ----------------
-  const int u = blockIdx.x * kConsumerWarps + warp;
-  if (u >= U) return;
-  const int k0 = unit_begin(u, T, U), k1 = unit_begin(u + 1, T, U);
-  Walk wk;
-  bool have = walk_begin(wk, prefix, ctxs, B, k0, k1);
-  int4 my_meta = make_int4(-1, 0, 0, T);
-  Consumer cs;
-  int first_seg = -1, cur_seg = -1, cur_b = 0, cur_hg = 0, seg_start = 0, seg_end = 0;
-  int stage = 0;
-  uint32_t phase = 0;
-  bool aborted = false;
-
-  auto finish_segment = [&]() {
-    const bool starts_here = seg_start >= k0, ends_here = seg_end <= k1;
-    if (starts_here && ends_here) {
-      cs.finish(p, cur_b, cur_hg, nullptr, lane);
-    } else {
-      const int slot_idx = (cur_seg == first_seg) ? 0 : 1;
-      float* rec = p.records + (static_cast<size_t>(u) * 2 + slot_idx) * p.rec_floats;
-      cs.finish(p, cur_b, cur_hg, rec, lane);
-      if (starts_here) my_meta = make_int4(cur_seg, unit_of_tile(seg_end - 1, T, U), slot_idx, T);
+  // ---------------- phase 2: merge split segments ----------------
+  // Every warp of the grid takes (unit, query head) items; the items of units
+  // that hold the first piece of a split segment merge that head.
+  cooperative_groups::this_grid().sync();
+  {
+    constexpr int kWarps = kConsumerWarps + 1;
+    const int gw = blockIdx.x * kWarps + warp, n_warps = gridDim.x * kWarps;
+    const int items = U * p.gp;
+    // At most 32 items per warp (U <= 8 per CTA and gp <= 16): load their
+    // metadata in one round, lane t for the warp's t-th item.
+    int4 my_item = make_int4(-1, 0, 0, 0);
+    {
+      const int i = gw + lane * n_warps;
+      if (i < items) my_item = __ldcg(p.meta + i / p.gp);
     }
-  };
-
-  while (have) {
-    const int seg = wk.b * p.ng + wk.hg;
-    if (seg != cur_seg) {
-      if (cur_seg >= 0) finish_segment();
-      cur_seg = seg;
-      if (first_seg < 0) first_seg = seg;
-      cur_b = wk.b;
-      cur_hg = wk.hg;
-      seg_start = prefix[wk.b] + wk.hg * wk.nb;
-      seg_end = seg_start + wk.nb;
-      cs.begin(p, wk.b, wk.hg, lane);
+    for (int t = 0; gw + t * n_warps < items; ++t) {
+      const int i = gw + t * n_warps;
+      int4 mt;
+      mt.x = __shfl_sync(0xffffffffu, my_item.x, t);
+      mt.y = __shfl_sync(0xffffffffu, my_item.y, t);
+      mt.z = __shfl_sync(0xffffffffu, my_item.z, t);
+      mt.w = __shfl_sync(0xffffffffu, my_item.w, t);
+      if (mt.x >= 0) merge_head<DT, D>(p, i / p.gp, mt, i % p.gp, lane);
     }
-    const int slot = warp * p.stages + stage;
-    if (!mbar_wait_bounded(&full_bar[slot], phase, abort_flag, kWaitLimitNs)) {
-      aborted = true;
-      break;
-    }
-    const int nv = min(kBlockTokens, wk.ctx - wk.j * kBlockTokens);
-    cs.tile(smem_u32(ring + static_cast<size_t>(slot) * kStageBytes), nv, p.scale_log2, lane);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[slot]);
-    if (++stage == p.stages) {
-      stage = 0;
-      phase ^= 1u;
-    }
-    if (wk.k + 1 < wk.k_end) walk_next(wk, prefix, ctxs, B, p.ng);
-    else have = false;
-  }
-  if (!aborted && cur_seg >= 0) finish_segment();
-  if (aborted) my_meta = make_int4(-1, 0, 0, T);
-  if (lane == 0) p.meta[u] = my_meta;
-}
-
-// ---------------------------------------------------------------------------
-// Merge: one warp per unit.  The unit that holds the first piece of a split
-// segment combines the pieces in unit order:
-//   M = max_i m_i,  w_i = 2^(m_i - M),  out = sum_i w_i O_i / sum_i w_i l_i
-// and every warp zero-fills the rows of its share of empty sequences.
-// ---------------------------------------------------------------------------
-struct MergeParams {
-  void* out;
-  const int32_t* context_lens;
-  const float* records;
-  const int4* meta;
-  int32_t batch;
-  int32_t n_q_heads;
-  int32_t gp;
-  int32_t ng;
-  int32_t num_units;
-  int32_t rec_floats;
-  int32_t max_ctx;
-};
-
-constexpr int kMergeWarps = 4;
-
-template <int DT, int D>
-__global__ void __launch_bounds__(kMergeWarps * 32) pkv_merge_kernel(const MergeParams p) {
-  using T = typename DTypeInfo<DT>::T;
-  constexpr int DPL = D / 32;  // dims per lane
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = blockIdx.x * kMergeWarps + warp;
-  if (u >= p.num_units) return;
-  const int U = p.num_units;
-  const int4 mt = p.meta[u];
-  if (mt.x >= 0) {
-    const int seg = mt.x, b = seg / p.ng, hg = seg % p.ng, u_hi = mt.y, n_tiles = mt.w;
-    for (int g = 0; g < p.gp; ++g) {
-      float M = -INFINITY;
-      for (int v = u; v <= u_hi; ++v) {
-        if (v > u && unit_begin(v, n_tiles, U) == unit_begin(v + 1, n_tiles, U)) continue;  // empty unit
-        const float* rec = p.records + (static_cast<size_t>(v) * 2 + (v == u ? mt.z : 0)) * p.rec_floats;
-        M = fmaxf(M, rec[g]);
+    // Sequences with no tokens get a zero output row.
+    const int total = B * p.ng;
+    for (int sgi = gw; sgi < total; sgi += n_warps) {
+      const int b = sgi / p.ng, hg = sgi % p.ng;
+      if (ctxs[b] != 0) continue;
+      for (int e = lane; e < p.gp * (D / 4); e += 32) {
+        const int g = e / (D / 4), d4 = (e % (D / 4)) * 4;
+        store4<DT>(static_cast<OutT*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + d4,
+                   0.f, 0.f, 0.f, 0.f);
       }
-      float L = 0.f, acc[DPL];
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-      for (int v = u; v <= u_hi; ++v) {
-        if (v > u && unit_begin(v, n_tiles, U) == unit_begin(v + 1, n_tiles, U)) continue;
-        const float* rec = p.records + (static_cast<size_t>(v) * 2 + (v == u ? mt.z : 0)) * p.rec_floats;
-        const float w = exp2f(rec[g] - M);
-        L = fmaf(w, rec[p.gp + g], L);
-        const float* ro = rec + 2 * p.gp + g * D + lane * DPL;
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, ro[i], acc[i]);
-      }
-      const float inv = 1.f / L;
-      T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
-      if constexpr (DT == kF32) {
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) ob[i] = acc[i] * inv;
-      } else {
-#pragma unroll
-        for (int i = 0; i < DPL; i += 2)
-          *reinterpret_cast<uint32_t*>(ob + i) = pack2<DT == kBF16>(acc[i] * inv, acc[i + 1] * inv);
-      }
-    }
-  }
-  // Sequences with no tokens get a zero output row.
-  const int total = p.batch * p.ng;
-  for (int s = u; s < total; s += U) {
-    const int b = s / p.ng, hg = s % p.ng;
-    if (clamp_ctx(__ldg(p.context_lens + b), p.max_ctx) != 0) continue;
-    for (int g = 0; g < p.gp; ++g) {
-      T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) ob[i] = T(0.f);
     }
   }
 }
