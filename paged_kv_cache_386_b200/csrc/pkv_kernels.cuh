@@ -565,6 +565,17 @@ __device__ __forceinline__ void store4(typename DTypeInfo<DT>::T* dst, float a, 
   }
 }
 
+// Prefetch this CTA's 1/gridDim share of a buffer of `bytes` (a multiple of
+// 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void prefetch_slice_l2(const void* base, size_t bytes) {
+  const size_t slice = ((bytes / gridDim.x) + 15) & ~static_cast<size_t>(15);
+  const size_t off = slice * blockIdx.x;
+  if (slice > 0 && off < bytes) {
+    const size_t n = bytes - off < slice ? bytes - off : slice;
+    bulk_prefetch_l2(static_cast<const uint8_t*>(base) + off, static_cast<uint32_t>(n));
+  }
+}
+
 // Copy the gp x head_dim Q rows of segment (b, hg) into a warp's shared
 // buffer with 16-byte cp.async (completion: cp_async_wait_all + __syncwarp).
 template <int ES, int D>
@@ -696,14 +707,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     *abort_flag = 0;
     mbar_fence_init();
-    // Bring this CTA's slice of q into L2 ahead of the consumers' copies.
-    const size_t q_bytes = static_cast<size_t>(B) * p.n_q_heads * D * ES;
-    const size_t slice = ((q_bytes / gridDim.x) + 15) & ~static_cast<size_t>(15);
-    const size_t off = slice * blockIdx.x;
-    if (slice > 0 && off < q_bytes) {
-      const size_t n = q_bytes - off < slice ? q_bytes - off : slice;
-      bulk_prefetch_l2(static_cast<const uint8_t*>(p.q) + off, static_cast<uint32_t>(n));
-    }
+    // Bring this CTA's slices of q and of the block table into L2: the
+    // consumers' Q copies and the producers' block-id loads then hit L2.
+    prefetch_slice_l2(p.q, static_cast<size_t>(B) * p.n_q_heads * D * ES);
+    if ((reinterpret_cast<uintptr_t>(p.block_tables) & 15u) == 0)
+      prefetch_slice_l2(p.block_tables, static_cast<size_t>(B) * p.max_blocks_per_seq * sizeof(int32_t) & ~size_t(15));
   }
   if (warp == kConsumerWarps && lane == 0) {
     tma_prefetch_desc(&tm_k);
