@@ -85,7 +85,8 @@ class ClockSampler:
     millisecond in a background thread during the timed region (read-only
     queries; no GPU setting is changed)."""
 
-    def __init__(self, device: torch.device, period_s: float = 0.001):
+    def __init__(self, device: torch.device, period_s: float = 0.01, enabled: bool = True):
+        self.enabled = enabled
         self.device = device
         self.period = period_s
         self.samples: list[tuple[int, int, int]] = []
@@ -112,6 +113,10 @@ class ClockSampler:
     def __enter__(self):
         import threading
         self._stop = threading.Event()
+        if not self.enabled:
+            self._thread = threading.Thread(target=lambda: None)
+            self._thread.start()
+            return self
         self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
         return self
@@ -241,7 +246,7 @@ def run_ours(args) -> None:
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev) as clocks:
+    with ClockSampler(dev, enabled=not args.no_clocks) as clocks:
         t0 = time.perf_counter()
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
@@ -335,7 +340,8 @@ def run_ours(args) -> None:
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": decode_bytes,
-                         "avg_launch_us": round(dec_avg_s * 1e6, 2)},
+                         "avg_launch_us": round(dec_avg_s * 1e6, 2),
+                         "median_launch_us": round(statistics.median(decode_ms) * 1e3, 2)},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_s / args.steps * 1e3, 4)},
@@ -430,7 +436,7 @@ def run_reference(args) -> None:
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="llama3_8b_gqa")
@@ -438,6 +444,7 @@ def main(argv=None) -> None:
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of a CUDA graph replay")
+    ap.add_argument("--no-clocks", action="store_true", help="do not sample SM clocks during the timed region")
     ap.add_argument("--ref-seqs", type=int, default=0, help="sequences per reference-arm step (0: all)")
     args = ap.parse_args(argv)
     if args.warmup < 3:

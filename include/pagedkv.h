@@ -173,7 +173,7 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
  * free memory to its KV-cache pool.  This entry point takes the same inputs
  * and outputs as paged_attention_decode, minus the workspace, and allocates
  * nothing: the scratch for split contexts lives in one file-scope device array
- * of PKV_STATIC_WORKSPACE_BYTES (20 MiB), which every GPU that loads the
+ * of PKV_STATIC_WORKSPACE_BYTES (24 MiB), which every GPU that loads the
  * library holds until the process exits.
  *
  * - Sizes whose scratch (paged_attention_workspace_size) exceeds the array are
@@ -189,7 +189,7 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
  *   without ordering) race on the array and give wrong results: order them.
  * Results are bit-identical to paged_attention_decode with its default split.
  */
-#define PKV_STATIC_WORKSPACE_BYTES (20u * 1024u * 1024u)
+#define PKV_STATIC_WORKSPACE_BYTES (24u * 1024u * 1024u)
 
 pkv_status paged_attention_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                           const int32_t* block_tables, int32_t max_blocks_per_seq,

@@ -272,12 +272,14 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
   const int gp = heads_per_segment(group, dtype, opt.force_simt == 1);
   const int gpad = gp == 1 ? 0 : (gp <= 8 ? 8 : 16);
   // One CTA per SM at most (the kernel's grid barrier needs every CTA
-  // resident), so the unit count is capped at 8 per SM.
+  // resident), so the unit count is capped at one per consumer warp of
+  // every SM.
   const int default_units = di.sm_count * kConsumerWarps;
   const int units = (opt.num_units > 0 && opt.num_units < default_units) ? opt.num_units : default_units;
   const int grid = (units + kConsumerWarps - 1) / kConsumerWarps;
 
-  // Ring depth: as many 8-slot rounds as shared memory allows (at most 4).
+  // Ring depth: as many slots per consumer warp as shared memory allows
+  // (at most 4; 2 with ten consumer warps and 8 KiB tiles).
   const int es = elem_bytes(dtype);
   const size_t stage_bytes = static_cast<size_t>(2) * (head_dim * es / 128) * kBoxBytes;
   // 1 KiB alignment slack, abort word, prefix sums and clamped lengths, and

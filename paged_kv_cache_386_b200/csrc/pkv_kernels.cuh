@@ -16,7 +16,7 @@
 //   straddles unit boundaries is a split context whose partial softmax states
 //   are merged, after a grid-wide barrier of the cooperative launch, by the
 //   unit that holds its first piece.
-// * Each CTA runs 8 consumer warps (units) and one producer warp.  Lane w of
+// * Each CTA runs 10 consumer warps (units) and one producer warp.  Lane w of
 //   the producer walks unit w's tiles, reads the physical block id from the
 //   block table one tile ahead and issues TMA tensor loads of the K and V tile
 //   into unit w's ring of `stages` shared-memory slots (mbarrier full/empty
@@ -46,7 +46,7 @@
 namespace pkv {
 
 constexpr int kBlockTokens = 16;
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 10;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kBoxBytes = 16 * 128;  // one TMA box: 16 tokens x 128 bytes
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -935,7 +935,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     constexpr int kWarps = kConsumerWarps + 1;
     const int gw = blockIdx.x * kWarps + warp, n_warps = gridDim.x * kWarps;
     const int items = U * p.gp;
-    // At most 32 items per warp (U <= 8 per CTA and gp <= 16): load their
+    // At most 32 items per warp (U <= kConsumerWarps per CTA, gp <= 16):
+    // load their
     // metadata in one round, lane t for the warp's t-th item.
     int4 my_item = make_int4(-1, 0, 0, 0);
     {
