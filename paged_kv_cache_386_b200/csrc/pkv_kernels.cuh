@@ -606,6 +606,49 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
   auto rec_of = [&](int j) -> const float* {  // record of piece j (unit u + j)
     return p.records + (static_cast<size_t>(u + j) * 2 + (j == 0 ? mt.z : 0)) * p.rec_floats;
   };
+  T* const ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
+  auto store = [&](const float (&acc)[DPL], float inv) {
+    if constexpr (DPL == 4) {
+      store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    } else if constexpr (DT == kF32) {
+      *reinterpret_cast<float2*>(ob) = make_float2(acc[0] * inv, acc[1] * inv);
+    } else {
+      *reinterpret_cast<uint32_t*>(ob) = pack2<DT == kBF16>(acc[0] * inv, acc[1] * inv);
+    }
+  };
+  if (n <= 8) {
+    // Common case: every load of every piece issued in one round.
+    float mj[8], lj[8], o[8][DPL];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float* r = rec_of(min(j, n - 1));
+      mj[j] = __ldcg(r + mo);
+      lj[j] = __ldcg(r + lo);
+      if constexpr (DPL == 4) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(r + oo));
+        o[j][0] = x.x; o[j][1] = x.y; o[j][2] = x.z; o[j][3] = x.w;
+      } else {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(r + oo));
+        o[j][0] = x.x; o[j][1] = x.y;
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < n) M = fmaxf(M, mj[j]);
+    float L = 0.f, acc[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float w = j < n ? exp2f(mj[j] - M) : 0.f;
+      L = fmaf(w, lj[j], L);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, o[j][i], acc[i]);
+    }
+    store(acc, 1.f / L);
+    return;
+  }
   // Scalars of pieces lane and lane + 32; pieces beyond 64 (rare) are folded
   // in by a plain loop.
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -654,15 +697,7 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
       for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wj, o[jj][i], acc[i]);
     }
   }
-  const float inv = 1.f / L;
-  T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
-  if constexpr (DPL == 4) {
-    store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  } else if constexpr (DT == kF32) {
-    *reinterpret_cast<float2*>(ob) = make_float2(acc[0] * inv, acc[1] * inv);
-  } else {
-    *reinterpret_cast<uint32_t*>(ob) = pack2<DT == kBF16>(acc[0] * inv, acc[1] * inv);
-  }
+  store(acc, 1.f / L);
 }
 
 // GPAD: 0 = CUDA-core consumer (gp == 1); 8 or 16 = tensor-core consumer.
