@@ -142,6 +142,45 @@ pkv_status paged_attention_decode(const void* q, const void* k_cache, const void
                                   int32_t head_dim, int32_t block_size, void* out, pkv_dtype dtype,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * paged_attention_decode_cascade -- paged_attention_decode for batches whose
+ * sequences share prefix blocks (prefix caching: sequences that start with the
+ * same block-aligned tokens point their tables at the same physical blocks,
+ * "Transformer anatomy" ch. 15 §15.6; refcounted block sharing for parallel
+ * sampling and prefix caching, "LLM Primer VI" ch. 8 §8.1 and §8.3).
+ *
+ * Group i owns a shared prefix of prefix_lens[i] tokens (a multiple of
+ * block_size) held by blocks prefix_block_tables[i][0 .. prefix_lens[i]/16).
+ * Sequence b with g = seq_group[b] >= 0 has the context "prefix of group g"
+ * followed by its private suffix of context_lens[b] tokens, held by
+ * block_tables[b][..]; seq_group[b] = -1 means no shared prefix (context_lens
+ * and block_tables then cover the whole context).  The result equals
+ * paged_attention_decode over the concatenated tables, within rounding.
+ *
+ * The prefix is read once per (group, kv head) and evaluated as one dense
+ * attention over all member rows on tensor cores; the suffixes go through the
+ * decode kernel, which continues from each row's prefix state.  16-bit dtypes
+ * only (PKV_F32 returns PKV_ERR_UNSUPPORTED).  A group id >= n_groups or a bad
+ * prefix length sets PKV_DEVERR_CONTEXT.
+ *
+ *   prefix_block_tables : device, int32 [n_groups][max_prefix_blocks]
+ *   prefix_lens, seq_group : device, int32 [n_groups], [batch]
+ *   workspace : at least paged_attention_cascade_workspace_size() bytes (or
+ *               NULL for a stream-ordered allocation), 256-byte aligned
+ */
+pkv_status paged_attention_cascade_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                                  int32_t head_dim, pkv_dtype dtype, size_t* bytes);
+
+pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, const void* v_cache,
+                                          int32_t n_groups, const int32_t* prefix_block_tables,
+                                          int32_t max_prefix_blocks, const int32_t* prefix_lens,
+                                          const int32_t* seq_group, const int32_t* block_tables,
+                                          int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                          int32_t batch, int32_t num_blocks, float scale,
+                                          int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                          int32_t block_size, void* out, pkv_dtype dtype,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* Tuning and test hooks for paged_attention_decode_ex. Zero-initialise. */
 typedef struct pkv_decode_options {
   int32_t num_units;   /* 0: default split (one work unit per consumer warp on every SM);

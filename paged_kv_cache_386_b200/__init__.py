@@ -23,6 +23,7 @@ import torch
 
 __all__ = [
     "paged_kv_append", "paged_attention_decode", "paged_attention_decode_noalloc",
+    "paged_attention_decode_cascade", "paged_attention_cascade_workspace_size",
     "paged_attention_workspace_size",
     "pkv_get_device_error", "pkv_status_string", "pkv_version", "PagedKVError", "library_path",
     "DEVERR_BLOCK_ID", "DEVERR_CONTEXT", "DEVERR_SLOT", "DEVERR_TIMEOUT",
@@ -73,6 +74,11 @@ def _load() -> ctypes.CDLL:
     lib.paged_attention_decode.restype = ctypes.c_int
     lib.paged_attention_decode_ex.argtypes = dec + [ctypes.POINTER(_Options)]
     lib.paged_attention_decode_ex.restype = ctypes.c_int
+    lib.paged_attention_cascade_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(sz)]
+    lib.paged_attention_cascade_workspace_size.restype = ctypes.c_int
+    lib.paged_attention_decode_cascade.argtypes = [p, p, p, i32, p, i32, p, p, p, i32, p, i32, i32, f32, i32, i32,
+                                                   i32, i32, p, ctypes.c_int, p, sz, p]
+    lib.paged_attention_decode_cascade.restype = ctypes.c_int
     lib.paged_attention_decode_noalloc.argtypes = dec[:15] + [p]
     lib.paged_attention_decode_noalloc.restype = ctypes.c_int
     lib.pkv_get_device_error.argtypes = [p, ctypes.POINTER(ctypes.c_uint32)]
@@ -157,6 +163,49 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
         B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
         ws_ptr, ws_bytes, _stream(stream), ctypes.byref(opts)), "paged_attention_decode")
+    return out
+
+
+def paged_attention_cascade_workspace_size(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                                           dtype: torch.dtype) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_load().paged_attention_cascade_workspace_size(batch, n_q_heads, n_kv_heads, head_dim,
+                                                          _DTYPE[dtype], ctypes.byref(out)),
+           "paged_attention_cascade_workspace_size")
+    return int(out.value)
+
+
+def paged_attention_decode_cascade(q, k_cache, v_cache, prefix_block_tables, prefix_lens, seq_group,
+                                   block_tables, context_lens, scale: float, out=None, workspace=None,
+                                   block_size: int = 16, stream=None):
+    """Decode for sequences that share prefix blocks: group i's prefix
+    (``prefix_lens[i]`` tokens in ``prefix_block_tables[i]``) is attended once
+    per kv head for all its members (``seq_group[b] == i``), then each
+    sequence's private suffix (``block_tables[b]``, ``context_lens[b]``
+    tokens) continues from that state."""
+    lib = _load()
+    B, n_q, d = q.shape
+    num_blocks, n_kv, bs, d2 = k_cache.shape
+    if d2 != d or bs != block_size or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch")
+    for t, name in ((prefix_block_tables, "prefix_block_tables"), (prefix_lens, "prefix_lens"),
+                    (seq_group, "seq_group"), (block_tables, "block_tables"), (context_lens, "context_lens")):
+        if t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    if out is None:
+        out = torch.empty_like(q)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    n_groups = prefix_lens.shape[0]
+    _check(lib.paged_attention_decode_cascade(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), n_groups,
+        _dev(prefix_block_tables, "prefix_block_tables") if n_groups else None,
+        prefix_block_tables.shape[1] if n_groups else 0,
+        _dev(prefix_lens, "prefix_lens") if n_groups else None, _dev(seq_group, "seq_group") if n_groups else None,
+        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+        B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
+        ws_ptr, ws_bytes, _stream(stream)), "paged_attention_decode_cascade")
     return out
 
 

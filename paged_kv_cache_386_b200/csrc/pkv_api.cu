@@ -7,6 +7,7 @@
 
 #include "pagedkv.h"
 #include "pkv_kernels.cuh"
+#include "pkv_prefix.cuh"
 
 namespace pkv {
 namespace {
@@ -184,6 +185,33 @@ pkv_status dispatch_dim(int head_dim, int gpad, const CUtensorMap& mk, const CUt
                         : dispatch_gpad<DT, 128>(gpad, mk, mv, p, grid, smem, stream);
 }
 
+// Shared-memory ring of the prefix kernel: three stages of 64 tokens of K and V.
+constexpr int kPrefixStages = 3;
+
+size_t prefix_init_bytes(int batch, int n_q_heads, int head_dim) {
+  return (static_cast<size_t>(batch) * n_q_heads * (head_dim + 2) * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+template <int DT, int D>
+pkv_status launch_prefix(const CUtensorMap& mk, const CUtensorMap& mv, const PrefixParams& pp, int n_kv, size_t smem,
+                         cudaStream_t stream) {
+  auto kern = pkv_prefix_kernel<DT, D>;
+  static bool opted_in[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  if (!opted_in[dev]) {
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - 256) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    opted_in[dev] = true;
+  }
+  const int rows = pp.batch * pp.group;
+  const dim3 grid((rows + kPrefixRows - 1) / kPrefixRows, n_kv, pp.n_groups);
+  kern<<<grid, kPrefixThreads, smem, stream>>>(mk, mv, pp);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace pkv
 
@@ -248,12 +276,19 @@ pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int3
   return PKV_OK;
 }
 
-pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const void* v_cache,
-                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
-                                     const int32_t* context_lens, int32_t batch, int32_t num_blocks, float scale,
-                                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
-                                     void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
-                                     void* stream, const pkv_decode_options* options) {
+}  // extern "C"
+
+namespace pkv {
+namespace {
+// The decode launch behind paged_attention_decode_ex and the cascade: `init`
+// and `seq_group` (both null for a plain decode) give an initial softmax state
+// per (sequence, query head).
+pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                       int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch, int32_t num_blocks,
+                       float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
+                       void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes, void* stream,
+                       const pkv_decode_options* options, const float* init, const int32_t* seq_group,
+                       int32_t n_groups) {
   pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                     num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
   if (st != PKV_OK || batch == 0) return st;
@@ -326,6 +361,9 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
   p.rec_floats = record_floats(gp, head_dim);
   p.head_dim = head_dim;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.init = init;
+  p.seq_group = seq_group;
+  p.n_groups = n_groups;
 
   if (st == PKV_OK) {
     switch (dtype) {
@@ -336,6 +374,21 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
   }
   if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == PKV_OK) st = PKV_ERR_CUDA;
   return st;
+}
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t batch, int32_t num_blocks, float scale,
+                                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
+                                     void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+                                     void* stream, const pkv_decode_options* options) {
+  return decode_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
+                     n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, workspace, workspace_bytes, stream,
+                     options, nullptr, nullptr, 0);
 }
 
 pkv_status paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -394,6 +447,88 @@ pkv_status paged_attention_decode_noalloc(const void* q, const void* k_cache, co
   return paged_attention_decode_ex(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                    num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, ws,
                                    PKV_STATIC_WORKSPACE_BYTES, stream, nullptr);
+}
+
+pkv_status paged_attention_cascade_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                                  int32_t head_dim, pkv_dtype dtype, size_t* bytes) {
+  size_t dec = 0;
+  const pkv_status st = paged_attention_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, dtype, &dec);
+  if (st != PKV_OK) return st;
+  *bytes = prefix_init_bytes(batch, n_q_heads, head_dim) + dec;
+  return PKV_OK;
+}
+
+pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, const void* v_cache, int32_t n_groups,
+                                          const int32_t* prefix_block_tables, int32_t max_prefix_blocks,
+                                          const int32_t* prefix_lens, const int32_t* seq_group,
+                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                          const int32_t* context_lens, int32_t batch, int32_t num_blocks,
+                                          float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                          int32_t block_size, void* out, pkv_dtype dtype, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
+                                    num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
+  if (st != PKV_OK || batch == 0) return st;
+  if (n_groups < 0 || n_groups > 65535) return PKV_ERR_INVALID_ARG;
+  if (dtype == PKV_F32) return PKV_ERR_UNSUPPORTED;  // the prefix GEMM runs on 16-bit tensor-core operands
+  if (n_groups > 0 && (!prefix_block_tables || !prefix_lens || !seq_group || max_prefix_blocks <= 0 ||
+                       max_prefix_blocks > (1 << 26)))
+    return PKV_ERR_INVALID_ARG;
+  if (n_groups == 0)
+    return decode_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks,
+                       scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, workspace, workspace_bytes,
+                       stream, nullptr, nullptr, nullptr, 0);
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  size_t need = 0;
+  st = paged_attention_cascade_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, dtype, &need);
+  if (st != PKV_OK) return st;
+  void* ws = workspace;
+  bool own = false;
+  if (ws == nullptr) {
+    if (cudaMallocAsync(&ws, need, s) != cudaSuccess) return PKV_ERR_CUDA;
+    own = true;
+  } else if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
+    return PKV_ERR_WORKSPACE;
+  }
+  const size_t init_bytes = prefix_init_bytes(batch, n_q_heads, head_dim);
+  float* init = static_cast<float*>(ws);
+
+  CUtensorMap mk, mv;
+  st = encode_cache_map(&mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
+  if (st == PKV_OK) st = encode_cache_map(&mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+  PrefixParams pp;
+  pp.q = q;
+  pp.prefix_tables = prefix_block_tables;
+  pp.prefix_lens = prefix_lens;
+  pp.seq_group = seq_group;
+  pp.init = init;
+  pp.batch = batch;
+  pp.n_groups = n_groups;
+  pp.max_prefix_blocks = max_prefix_blocks;
+  pp.num_blocks = num_blocks;
+  pp.n_q_heads = n_q_heads;
+  pp.group = n_q_heads / n_kv_heads;
+  pp.stages = kPrefixStages;
+  pp.scale_log2 = scale * 1.4426950408889634f;
+  const size_t stage_bytes = static_cast<size_t>(2) * kPrefixBlocks * (head_dim * 2 / 128) * kBoxBytes;
+  const size_t smem = 1024 + kPrefixStages * (stage_bytes + 2 * sizeof(uint64_t)) + 16 + static_cast<size_t>(batch) * 4;
+  if (smem + 256 > static_cast<size_t>(di.smem_optin)) st = st == PKV_OK ? PKV_ERR_UNSUPPORTED : st;
+  if (st == PKV_OK) {
+    if (dtype == PKV_F16)
+      st = head_dim == 64 ? launch_prefix<kF16, 64>(mk, mv, pp, n_kv_heads, smem, s)
+                          : launch_prefix<kF16, 128>(mk, mv, pp, n_kv_heads, smem, s);
+    else
+      st = head_dim == 64 ? launch_prefix<kBF16, 64>(mk, mv, pp, n_kv_heads, smem, s)
+                          : launch_prefix<kBF16, 128>(mk, mv, pp, n_kv_heads, smem, s);
+  }
+  if (st == PKV_OK)
+    st = decode_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
+                     n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, static_cast<uint8_t*>(ws) + init_bytes,
+                     need - init_bytes, stream, nullptr, init, seq_group, n_groups);
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == PKV_OK) st = PKV_ERR_CUDA;
+  return st;
 }
 
 pkv_status pkv_get_device_error(void* stream, uint32_t* flags) {

@@ -119,6 +119,13 @@ struct DecodeParams {
   const int32_t* context_lens;
   float* records;  // [num_units][2][rec_floats]: O[gp][D], m[gp], l[gp]
   int4* meta;      // [num_units]: split segment whose first piece the unit holds
+  // Optional initial softmax state per (sequence, query head) -- the shared
+  // prefix part of a cascade decode: O [batch][n_q][D] unnormalised, then
+  // m [batch][n_q] (log2 units), then l [batch][n_q].  Used for sequences with
+  // seq_group[b] >= 0 when `init` is not null.
+  const float* init;
+  const int32_t* seq_group;
+  int32_t n_groups;
   int32_t max_blocks_per_seq;
   int32_t batch;
   int32_t num_blocks;
@@ -138,6 +145,18 @@ struct Walk {
   int b, hg, j, nb, ctx;
   int k, k_end;
 };
+
+// Does sequence b continue from an initial state?  A group id outside
+// [0, n_groups) is flagged and ignored (its state was never computed).
+__device__ __forceinline__ bool has_init(const DecodeParams& p, int b) {
+  const int gi = __ldg(p.seq_group + b);
+  if (gi < 0) return false;
+  if (gi >= p.n_groups) {
+    flag_error(PKV_DEVERR_CONTEXT);
+    return false;
+  }
+  return true;
+}
 
 __device__ __forceinline__ int clamp_ctx(int c, int max_ctx) { return c < 0 ? 0 : (c > max_ctx ? max_ctx : c); }
 
@@ -226,6 +245,28 @@ struct MmaConsumer {
     for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     m[0] = m[1] = -INFINITY;
     l[0] = l[1] = 0.f;
+  }
+
+  // Continue from a given partial state (the segment's first piece only).
+  __device__ __forceinline__ void load_init(const DecodeParams& p, int b, int hg, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const size_t nqb = static_cast<size_t>(p.batch) * p.n_q_heads;
+    constexpr int kRows = (GPAD == 16) ? 2 : 1;
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      const int row = g + 8 * r;
+      if (row >= p.gp) continue;
+      const size_t rowi = static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + row;
+      const float* oi = p.init + rowi * D;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const float2 x = __ldg(reinterpret_cast<const float2*>(oi + n * 8 + 2 * t));
+        o[n][2 * r] = x.x;
+        o[n][2 * r + 1] = x.y;
+      }
+      m[r] = __ldg(p.init + nqb * D + rowi);
+      l[r] = t == 0 ? __ldg(p.init + nqb * D + nqb + rowi) : 0.f;
+    }
   }
 
   __device__ __forceinline__ void tile(uint32_t kbase, int nv, float scale_log2, int lane) {
@@ -429,6 +470,20 @@ struct SimtConsumer {
     for (int i = 0; i < DL; ++i) o[i] = 0.f;
     m = -INFINITY;
     l = 0.f;
+  }
+
+  // Continue from a given partial state (the segment's first piece only):
+  // the token lanes' partial sums are added up at the end, so lane tp == 0
+  // carries the initial O and l.
+  __device__ __forceinline__ void load_init(const DecodeParams& p, int b, int hg, int lane) {
+    const int tp = lane & 7, sub = lane >> 3;
+    const size_t nqb = static_cast<size_t>(p.batch) * p.n_q_heads;
+    const size_t rowi = static_cast<size_t>(b) * p.n_q_heads + hg;
+    const float* oi = p.init + rowi * D + sub * DL;
+#pragma unroll
+    for (int i = 0; i < DL; ++i) o[i] = tp == 0 ? __ldg(oi + i) : 0.f;
+    m = __ldg(p.init + nqb * D + rowi);
+    l = tp == 0 ? __ldg(p.init + nqb * D + nqb + rowi) : 0.f;
   }
 
   __device__ __forceinline__ void tile(uint32_t kbase, int nv, float scale_log2, int lane) {
@@ -928,6 +983,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           cp_async_wait_all();
           __syncwarp();
           cs.begin(qbuf, p.gp, lane);
+          if (p.init != nullptr && wk.j == 0 && has_init(p, wk.b)) cs.load_init(p, wk.b, wk.hg, lane);
           __syncwarp();
           q_ready = false;
         }
@@ -987,15 +1043,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       mt.w = __shfl_sync(0xffffffffu, my_item.w, t);
       if (mt.x >= 0) merge_head<DT, D>(p, i / p.gp, mt, i % p.gp, lane);
     }
-    // Sequences with no tokens get a zero output row.
+    // Sequences with no tokens get a zero output row, or, when an initial
+    // state is given for them, that state normalised.
     const int total = B * p.ng;
+    const size_t nqb = static_cast<size_t>(B) * p.n_q_heads;
     for (int sgi = gw; sgi < total; sgi += n_warps) {
       const int b = sgi / p.ng, hg = sgi % p.ng;
       if (ctxs[b] != 0) continue;
+      const bool with_init = p.init != nullptr && has_init(p, b);
       for (int e = lane; e < p.gp * (D / 4); e += 32) {
         const int g = e / (D / 4), d4 = (e % (D / 4)) * 4;
-        store4<DT>(static_cast<OutT*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + d4,
-                   0.f, 0.f, 0.f, 0.f);
+        const size_t rowi = static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        float inv = 0.f;
+        if (with_init) {
+          x = __ldg(reinterpret_cast<const float4*>(p.init + rowi * D + d4));
+          const float li = __ldg(p.init + nqb * D + nqb + rowi);
+          inv = li > 0.f ? 1.f / li : 0.f;
+        }
+        store4<DT>(static_cast<OutT*>(p.out) + rowi * D + d4, x.x * inv, x.y * inv, x.z * inv, x.w * inv);
       }
     }
   }

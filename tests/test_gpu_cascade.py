@@ -1,0 +1,119 @@
+"""Cascade decode (shared prefix attended once per group and kv head, then the
+private suffixes) against the CPU oracle on the full, concatenated tables."""
+
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_386_b200 as pkv
+import workloads as W
+from tests.gpu_helpers import assert_close, bits, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def run_cascade(w, cv=None, check_errors=True, workspace=None):
+    dev = torch.device("cuda")
+    kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
+    if w.appended:
+        pkv.paged_kv_append(w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev), kc, vc)
+    cv = cv or W.cascade_view(w)
+    out = pkv.paged_attention_decode_cascade(
+        w.q.to(dev), kc, vc, cv.prefix_block_tables.to(dev), cv.prefix_lens.to(dev), cv.seq_group.to(dev),
+        cv.block_tables.to(dev), cv.context_lens.to(dev), w.scale, workspace=workspace)
+    torch.cuda.synchronize()
+    if check_errors:
+        assert pkv.pkv_get_device_error() == 0
+    return out.cpu()
+
+
+def check(w, rows=None):
+    out = run_cascade(w)
+    ref, _, _ = oracle.workload_decode(w, rows=rows)
+    return assert_close(out, ref, w.dtype, rows=rows, what=w.name)
+
+
+SMALL = {
+    "shared_prefix_small": lambda: W.shared_prefix(n_seqs=12, prefix=512, seed=41),
+    "best_of_8_small": lambda: W.best_of_n(prompts=3, n=8, seed=42),
+    "prefix_ragged_tile": lambda: W.shared_prefix(n_seqs=5, prefix=272, suffix=(16, 100), seed=43),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_cascade_small_full_output(name):
+    check(SMALL[name]())
+
+
+@pytest.mark.parametrize("name", ["shared_prefix_70b", "best_of_8"])
+def test_cascade_full_size_sampled(name):
+    w = W.shared_prefix(seed=0) if name == "shared_prefix_70b" else W.best_of_n(seed=0)
+    check(w, rows=sample_rows(w, 128))
+
+
+SHAPES = [
+    (torch.bfloat16, 128, 8, 8),     # G=1: CUDA-core suffix path continues from the prefix state
+    (torch.float16, 64, 16, 4),      # G=4, d=64
+    (torch.bfloat16, 128, 32, 2),    # G=16: 16-row tensor-core tiles
+    (torch.bfloat16, 128, 40, 4),    # G=10
+]
+
+
+@pytest.mark.parametrize("dtype,d,nq,nkv", SHAPES, ids=[f"{str(s[0])[6:]}-d{s[1]}-{s[2]}x{s[3]}" for s in SHAPES])
+def test_cascade_head_shapes(dtype, d, nq, nkv):
+    lens = [160 + 5, 160 + 40, 160 + 1, 160 + 77, 160 + 16]
+    w = W.build_workload("cshape", lens, nq, nkv, d, dtype, seed=44, groups=[([0, 1, 2, 3, 4], 160)])
+    check(w)
+
+
+def test_cascade_mixed_groups_and_loners():
+    lens = [96 + 10, 300, 96 + 33, 64 + 5, 64 + 70, 50, 96 + 1]
+    w = W.build_workload("mixed", lens, 16, 2, 128, torch.bfloat16, seed=45,
+                         groups=[([0, 2, 6], 96), ([3, 4], 64)])
+    cv = W.cascade_view(w)
+    assert cv.seq_group.tolist() == [0, -1, 0, 1, 1, -1, 0]
+    check(w)
+
+
+def test_cascade_empty_suffix_and_empty_prefix():
+    w = W.build_workload("edges", [64 + 20, 64 + 3, 48 + 9], 8, 2, 128, torch.bfloat16, seed=46, append=False,
+                         groups=[([0, 1], 64), ([2], 48)])
+    w.context_lens[1] = 64          # sequence 1 is exactly the shared prefix
+    cv = W.cascade_view(w)
+    assert int(cv.context_lens[1]) == 0
+    cv.prefix_lens[1] = 0           # group 1: no shared tokens after all
+    wide = torch.full((w.batch, w.max_blocks_per_seq), -1, dtype=torch.int32)
+    wide[:, : cv.block_tables.shape[1]] = cv.block_tables
+    wide[2] = w.block_tables[2]     # its suffix is then its whole context
+    cv.block_tables = wide
+    cv.context_lens[2] = w.context_lens[2]
+    out = run_cascade(w, cv)
+    ref, _, _ = oracle.workload_decode(w)
+    assert_close(out, ref, w.dtype, what="edges")
+
+
+def test_cascade_matches_plain_decode():
+    w = W.shared_prefix(n_seqs=8, prefix=256, seed=47)
+    out_c = run_cascade(w)
+    dev = torch.device("cuda")
+    kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
+    pkv.paged_kv_append(w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev), kc, vc)
+    out_p = pkv.paged_attention_decode(w.q.to(dev), kc, vc, w.block_tables.to(dev), w.context_lens.to(dev),
+                                       w.scale).cpu()
+    assert_close(out_c, out_p.double(), w.dtype, what="cascade vs plain")
+    assert torch.equal(bits(run_cascade(w)), bits(out_c))   # deterministic
+
+
+def test_cascade_bad_group_id_sets_flag():
+    w = W.shared_prefix(n_seqs=4, prefix=64, seed=48)
+    cv = W.cascade_view(w)
+    cv.seq_group[2] = 5   # no such group
+    run_cascade(w, cv, check_errors=False)
+    assert pkv.pkv_get_device_error() & pkv.DEVERR_CONTEXT
+
+
+def test_cascade_fp32_is_unsupported():
+    w = W.build_workload("f32", [40, 50], 4, 2, 64, torch.float32, seed=49, groups=[([0, 1], 32)])
+    with pytest.raises(pkv.PagedKVError) as e:
+        run_cascade(w)
+    assert e.value.status == 2

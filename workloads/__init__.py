@@ -230,6 +230,43 @@ def _randn(shape, dtype, gen, chunk_elems: int = 1 << 26) -> torch.Tensor:
     return out
 
 
+@dataclass
+class CascadeView:
+    """The same workload split into shared prefixes and private suffixes."""
+    prefix_block_tables: torch.Tensor  # int32 [n_groups, max_prefix_blocks]
+    prefix_lens: torch.Tensor          # int32 [n_groups]
+    seq_group: torch.Tensor            # int32 [batch], -1 = no group
+    block_tables: torch.Tensor         # int32 [batch, max suffix blocks]
+    context_lens: torch.Tensor         # int32 [batch] suffix tokens
+
+
+def cascade_view(w: DecodeWorkload) -> CascadeView:
+    """Table bookkeeping only: the shared prefix blocks of each group (from
+    ``w.meta['groups']``) and, per sequence, the remaining private blocks."""
+    groups = w.meta.get("groups", [])
+    bs = w.block_size
+    n_groups = len(groups)
+    max_pb = max([pre // bs for _, pre in groups] + [1])
+    ptab = torch.full((max(n_groups, 1), max_pb), -1, dtype=torch.int32)
+    plen = torch.zeros(max(n_groups, 1), dtype=torch.int32)
+    seq_group = torch.full((w.batch,), -1, dtype=torch.int32)
+    for gi, (members, pre) in enumerate(groups):
+        nb = pre // bs
+        ptab[gi, :nb] = w.block_tables[members[0], :nb]
+        plen[gi] = pre
+        for b in members:
+            seq_group[b] = gi
+    skip = [int(plen[int(seq_group[b])]) // bs if seq_group[b] >= 0 else 0 for b in range(w.batch)]
+    lens = [n - s * bs for n, s in zip(w.lens(), skip)]
+    width = max(1, max((w.max_blocks_per_seq - s) for s in skip))
+    tab = torch.full((w.batch, width), -1, dtype=torch.int32)
+    for b in range(w.batch):
+        row = w.block_tables[b, skip[b]:]
+        tab[b, : row.numel()] = row
+    return CascadeView(ptab[:n_groups] if n_groups else ptab[:0], plen[:n_groups], seq_group, tab,
+                       torch.tensor(lens, dtype=torch.int32))
+
+
 # ---------------------------------------------------------------------------
 # The five workload shapes (Llama-class, block size 16).
 # ---------------------------------------------------------------------------
