@@ -193,14 +193,29 @@ def run_ours(args) -> None:
     q, k_new, v_new = w.q.to(dev), w.k_new.to(dev), w.v_new.to(dev)
     slots, bt, cl = w.slot_mapping.to(dev), w.block_tables.to(dev), w.context_lens.to(dev)
     out = torch.empty_like(q)
-    ws = torch.empty(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
-                                                        w.dtype), dtype=torch.uint8, device=dev)
+    if args.cascade:
+        # Shared prefixes attended once per group and kv head, then the suffixes.
+        cv = W.cascade_view(w)
+        c_pt, c_pl, c_sg, c_bt, c_cl = (t.to(dev) for t in (cv.prefix_block_tables, cv.prefix_lens, cv.seq_group,
+                                                             cv.block_tables, cv.context_lens))
+        ws = torch.empty(pkv.paged_attention_cascade_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
+                                                                    w.dtype), dtype=torch.uint8, device=dev)
+    else:
+        ws = torch.empty(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
+                                                            w.dtype), dtype=torch.uint8, device=dev)
+
+    def decode(stream_=None):
+        if args.cascade:
+            pkv.paged_attention_decode_cascade(q, kc, vc, c_pt, c_pl, c_sg, c_bt, c_cl, w.scale, out=out,
+                                               workspace=ws, stream=stream_)
+        else:
+            pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream_)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
         pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
-        pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream)
+        decode(stream)
 
     # Warm-up: W steps, continued until 0.3 s have passed so that the SM
     # clock has left its idle state before timing.
@@ -230,7 +245,7 @@ def run_ours(args) -> None:
                 ev_a.record()
                 pkv.paged_kv_append(k_new, v_new, slots, kc, vc)
                 ev_b.record()
-                pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws)
+                decode()
                 ev_c.record()
             stream.wait_stream(cap)
             for _ in range(args.warmup):
@@ -260,7 +275,7 @@ def run_ours(args) -> None:
                 a.record(stream)
                 pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
                 b.record(stream)
-                pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream)
+                decode(stream)
                 c.record(stream)
                 c.synchronize()
                 step_ms.append(a.elapsed_time(c))
@@ -281,8 +296,13 @@ def run_ours(args) -> None:
     # End to end through the public API with host buffers: pinned host ->
     # device copies of this step's inputs, append + decode, device -> host read
     # of the output, all inside the timed region.
-    h_in = [t.pin_memory() for t in (w.q, w.k_new, w.v_new, w.slot_mapping, w.block_tables, w.context_lens)]
-    d_in = [q, k_new, v_new, slots, bt, cl]
+    if args.cascade:
+        h_in = [t.pin_memory() for t in (w.q, w.k_new, w.v_new, w.slot_mapping, cv.prefix_block_tables,
+                                         cv.prefix_lens, cv.seq_group, cv.block_tables, cv.context_lens)]
+        d_in = [q, k_new, v_new, slots, c_pt, c_pl, c_sg, c_bt, c_cl]
+    else:
+        h_in = [t.pin_memory() for t in (w.q, w.k_new, w.v_new, w.slot_mapping, w.block_tables, w.context_lens)]
+        d_in = [q, k_new, v_new, slots, bt, cl]
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = h_out.numel() * h_out.element_size()
@@ -291,7 +311,7 @@ def run_ours(args) -> None:
         for d, h in zip(d_in, h_in):
             d.copy_(h, non_blocking=True)
         pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
-        pkv.paged_attention_decode(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream)
+        decode(stream)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -333,10 +353,13 @@ def run_ours(args) -> None:
                        "mean_context": round(tr["tokens"] / w.batch, 1), "parallelism": f"replicas x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed)", "seed": args.seed,
                        "warmup_steps_run": warm_steps,
-                       "launch": launch_note},
+                       "launch": launch_note,
+                       "decode": "cascade (shared prefix once per group)" if args.cascade else "paged decode"},
             "tokens_per_s_per_layer": round(tokens_per_s, 1),
             "kv_bytes_per_step": kv_bytes,
-            "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (pkv_decode_kernel)",
+            "roofline": {"bound": "hbm",
+                         "kernel": ("paged_attention_decode_cascade (pkv_prefix_kernel + pkv_decode_kernel)"
+                                    if args.cascade else "paged_attention_decode (pkv_decode_kernel)"),
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": decode_bytes,
@@ -345,7 +368,7 @@ def run_ours(args) -> None:
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_s / args.steps * 1e3, 4)},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": (3 if args.cascade else 2) * args.steps,
             "clocks": clocks.summary(),
             "wall_s_timed_loop": round(wall, 4),
         }
@@ -445,6 +468,8 @@ def main(argv=None) -> None:
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of a CUDA graph replay")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample SM clocks during the timed region")
+    ap.add_argument("--cascade", action="store_true",
+                    help="decode shared-prefix workloads with paged_attention_decode_cascade")
     ap.add_argument("--ref-seqs", type=int, default=0, help="sequences per reference-arm step (0: all)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
