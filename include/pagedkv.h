@@ -70,7 +70,9 @@ typedef enum pkv_status {
   PKV_ERR_UNSUPPORTED = 2,   /* block_size, head_dim, dtype or batch outside the supported set */
   PKV_ERR_OUT_OF_RANGE = 3,  /* a kernel saw a bad block id, context length or slot */
   PKV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
-  PKV_ERR_WORKSPACE = 5      /* workspace too small */
+  PKV_ERR_WORKSPACE = 5,     /* workspace too small */
+  PKV_ERR_NO_BLOCKS = 6,     /* block manager: not enough free or evictable blocks (nothing changed) */
+  PKV_ERR_HOST_MEMORY = 7    /* block manager: host allocation failed (the manager must be destroyed) */
 } pkv_status;
 
 /* Bits of the device error word (pkv_get_device_error). */
@@ -236,6 +238,126 @@ pkv_status paged_attention_decode_noalloc(const void* q, const void* k_cache, co
                                           float scale, int32_t n_q_heads, int32_t n_kv_heads,
                                           int32_t head_dim, int32_t block_size, void* out,
                                           pkv_dtype dtype, void* stream);
+
+/*
+ * paged_kv_copy_blocks -- copy whole physical blocks inside the pool, both
+ * caches: for p in [0, n_pairs),
+ *   k_cache[dst[p]] = k_cache[src[p]],  v_cache[dst[p]] = v_cache[src[p]]
+ * (every kv head, token and dim of the block).  This is the copy of
+ * copy-on-write: a block shared by several block tables ("LLM Primer VI"
+ * ch. 8 §8.1, refcounted sharing for parallel sampling) that one of them is
+ * about to append to is first duplicated into a fresh block.  pkv_bm_append
+ * emits the pairs; run this copy before paged_kv_append writes the new token.
+ * The copy is bit-exact.  A dst block must not appear twice nor be a src of
+ * the same call (the pairs would race).  A src or dst outside [0, num_blocks)
+ * skips that pair and sets PKV_DEVERR_BLOCK_ID.
+ *
+ *   src_blocks, dst_blocks : device, int32 [n_pairs]
+ *   k_cache, v_cache       : device, [num_blocks][n_kv_heads][block_size][head_dim], dtype
+ *   stream                 : cudaStream_t
+ */
+pkv_status paged_kv_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_blocks,
+                                const int32_t* dst_blocks, int32_t n_pairs, int32_t num_blocks,
+                                int32_t block_size, int32_t n_kv_heads, int32_t head_dim,
+                                pkv_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Host block manager (pkv_bm_*): the allocator that produces the block tables
+ * and slot mappings the kernels above consume.  Pure host code; no call
+ * touches the GPU.  Not thread-safe: one manager per scheduler thread.
+ *
+ * Model ("Transformer anatomy" ch. 15 §15.5): a pool of num_blocks physical
+ * blocks of block_size tokens; every sequence owns a block table; a new token
+ * goes into the sequence's last block, and a new block is taken from the free
+ * pool when that block is full; freeing a sequence returns its blocks.
+ * Blocks are refcounted so that several tables can point at one block
+ * ("LLM Primer VI" ch. 8 §8.1): pkv_bm_fork shares all blocks of a sequence,
+ * and an append into a shared, partly filled last block first moves the
+ * appending sequence onto a private copy (copy-on-write).
+ *
+ * Prefix caching ("Transformer anatomy" ch. 15 §15.6; "LLM Primer VI" ch. 8
+ * §8.3): when enabled, each full prompt block is keyed by a hash that the
+ * caller supplies (pkv_bm_hash_blocks computes the chained hash used by the
+ * tests: block i's key covers all tokens up to the end of block i).  A new
+ * sequence whose leading block keys are cached shares those blocks and
+ * reports how many prompt tokens need no prefill.  A cached block whose
+ * refcount drops to 0 stays cached and evictable; eviction takes the least
+ * recently released one.  Partly filled blocks are never cached.
+ *
+ * Determinism: a new block is the lowest-numbered free block; if none is
+ * free, the least recently released cached block is evicted (its key is
+ * dropped).  pkv_bm_free releases a sequence's blocks from its last block to
+ * its first, so a prefix outlives its own suffix in the LRU order.
+ *
+ * Every call validates first and changes nothing when it returns an error.
+ * ------------------------------------------------------------------------ */
+typedef struct pkv_block_manager pkv_block_manager;
+
+typedef struct pkv_bm_stats_t {
+  int32_t num_blocks;
+  int32_t free_blocks;         /* refcount 0 and not cached */
+  int32_t cached_idle_blocks;  /* refcount 0, cached, evictable (LRU list) */
+  int32_t used_blocks;         /* refcount > 0 */
+  int32_t cached_blocks;       /* blocks holding a prefix-cache key, used or idle */
+  int32_t sequences;
+  int64_t tokens;              /* sum of sequence lengths */
+  int64_t allocated_slots;     /* sum over sequences of table length * block_size */
+} pkv_bm_stats_t;
+
+/* Create a manager over blocks [0, num_blocks).  enable_prefix_cache != 0
+ * turns the hash-keyed prefix cache on.  *out is owned by the caller and
+ * released with pkv_bm_destroy. */
+pkv_status pkv_bm_create(int32_t num_blocks, int32_t block_size, int32_t enable_prefix_cache,
+                         pkv_block_manager** out);
+void pkv_bm_destroy(pkv_block_manager* bm);
+
+/* Chained block keys of a prompt: for every full block i of `tokens`
+ * (n_tokens / block_size of them), hashes[i] = FNV-1a 64 over the 8
+ * little-endian bytes of the previous key (seed for i = 0) followed by the
+ * block's tokens as little-endian int32.  hashes: host, n_tokens / block_size
+ * entries. */
+pkv_status pkv_bm_hash_blocks(const int32_t* tokens, int64_t n_tokens, int32_t block_size, uint64_t seed,
+                              uint64_t* hashes);
+
+/* Add a sequence holding n_prompt_tokens tokens (ceil(n / block_size)
+ * blocks).  block_hashes (host, n_prompt_tokens / block_size keys, or NULL)
+ * are the keys of its full blocks.  The leading run of keys found in the
+ * cache shares the cached blocks; the other blocks are new, and new full
+ * blocks are registered under their keys.  *n_cached_tokens (may be NULL)
+ * receives the shared prompt tokens, a multiple of block_size, whose K/V are
+ * already in the cache.  PKV_ERR_INVALID_ARG if seq_id exists. */
+pkv_status pkv_bm_add_sequence(pkv_block_manager* bm, int64_t seq_id, int64_t n_prompt_tokens,
+                               const uint64_t* block_hashes, int64_t* n_cached_tokens);
+
+/* New sequence `child` with the same tokens as `parent`, sharing every
+ * block of it (refcount + 1 each). */
+pkv_status pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t child);
+
+/* Reserve the slot of one new token for each of n distinct sequences, in
+ * order.  slot_mapping (host, int64 [n]) receives block * block_size +
+ * offset, ready for paged_kv_append.  cow_src / cow_dst (host, int32, room
+ * for n each) receive the copy-on-write pairs, *n_cow their count; copy them
+ * with paged_kv_copy_blocks before writing the new tokens.  Context lengths
+ * grow by one.  PKV_ERR_NO_BLOCKS if the pool cannot supply the new and
+ * copied blocks of the whole call. */
+pkv_status pkv_bm_append(pkv_block_manager* bm, const int64_t* seq_ids, int32_t n, int64_t* slot_mapping,
+                         int32_t* cow_src, int32_t* cow_dst, int32_t* n_cow);
+
+/* Drop a sequence and release its blocks (last block first). */
+pkv_status pkv_bm_free(pkv_block_manager* bm, int64_t seq_id);
+
+/* Export the block tables and context lengths of n sequences, row i for
+ * seq_ids[i]: block_tables (host, int32 [n][width], unused entries -1) and
+ * context_lens (host, int32 [n]).  PKV_ERR_INVALID_ARG if a table is longer
+ * than width or a sequence is unknown. */
+pkv_status pkv_bm_get_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int32_t n, int32_t width,
+                             int32_t* block_tables, int32_t* context_lens);
+
+/* Pool occupancy counters. */
+pkv_status pkv_bm_stats(const pkv_block_manager* bm, pkv_bm_stats_t* out);
+
+/* Refcount of one block. */
+pkv_status pkv_bm_refcount(const pkv_block_manager* bm, int32_t block, int32_t* refcount);
 
 /*
  * pkv_get_device_error -- synchronise `stream`, then read and clear the

@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "paged_kv_append", "paged_attention_decode", "paged_attention_decode_noalloc",
     "paged_attention_decode_cascade", "paged_attention_cascade_workspace_size",
-    "paged_attention_workspace_size",
+    "paged_attention_workspace_size", "paged_kv_copy_blocks", "BlockManager", "pkv_bm_hash_blocks",
     "pkv_get_device_error", "pkv_status_string", "pkv_version", "PagedKVError", "library_path",
     "DEVERR_BLOCK_ID", "DEVERR_CONTEXT", "DEVERR_SLOT", "DEVERR_TIMEOUT",
 ]
@@ -35,6 +35,7 @@ PKV_F32, PKV_F16, PKV_BF16 = 0, 1, 2
 _DTYPE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
 
 PKV_OK = 0
+PKV_ERR_INVALID_ARG, PKV_ERR_NO_BLOCKS = 1, 6
 DEVERR_BLOCK_ID, DEVERR_CONTEXT, DEVERR_SLOT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 
@@ -47,6 +48,13 @@ class PagedKVError(RuntimeError):
 class _Options(ctypes.Structure):
     _fields_ = [("num_units", ctypes.c_int32), ("force_simt", ctypes.c_int32),
                 ("reserved", ctypes.c_int32 * 6)]
+
+
+class _BMStats(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("free_blocks", ctypes.c_int32),
+                ("cached_idle_blocks", ctypes.c_int32), ("used_blocks", ctypes.c_int32),
+                ("cached_blocks", ctypes.c_int32), ("sequences", ctypes.c_int32),
+                ("tokens", ctypes.c_int64), ("allocated_slots", ctypes.c_int64)]
 
 
 _lib = None
@@ -87,6 +95,23 @@ def _load() -> ctypes.CDLL:
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_version.argtypes = []
     lib.pkv_version.restype = ctypes.c_int32
+    lib.paged_kv_copy_blocks.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p]
+    lib.paged_kv_copy_blocks.restype = ctypes.c_int
+    i64, u64 = ctypes.c_int64, ctypes.c_uint64
+    for name, args in (("pkv_bm_create", [i32, i32, i32, ctypes.POINTER(p)]),
+                       ("pkv_bm_hash_blocks", [p, i64, i32, u64, p]),
+                       ("pkv_bm_add_sequence", [p, i64, i64, p, ctypes.POINTER(i64)]),
+                       ("pkv_bm_fork", [p, i64, i64]),
+                       ("pkv_bm_append", [p, p, i32, p, p, p, ctypes.POINTER(i32)]),
+                       ("pkv_bm_free", [p, i64]),
+                       ("pkv_bm_get_tables", [p, p, i32, i32, p, p]),
+                       ("pkv_bm_stats", [p, ctypes.POINTER(_BMStats)]),
+                       ("pkv_bm_refcount", [p, i32, ctypes.POINTER(i32)])):
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.pkv_bm_destroy.argtypes = [p]
+    lib.pkv_bm_destroy.restype = None
     _lib = lib
     return lib
 
@@ -238,3 +263,119 @@ def pkv_get_device_error(stream=None) -> int:
     if st not in (PKV_OK, 3):
         raise PagedKVError(st, "pkv_get_device_error")
     return int(flags.value)
+
+
+def paged_kv_copy_blocks(k_cache, v_cache, src_blocks, dst_blocks, block_size: int = 16, stream=None) -> None:
+    """Copy whole blocks ``src_blocks[p] -> dst_blocks[p]`` in both caches
+    (the copy of copy-on-write)."""
+    lib = _load()
+    num_blocks, n_kv, bs, d = k_cache.shape
+    if bs != block_size or tuple(v_cache.shape) != tuple(k_cache.shape) or v_cache.dtype != k_cache.dtype:
+        raise ValueError("cache shapes disagree")
+    if src_blocks.dtype != torch.int32 or dst_blocks.dtype != torch.int32 or src_blocks.shape != dst_blocks.shape:
+        raise ValueError("src_blocks and dst_blocks must be int32 of one shape")
+    n = src_blocks.numel()
+    if n == 0:
+        return
+    _check(lib.paged_kv_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                    _dev(src_blocks, "src_blocks"), _dev(dst_blocks, "dst_blocks"), n,
+                                    num_blocks, bs, n_kv, d, _DTYPE[k_cache.dtype], _stream(stream)),
+           "paged_kv_copy_blocks")
+
+
+def _host(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
+    t = torch.as_tensor(t, dtype=dtype)
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    return t.contiguous()
+
+
+def pkv_bm_hash_blocks(tokens, block_size: int = 16, seed: int = 0) -> list[int]:
+    """Chained FNV-1a keys of the full blocks of a prompt (host call)."""
+    t = _host(tokens, torch.int32, "tokens").reshape(-1)
+    n = t.numel() // block_size
+    out = (ctypes.c_uint64 * max(n, 1))()
+    _check(_load().pkv_bm_hash_blocks(t.data_ptr() if t.numel() else None, t.numel(), block_size,
+                                      ctypes.c_uint64(seed & (2**64 - 1)), out), "pkv_bm_hash_blocks")
+    return [int(out[i]) for i in range(n)]
+
+
+class BlockManager:
+    """Host block manager of the pool (C++ behind the pkv_bm_* entry points):
+    free pool, per-sequence block tables, refcounted fork with copy-on-write
+    of a shared last block, and an optional hash-keyed prefix cache with LRU
+    eviction.  Everything runs on the host; the outputs feed
+    paged_kv_copy_blocks, paged_kv_append and the decode entry points."""
+
+    def __init__(self, num_blocks: int, block_size: int = 16, prefix_cache: bool = False):
+        self._lib = _load()
+        h = ctypes.c_void_p()
+        _check(self._lib.pkv_bm_create(num_blocks, block_size, int(bool(prefix_cache)), ctypes.byref(h)),
+               "pkv_bm_create")
+        self._h = h
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def add_sequence(self, seq_id: int, n_prompt_tokens: int, block_hashes=None) -> int:
+        """Returns the number of prompt tokens found in the prefix cache."""
+        cached = ctypes.c_int64(0)
+        arr = None
+        if block_hashes is not None and len(block_hashes):
+            arr = (ctypes.c_uint64 * len(block_hashes))(*[int(x) & (2**64 - 1) for x in block_hashes])
+        _check(self._lib.pkv_bm_add_sequence(self._h, seq_id, n_prompt_tokens, arr, ctypes.byref(cached)),
+               "pkv_bm_add_sequence")
+        return int(cached.value)
+
+    def fork(self, parent: int, child: int) -> None:
+        _check(self._lib.pkv_bm_fork(self._h, parent, child), "pkv_bm_fork")
+
+    def append(self, seq_ids):
+        """One new token for each sequence: returns (slot_mapping int64,
+        cow_src int32, cow_dst int32), host tensors."""
+        ids = _host(seq_ids, torch.int64, "seq_ids").reshape(-1)
+        n = ids.numel()
+        slots = torch.empty(n, dtype=torch.int64)
+        src = torch.empty(max(n, 1), dtype=torch.int32)
+        dst = torch.empty(max(n, 1), dtype=torch.int32)
+        ncow = ctypes.c_int32(0)
+        _check(self._lib.pkv_bm_append(self._h, ids.data_ptr() if n else None, n,
+                                       slots.data_ptr() if n else None, src.data_ptr(), dst.data_ptr(),
+                                       ctypes.byref(ncow)), "pkv_bm_append")
+        k = ncow.value
+        return slots, src[:k].clone(), dst[:k].clone()
+
+    def free(self, seq_id: int) -> None:
+        _check(self._lib.pkv_bm_free(self._h, seq_id), "pkv_bm_free")
+
+    def tables(self, seq_ids, width: int):
+        """(block_tables int32 [n, width] with -1 padding, context_lens int32 [n]) on the host."""
+        ids = _host(seq_ids, torch.int64, "seq_ids").reshape(-1)
+        n = ids.numel()
+        bt = torch.empty((n, width), dtype=torch.int32)
+        cl = torch.empty(n, dtype=torch.int32)
+        if n:
+            _check(self._lib.pkv_bm_get_tables(self._h, ids.data_ptr(), n, width, bt.data_ptr(), cl.data_ptr()),
+                   "pkv_bm_get_tables")
+        return bt, cl
+
+    def stats(self) -> dict:
+        st = _BMStats()
+        _check(self._lib.pkv_bm_stats(self._h, ctypes.byref(st)), "pkv_bm_stats")
+        return {name: int(getattr(st, name)) for name, _ in _BMStats._fields_}
+
+    def refcount(self, block: int) -> int:
+        rc = ctypes.c_int32(0)
+        _check(self._lib.pkv_bm_refcount(self._h, block, ctypes.byref(rc)), "pkv_bm_refcount")
+        return int(rc.value)

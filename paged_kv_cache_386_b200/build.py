@@ -16,7 +16,7 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libpagedkv.so"
-SOURCES = [CSRC / "pkv_api.cu"]
+SOURCES = [CSRC / "pkv_api.cu", CSRC / "pkv_block_manager.cpp"]
 HEADERS = sorted(CSRC.glob("*.cuh")) + [ROOT / "include" / "pagedkv.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

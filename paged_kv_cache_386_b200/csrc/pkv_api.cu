@@ -229,6 +229,8 @@ const char* pkv_status_string(pkv_status s) {
     case PKV_ERR_OUT_OF_RANGE: return "a kernel saw an out-of-range block id, context length or slot";
     case PKV_ERR_CUDA: return "CUDA runtime error";
     case PKV_ERR_WORKSPACE: return "workspace too small";
+    case PKV_ERR_NO_BLOCKS: return "not enough free or evictable blocks";
+    case PKV_ERR_HOST_MEMORY: return "host allocation failed";
     default: return "unknown status";
   }
 }
@@ -260,6 +262,34 @@ pkv_status paged_kv_append(const void* k, const void* v, const int64_t* slot_map
   const int64_t want = (p.total + 255) / 256;
   const int grid = static_cast<int>(want < int64_t(di.sm_count) * 8 ? want : int64_t(di.sm_count) * 8);
   pkv_append_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status paged_kv_copy_blocks(void* k_cache, void* v_cache, const int32_t* src_blocks, const int32_t* dst_blocks,
+                                int32_t n_pairs, int32_t num_blocks, int32_t block_size, int32_t n_kv_heads,
+                                int32_t head_dim, pkv_dtype dtype, void* stream) {
+  if (n_pairs < 0 || num_blocks <= 0 || block_size <= 0 || n_kv_heads <= 0 || head_dim <= 0)
+    return PKV_ERR_INVALID_ARG;
+  const int es = elem_bytes(dtype);
+  if (es == 0 || block_size != kBlockTokens || (head_dim * es) % 16 != 0) return PKV_ERR_UNSUPPORTED;
+  if (n_pairs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !src_blocks || !dst_blocks || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(src_blocks) & 3u) || (reinterpret_cast<uintptr_t>(dst_blocks) & 3u))
+    return PKV_ERR_INVALID_ARG;
+  const int64_t chunks = static_cast<int64_t>(n_kv_heads) * block_size * head_dim * es / 16;
+  if (chunks > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  CopyParams p;
+  p.k_cache = static_cast<uint8_t*>(k_cache);
+  p.v_cache = static_cast<uint8_t*>(v_cache);
+  p.src = src_blocks;
+  p.dst = dst_blocks;
+  p.n_pairs = n_pairs;
+  p.num_blocks = num_blocks;
+  p.chunks = static_cast<int32_t>(chunks);
+  const int grid = n_pairs < di.sm_count * 8 ? n_pairs : di.sm_count * 8;
+  pkv_copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

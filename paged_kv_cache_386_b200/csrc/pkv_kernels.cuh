@@ -1,5 +1,6 @@
 // pkv_kernels.cuh -- sm_100a kernels of the paged KV cache:
 //   pkv_append_kernel   scatter of new K/V rows into their slots
+//   pkv_copy_blocks_kernel  whole-block copies for copy-on-write
 //   pkv_decode_kernel   persistent split-KV paged decode attention, with the
 //                       log-sum-exp merge of split contexts after a grid-wide
 //                       barrier
@@ -106,6 +107,52 @@ __global__ void __launch_bounds__(256) pkv_append_kernel(const AppendParams p) {
     const int4 vv = __ldg(reinterpret_cast<const int4*>(p.v + src));
     *reinterpret_cast<int4*>(p.k_cache + dst) = kv;
     *reinterpret_cast<int4*>(p.v_cache + dst) = vv;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Block copy (copy-on-write of shared blocks)
+// ---------------------------------------------------------------------------
+struct CopyParams {
+  uint8_t* k_cache;
+  uint8_t* v_cache;
+  const int32_t* src;
+  const int32_t* dst;
+  int32_t n_pairs;
+  int32_t num_blocks;
+  int32_t chunks;  // 16-byte chunks per block of one cache
+};
+
+// CTAs stride over the pairs; the threads of a CTA stream one block of K and
+// one of V, four 16-byte loads in flight per thread before the stores.
+__global__ void __launch_bounds__(256) pkv_copy_blocks_kernel(const CopyParams p) {
+  for (int pair = blockIdx.x; pair < p.n_pairs; pair += gridDim.x) {
+    const int32_t s = __ldg(p.src + pair), d = __ldg(p.dst + pair);
+    if (s < 0 || s >= p.num_blocks || d < 0 || d >= p.num_blocks) {
+      if (threadIdx.x == 0) flag_error(PKV_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const int64_t so = static_cast<int64_t>(s) * p.chunks, dof = static_cast<int64_t>(d) * p.chunks;
+    const int4* ks = reinterpret_cast<const int4*>(p.k_cache) + so;
+    const int4* vs = reinterpret_cast<const int4*>(p.v_cache) + so;
+    int4* kd = reinterpret_cast<int4*>(p.k_cache) + dof;
+    int4* vd = reinterpret_cast<int4*>(p.v_cache) + dof;
+    for (int c0 = threadIdx.x; c0 < p.chunks; c0 += 2 * blockDim.x) {
+      const int c1 = c0 + blockDim.x;
+      const bool two = c1 < p.chunks;
+      const int4 a = ks[c0], b = vs[c0];
+      int4 e = make_int4(0, 0, 0, 0), f = e;
+      if (two) {
+        e = ks[c1];
+        f = vs[c1];
+      }
+      kd[c0] = a;
+      vd[c0] = b;
+      if (two) {
+        kd[c1] = e;
+        vd[c1] = f;
+      }
+    }
   }
 }
 

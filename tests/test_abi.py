@@ -32,7 +32,9 @@ def test_header_declares_expected_entry_points():
     names = set(declared_functions())
     assert {"paged_kv_append", "paged_attention_decode", "paged_attention_decode_ex",
             "paged_attention_workspace_size", "pkv_get_device_error", "pkv_status_string",
-            "pkv_version"} <= names
+            "pkv_version", "paged_kv_copy_blocks", "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_hash_blocks",
+            "pkv_bm_add_sequence", "pkv_bm_fork", "pkv_bm_append", "pkv_bm_free", "pkv_bm_get_tables",
+            "pkv_bm_stats", "pkv_bm_refcount"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -41,7 +43,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for s in range(6):
+    for s in range(8):
         assert pkv.pkv_status_string(s)
     assert pkv.pkv_status_string(99) == "unknown status"
     assert pkv.pkv_version() >= 10000
@@ -94,6 +96,16 @@ def test_append_host_validation(lib):
     assert f(None, None, None, 0, None, None, 8, 16, 2, 128, 2, None) == 0
     assert f(None, None, None, 4, None, None, 8, 16, 2, 128, 2, None) == INVALID
     assert f(16, 32, 4, 4, 64, 128, 8, 16, 2, 128, 2, None) == INVALID   # slot_mapping misaligned
+
+
+def test_copy_blocks_host_validation(lib):
+    f = lib.paged_kv_copy_blocks
+    assert f(None, None, None, None, -1, 8, 16, 2, 128, 2, None) == INVALID
+    assert f(None, None, None, None, 4, 8, 32, 2, 128, 2, None) == UNSUPPORTED
+    assert f(None, None, None, None, 4, 8, 16, 2, 128, 7, None) == UNSUPPORTED
+    assert f(None, None, None, None, 0, 8, 16, 2, 128, 2, None) == 0
+    assert f(None, None, None, None, 4, 8, 16, 2, 128, 2, None) == INVALID
+    assert f(16, 32, 2, 64, 4, 8, 16, 2, 128, 2, None) == INVALID       # src_blocks misaligned
 
 
 def test_workspace_size_validation(lib):
