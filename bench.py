@@ -198,10 +198,10 @@ def run_ours(args) -> None:
         cv = W.cascade_view(w)
         c_pt, c_pl, c_sg, c_bt, c_cl = (t.to(dev) for t in (cv.prefix_block_tables, cv.prefix_lens, cv.seq_group,
                                                              cv.block_tables, cv.context_lens))
-        ws = torch.empty(pkv.paged_attention_cascade_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
+        ws = torch.zeros(pkv.paged_attention_cascade_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
                                                                     w.dtype), dtype=torch.uint8, device=dev)
     else:
-        ws = torch.empty(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
+        ws = torch.zeros(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
                                                             w.dtype), dtype=torch.uint8, device=dev)
 
     def decode(stream_=None):

@@ -80,6 +80,8 @@ typedef enum pkv_status {
 #define PKV_DEVERR_CONTEXT 0x2u    /* context length < 0 or > max_blocks_per_seq * block_size: clamped */
 #define PKV_DEVERR_SLOT 0x4u       /* slot >= num_blocks * block_size: the token was not written */
 #define PKV_DEVERR_TIMEOUT 0x8u    /* a bounded in-kernel wait (2 s) gave up: that launch wrote no result */
+#define PKV_DEVERR_SCHEDULE 0x10u  /* the decode workspace was not zero-filled before its first use: that
+                                      launch's result is wrong (the workspace is zeroed again) */
 
 /*
  * paged_kv_append -- write the K/V of new tokens into their cache slots.
@@ -112,6 +114,14 @@ pkv_status paged_kv_append(const void* k, const void* v, const int64_t* slot_map
 pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
                                           int32_t head_dim, pkv_dtype dtype, size_t* bytes);
 
+typedef struct pkv_decode_options pkv_decode_options;
+
+/* The same for paged_attention_decode_ex with `options` (NULL = defaults):
+ * balancing chunks need (1 + balance_chunks) times the records. */
+pkv_status paged_attention_workspace_size_ex(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                             int32_t head_dim, pkv_dtype dtype,
+                                             const pkv_decode_options* options, size_t* bytes);
+
 /*
  * paged_attention_decode -- single-query attention through the block table.
  *
@@ -132,9 +142,14 @@ pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int3
  *
  *   workspace     : device scratch of at least paged_attention_workspace_size()
  *                   bytes, 256-byte aligned, owned by the caller and not
- *                   shared by two calls in flight at once; NULL makes the
- *                   library take a stream-ordered allocation for this call
- *                   (cudaMallocAsync / cudaFreeAsync on `stream`)
+ *                   shared by two calls in flight at once.  Used with
+ *                   balancing chunks (paged_attention_decode_ex), it must be
+ *                   zero-filled before its first use; every call leaves it
+ *                   ready for the next (one that was not cleared gives a
+ *                   wrong result for that call and sets PKV_DEVERR_SCHEDULE).
+ *                   NULL makes the library take a stream-ordered allocation
+ *                   for this call (cudaMallocAsync / cudaFreeAsync on
+ *                   `stream`)
  *   workspace_bytes : size of `workspace`
  */
 pkv_status paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -184,13 +199,20 @@ pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, co
                                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* Tuning and test hooks for paged_attention_decode_ex. Zero-initialise. */
-typedef struct pkv_decode_options {
+struct pkv_decode_options {
   int32_t num_units;   /* 0: default split (one work unit per consumer warp on every SM);
                           n > 0: use at most n work units (n = 1 computes every row in one
                           unit, with no split and no merge) */
   int32_t force_simt;  /* 1: CUDA-core path even where the tensor-core path applies */
-  int32_t reserved[6]; /* must be zero */
-} pkv_decode_options;
+  int32_t balance_chunks;  /* 0: none (default: every unit runs exactly its own tile range);
+                              1..4: balancing chunks cut from the end of each unit's range and
+                              claimed at run time by the first warps to run out of work.  The
+                              result stays deterministic.  Needs the larger workspace of
+                              paged_attention_workspace_size_ex, zero-filled before first use.
+                              Measured on B200 it costs more than the imbalance it removes */
+  int32_t static_permille; /* 0: default (800); 500..999: share of its range a unit keeps */
+  int32_t reserved[4]; /* must be zero */
+};
 
 /* paged_attention_decode with options (NULL options = paged_attention_decode). */
 pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const void* v_cache,
@@ -217,17 +239,17 @@ pkv_status paged_attention_decode_ex(const void* q, const void* k_cache, const v
  * of PKV_STATIC_WORKSPACE_BYTES (24 MiB), which every GPU that loads the
  * library holds until the process exits.
  *
- * - Sizes whose scratch (paged_attention_workspace_size) exceeds the array are
- *   rejected with PKV_ERR_WORKSPACE before anything is enqueued.  On a 148-SM
- *   B200 every supported shape fits.
+ * - Sizes whose scratch (paged_attention_workspace_size) exceeds the array
+ *   are rejected with PKV_ERR_WORKSPACE before anything is enqueued.  On a
+ *   148-SM B200 every supported shape fits.
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current and caches it; make that
  *   first call before any stream capture.
  * - Every call on a device shares the one array and it keeps the last call's
- *   contents.  Nothing in it has to start at zero: each call rewrites the
- *   per-unit metadata before its merge reads any record.  Calls whose work
- *   overlaps on the GPU (on different streams, or from several host threads
- *   without ordering) race on the array and give wrong results: order them.
+ *   contents.  The array starts zero-filled and every call leaves its
+ *   scheduling counter at zero again.  Calls whose work overlaps on the GPU
+ *   (on different streams, or from several host threads without ordering)
+ *   race on the array and give wrong results: order them.
  * Results are bit-identical to paged_attention_decode with its default split.
  */
 #define PKV_STATIC_WORKSPACE_BYTES (24u * 1024u * 1024u)

@@ -26,7 +26,7 @@ __all__ = [
     "paged_attention_decode_cascade", "paged_attention_cascade_workspace_size",
     "paged_attention_workspace_size", "paged_kv_copy_blocks", "BlockManager", "pkv_bm_hash_blocks",
     "pkv_get_device_error", "pkv_status_string", "pkv_version", "PagedKVError", "library_path",
-    "DEVERR_BLOCK_ID", "DEVERR_CONTEXT", "DEVERR_SLOT", "DEVERR_TIMEOUT",
+    "DEVERR_BLOCK_ID", "DEVERR_CONTEXT", "DEVERR_SLOT", "DEVERR_TIMEOUT", "DEVERR_SCHEDULE", "new_workspace",
 ]
 
 _LIB_PATH = Path(__file__).resolve().parent / "libpagedkv.so"
@@ -36,7 +36,7 @@ _DTYPE = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF
 
 PKV_OK = 0
 PKV_ERR_INVALID_ARG, PKV_ERR_NO_BLOCKS = 1, 6
-DEVERR_BLOCK_ID, DEVERR_CONTEXT, DEVERR_SLOT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEVERR_BLOCK_ID, DEVERR_CONTEXT, DEVERR_SLOT, DEVERR_TIMEOUT, DEVERR_SCHEDULE = 0x1, 0x2, 0x4, 0x8, 0x10
 
 
 class PagedKVError(RuntimeError):
@@ -47,7 +47,8 @@ class PagedKVError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("num_units", ctypes.c_int32), ("force_simt", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("balance_chunks", ctypes.c_int32), ("static_permille", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
 
 
 class _BMStats(ctypes.Structure):
@@ -77,6 +78,9 @@ def _load() -> ctypes.CDLL:
     lib.paged_kv_append.restype = ctypes.c_int
     lib.paged_attention_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(sz)]
     lib.paged_attention_workspace_size.restype = ctypes.c_int
+    lib.paged_attention_workspace_size_ex.argtypes = [i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(_Options),
+                                                      ctypes.POINTER(sz)]
+    lib.paged_attention_workspace_size_ex.restype = ctypes.c_int
     dec = [p, p, p, p, i32, p, i32, i32, f32, i32, i32, i32, i32, p, ctypes.c_int, p, sz, p]
     lib.paged_attention_decode.argtypes = dec
     lib.paged_attention_decode.restype = ctypes.c_int
@@ -158,18 +162,28 @@ def paged_kv_append(k, v, slot_mapping, k_cache, v_cache, block_size: int = 16, 
 
 
 def paged_attention_workspace_size(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
-                                   dtype: torch.dtype) -> int:
+                                   dtype: torch.dtype, balance_chunks: int = 0) -> int:
     out = ctypes.c_size_t(0)
-    _check(_load().paged_attention_workspace_size(batch, n_q_heads, n_kv_heads, head_dim,
-                                                  _DTYPE[dtype], ctypes.byref(out)),
+    opts = _Options(balance_chunks=int(balance_chunks))
+    _check(_load().paged_attention_workspace_size_ex(batch, n_q_heads, n_kv_heads, head_dim,
+                                                     _DTYPE[dtype], ctypes.byref(opts), ctypes.byref(out)),
            "paged_attention_workspace_size")
     return int(out.value)
 
 
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A decode workspace: zero-filled device bytes, as the library requires
+    before a workspace's first use (each call leaves it ready for the next)."""
+    return torch.zeros(int(nbytes), dtype=torch.uint8, device=device or "cuda")
+
+
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out=None,
                            workspace=None, num_units: int = 0, force_simt: bool = False,
+                           balance_chunks: int = 0, static_permille: int = 0,
                            block_size: int = 16, stream=None):
-    """Single-query attention through the block table; returns ``out``."""
+    """Single-query attention through the block table; returns ``out``.
+    With ``balance_chunks`` > 0 the workspace (see new_workspace) must be
+    zero-filled before its first use."""
     lib = _load()
     B, n_q, d = q.shape
     num_blocks, n_kv, bs, d2 = k_cache.shape
@@ -182,7 +196,8 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
-    opts = _Options(num_units=int(num_units), force_simt=int(bool(force_simt)))
+    opts = _Options(num_units=int(num_units), force_simt=int(bool(force_simt)),
+                    balance_chunks=int(balance_chunks), static_permille=int(static_permille))
     _check(lib.paged_attention_decode_ex(
         _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),

@@ -75,12 +75,18 @@ int heads_per_segment(int group, pkv_dtype dt, bool force_simt) {
 
 int record_floats(int gp, int head_dim) { return (gp * (head_dim + 2) + 3) & ~3; }
 
-size_t meta_bytes(int units) { return (static_cast<size_t>(units) * sizeof(int4) + 255) & ~static_cast<size_t>(255); }
+size_t meta_bytes(int chunks) { return (static_cast<size_t>(chunks) * sizeof(int4) + 255) & ~static_cast<size_t>(255); }
 
-// Per work unit: one metadata entry and two partial-softmax records (its
-// first and last segment).
-size_t workspace_for(int units, int gp, int head_dim) {
-  return meta_bytes(units) + static_cast<size_t>(units) * 2 * record_floats(gp, head_dim) * sizeof(float);
+constexpr int kDefaultSubChunks = 0;  // balancing chunks cost more than they recover on B200
+constexpr int kDefaultStaticPermille = 800;
+constexpr size_t kSchedBytes = 256;  // claim counter of the balancing chunks
+
+// Workspace: the claim counter, then per chunk (units x (1 + sub_chunks)) one
+// metadata entry and two partial-softmax records (its first and last
+// segment).
+size_t workspace_for(int units, int sub_chunks, int gp, int head_dim) {
+  const size_t chunks = static_cast<size_t>(units) * (1 + sub_chunks);
+  return kSchedBytes + meta_bytes(static_cast<int>(chunks)) + chunks * 2 * record_floats(gp, head_dim) * sizeof(float);
 }
 
 struct DecodeShape {
@@ -295,6 +301,11 @@ pkv_status paged_kv_copy_blocks(void* k_cache, void* v_cache, const int32_t* src
 
 pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                           pkv_dtype dtype, size_t* bytes) {
+  return paged_attention_workspace_size_ex(batch, n_q_heads, n_kv_heads, head_dim, dtype, nullptr, bytes);
+}
+
+pkv_status paged_attention_workspace_size_ex(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                             pkv_dtype dtype, const pkv_decode_options* options, size_t* bytes) {
   if (!bytes || batch < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0 || head_dim <= 0)
     return PKV_ERR_INVALID_ARG;
   if (elem_bytes(dtype) == 0 || (head_dim != 64 && head_dim != 128)) return PKV_ERR_UNSUPPORTED;
@@ -302,7 +313,9 @@ pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int3
   if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
   // Sized for the widest head group so that force_simt never needs more.
   const int gp = heads_per_segment(n_q_heads / n_kv_heads, dtype, false);
-  *bytes = workspace_for(di.sm_count * kConsumerWarps, gp, head_dim);
+  const int sub = (options && options->balance_chunks > 0) ? options->balance_chunks : kDefaultSubChunks;
+  if (sub > 4) return PKV_ERR_INVALID_ARG;
+  *bytes = workspace_for(di.sm_count * kConsumerWarps, sub, gp, head_dim);
   return PKV_OK;
 }
 
@@ -325,10 +338,15 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   pkv_decode_options opt = {};
   if (options) {
     opt = *options;
-    for (int i = 0; i < 6; ++i)
+    for (int i = 0; i < 4; ++i)
       if (opt.reserved[i] != 0) return PKV_ERR_INVALID_ARG;
     if (opt.num_units < 0 || (opt.force_simt != 0 && opt.force_simt != 1)) return PKV_ERR_INVALID_ARG;
+    if (opt.balance_chunks < 0 || opt.balance_chunks > 4) return PKV_ERR_INVALID_ARG;
+    if (opt.static_permille != 0 && (opt.static_permille < 500 || opt.static_permille > 999))
+      return PKV_ERR_INVALID_ARG;
   }
+  const int sub_chunks = opt.balance_chunks == 0 ? kDefaultSubChunks : opt.balance_chunks;
+  const int static_permille = opt.static_permille == 0 ? kDefaultStaticPermille : opt.static_permille;
   DeviceInfo di;
   if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -352,18 +370,22 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   const size_t qbuf_bytes = static_cast<size_t>(gpad == 0 ? 1 : gpad) * head_dim * es;
   const size_t fixed =
       1024 + kConsumerWarps * qbuf_bytes + 16 + static_cast<size_t>(2 * batch + 1) * sizeof(int) + 256;
-  const size_t per_round = kConsumerWarps * (stage_bytes + 2 * sizeof(uint64_t));
+  const size_t per_round = kConsumerWarps * (stage_bytes + 2 * sizeof(uint64_t) + 4 * sizeof(int));
   if (fixed + per_round > static_cast<size_t>(di.smem_optin)) return PKV_ERR_UNSUPPORTED;
   int stages = static_cast<int>((di.smem_optin - fixed) / per_round);
   if (stages > 4) stages = 4;
   const size_t smem = fixed - 256 + stages * per_round;
 
-  const size_t need = workspace_for(units, gp, head_dim);
+  const size_t need = workspace_for(units, sub_chunks, gp, head_dim);
   void* ws = workspace;
   bool own = false;
   if (ws == nullptr) {
     if (cudaMallocAsync(&ws, need, s) != cudaSuccess) return PKV_ERR_CUDA;
     own = true;
+    if (cudaMemsetAsync(ws, 0, kSchedBytes, s) != cudaSuccess) {
+      cudaFreeAsync(ws, s);
+      return PKV_ERR_CUDA;
+    }
   } else if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
     return PKV_ERR_WORKSPACE;
   }
@@ -377,8 +399,10 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   p.out = out;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
-  p.meta = static_cast<int4*>(ws);
-  p.records = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + meta_bytes(units));
+  const int chunks = units * (1 + sub_chunks);
+  p.sched = static_cast<int*>(ws);
+  p.meta = reinterpret_cast<int4*>(static_cast<uint8_t*>(ws) + kSchedBytes);
+  p.records = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kSchedBytes + meta_bytes(chunks));
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.batch = batch;
   p.num_blocks = num_blocks;
@@ -387,6 +411,8 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   p.gp = gp;
   p.ng = n_q_heads / gp;
   p.num_units = units;
+  p.sub_chunks = sub_chunks;
+  p.static_permille = static_permille;
   p.stages = stages;
   p.rec_floats = record_floats(gp, head_dim);
   p.head_dim = head_dim;
@@ -467,10 +493,12 @@ pkv_status paged_attention_decode_noalloc(const void* q, const void* k_cache, co
   pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                     num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
   if (st != PKV_OK || batch == 0) return st;
-  size_t need = 0;
-  st = paged_attention_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, dtype, &need);
-  if (st != PKV_OK) return st;
-  if (need > PKV_STATIC_WORKSPACE_BYTES) return PKV_ERR_WORKSPACE;  // beyond the static maximum
+  if (n_q_heads % n_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  const int gp = heads_per_segment(n_q_heads / n_kv_heads, dtype, false);
+  if (workspace_for(di.sm_count * kConsumerWarps, kDefaultSubChunks, gp, head_dim) > PKV_STATIC_WORKSPACE_BYTES)
+    return PKV_ERR_WORKSPACE;
   void* ws = nullptr;
   st = static_workspace(&ws);
   if (st != PKV_OK) return st;
@@ -516,13 +544,18 @@ pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, co
   if (st != PKV_OK) return st;
   void* ws = workspace;
   bool own = false;
+  const size_t init_bytes = prefix_init_bytes(batch, n_q_heads, head_dim);
   if (ws == nullptr) {
     if (cudaMallocAsync(&ws, need, s) != cudaSuccess) return PKV_ERR_CUDA;
     own = true;
+    // The decode part's scheduling counter starts at zero.
+    if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + init_bytes, 0, kSchedBytes, s) != cudaSuccess) {
+      cudaFreeAsync(ws, s);
+      return PKV_ERR_CUDA;
+    }
   } else if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
     return PKV_ERR_WORKSPACE;
   }
-  const size_t init_bytes = prefix_init_bytes(batch, n_q_heads, head_dim);
   float* init = static_cast<float*>(ws);
 
   CUtensorMap mk, mv;

@@ -51,6 +51,8 @@ constexpr int kConsumerWarps = 10;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kBoxBytes = 16 * 128;  // one TMA box: 16 tokens x 128 bytes
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Tiles before a chunk's end at which its producer lane claims the next chunk.
+constexpr int kClaimAhead = 3;
 
 enum DType { kF32 = 0, kF16 = 1, kBF16 = 2 };
 
@@ -164,8 +166,9 @@ struct DecodeParams {
   void* out;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  float* records;  // [num_units][2][rec_floats]: O[gp][D], m[gp], l[gp]
-  int4* meta;      // [num_units]: split segment whose first piece the unit holds
+  float* records;  // [chunks][2][rec_floats]: O[gp][D], m[gp], l[gp]
+  int4* meta;      // [chunks]: split segment whose first piece the chunk holds
+  int* sched;      // [0]: claim counter of the balancing chunks (0 between launches)
   // Optional initial softmax state per (sequence, query head) -- the shared
   // prefix part of a cascade decode: O [batch][n_q][D] unnormalised, then
   // m [batch][n_q] (log2 units), then l [batch][n_q].  Used for sequences with
@@ -181,6 +184,8 @@ struct DecodeParams {
   int32_t gp;          // query heads per segment
   int32_t ng;          // segments per sequence (n_q_heads / gp)
   int32_t num_units;
+  int32_t sub_chunks;      // balancing chunks cut from the end of each unit's range (0..4)
+  int32_t static_permille; // share of each unit's range that the unit keeps
   int32_t stages;      // ring slots per consumer warp
   int32_t rec_floats;  // floats per partial record: gp * (head_dim + 2), rounded up to 4
   int32_t head_dim;
@@ -242,12 +247,95 @@ __device__ __forceinline__ void walk_next(Walk& w, const int* prefix, const int*
   }
 }
 
-__device__ __forceinline__ int unit_of_tile(int k, int T, int U) {
-  return static_cast<int>(((static_cast<int64_t>(k) + 1) * U - 1) / T);
+// Work partition.  The T tiles are cut into U units of Lq = T / U tiles,
+// the first r = T % U of them one tile longer, so that the boundaries need no
+// division.  Unit u's range [a, a + L) is cut into chunk u * (M + 1) (its
+// first S = L * static_permille / 1000 tiles, run by unit u's own warp) and M
+// balancing chunks that split the other D = L - S tiles in the ratio
+// M : M-1 : ... : 1.  Balancing chunks are claimed at run time through an
+// atomic counter, largest first over all units, by the producer lanes whose
+// warps run out of work first.  Chunk boundaries depend only on (T, U, M, S),
+// so the result does not depend on which warp runs a chunk.  Chunk ids
+// follow tile order.
+struct Sched {
+  int U, M, Lq, r;
+  int Sq, Dq, Sr, Dr;  // S and D of units of Lq tiles and of Lq + 1 tiles
+};
+
+__device__ __forceinline__ int sub_cum(int i, int M) { return i * (2 * M + 1 - i) / 2; }
+
+// x / (M (M + 1) / 2) with a constant divisor per case.
+__device__ __forceinline__ int div_sub_weight(int64_t x, int M) {
+  switch (M) {
+    case 1: return static_cast<int>(x);
+    case 2: return static_cast<int>(x / 3);
+    case 3: return static_cast<int>(x / 6);
+    default: return static_cast<int>(x / 10);
+  }
 }
 
-__device__ __forceinline__ int unit_begin(int u, int T, int U) {
-  return static_cast<int>(static_cast<int64_t>(u) * T / U);
+__device__ __forceinline__ int div_small(int x, int d) {  // d in 1..5
+  switch (d) {
+    case 1: return x;
+    case 2: return x / 2;
+    case 3: return x / 3;
+    case 4: return x / 4;
+    default: return x / 5;
+  }
+}
+
+__device__ __forceinline__ Sched make_sched(int T, int num_units, int M, int fpm) {
+  Sched sc;
+  sc.U = min(num_units, max(T, 1));  // at most one unit per tile: no unit is empty
+  sc.Lq = T / sc.U;
+  sc.r = T - sc.Lq * sc.U;
+  sc.Sq = static_cast<int>(static_cast<int64_t>(sc.Lq) * fpm / 1000);
+  sc.Dq = sc.Lq - sc.Sq;
+  sc.Sr = static_cast<int>(static_cast<int64_t>(sc.Lq + 1) * fpm / 1000);
+  sc.Dr = sc.Lq + 1 - sc.Sr;
+  // Balancing chunks only when every chunk of every unit gets a tile.
+  sc.M = (M > 0 && sc.Sq >= 1 && sc.Dq >= M * (M + 1) / 2) ? M : 0;
+  return sc;
+}
+
+__device__ __forceinline__ int unit_begin(const Sched& sc, int u) { return u * sc.Lq + min(u, sc.r); }
+
+__device__ __forceinline__ int unit_of_tile(const Sched& sc, int k) {
+  const int edge = sc.r * (sc.Lq + 1);
+  return k < edge ? k / (sc.Lq + 1) : sc.r + (k - edge) / sc.Lq;
+}
+
+__device__ __forceinline__ void chunk_bounds(const Sched& sc, int c, int& k0, int& k1) {
+  const int u = div_small(c, sc.M + 1), i = c - u * (sc.M + 1);
+  const int a = unit_begin(sc, u);
+  const bool longer = u < sc.r;
+  if (sc.M == 0) {
+    k0 = a;
+    k1 = a + sc.Lq + longer;
+    return;
+  }
+  const int S = longer ? sc.Sr : sc.Sq, D = longer ? sc.Dr : sc.Dq;
+  if (i == 0) {
+    k0 = a;
+    k1 = a + S;
+  } else {
+    k0 = a + S + div_sub_weight(static_cast<int64_t>(D) * sub_cum(i - 1, sc.M), sc.M);
+    k1 = a + S + div_sub_weight(static_cast<int64_t>(D) * sub_cum(i, sc.M), sc.M);
+  }
+}
+
+__device__ __forceinline__ int chunk_of_tile(const Sched& sc, int k) {
+  const int u = unit_of_tile(sc, k);
+  if (sc.M == 0) return u;
+  const int a = unit_begin(sc, u);
+  const bool longer = u < sc.r;
+  const int S = longer ? sc.Sr : sc.Sq, D = longer ? sc.Dr : sc.Dq;
+  int i = 0;
+  if (k >= a + S) {
+    i = 1;
+    while (i < sc.M && k >= a + S + div_sub_weight(static_cast<int64_t>(D) * sub_cum(i, sc.M), sc.M)) ++i;
+  }
+  return u * (sc.M + 1) + i;
 }
 
 // Byte offset of (token, dim) inside one K or V tile in shared memory: boxes of
@@ -691,9 +779,9 @@ __device__ __forceinline__ void q_fetch(uint8_t* qbuf, const void* q, int n_q_he
 }
 
 // Phase 2 of the decode kernel: one warp merges query head g of the split
-// segment whose first piece unit u holds (mt = meta[u]); the pieces are held
-// by units u..u_hi (units are never empty: their count is capped at the tile
-// count) and are combined in unit order as
+// segment whose first piece chunk u holds (mt = meta[u]); the pieces are held
+// by chunks u..u_hi (chunks are never empty) and are combined in chunk (tile)
+// order as
 //   M = max_i m_i,  w_i = 2^(m_i - M),  out = sum_i w_i O_i / sum_i w_i l_i.
 // Lane j holds the scalars of pieces j and j + 32; each lane owns D/32 dims
 // of the numerator and walks the pieces eight loads at a time, the weights
@@ -705,7 +793,7 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
   constexpr int DPL = D / 32;
   const int seg = mt.x, b = seg / p.ng, hg = seg % p.ng, n = mt.y - u + 1;
   const int mo = p.gp * D + g, lo = p.gp * D + p.gp + g, oo = g * D + lane * DPL;
-  auto rec_of = [&](int j) -> const float* {  // record of piece j (unit u + j)
+  auto rec_of = [&](int j) -> const float* {  // record of piece j (chunk u + j)
     return p.records + (static_cast<size_t>(u + j) * 2 + (j == 0 ? mt.z : 0)) * p.rec_floats;
   };
   T* const ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
@@ -828,7 +916,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint8_t* qbufs = ring + static_cast<size_t>(n_slots) * kStageBytes;  // [warps][kQBufBytes]
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(qbufs + kConsumerWarps * kQBufBytes);
   uint64_t* empty_bar = full_bar + n_slots;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty_bar + n_slots);
+  int4* slot_info = reinterpret_cast<int4*>(empty_bar + n_slots);  // [n_slots]: next chunk, from the producer
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(slot_info + n_slots);
   int* prefix = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 4));  // [batch + 1]
   int* ctxs = prefix + p.batch + 1;                                                    // [batch]
   __shared__ int warp_sums[kConsumerWarps + 1];
@@ -887,75 +976,96 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __syncthreads();
 
   const int T = prefix[B];
-  // At most one unit per tile, so that no unit is empty.
-  const int U = min(p.num_units, max(T, 1));
-  int4 my_meta = make_int4(-1, 0, 0, T);  // consumer warps: split segment this unit merges
+  const Sched sc = make_sched(T, p.num_units, p.sub_chunks, p.static_permille);
+  const int U = sc.U, M = sc.M;
+  const int n_chunks = U * (M + 1);
 
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
-    // Lane w feeds unit w.  Lanes never wait for each other: each polls its
-    // own next ring slot (non-blocking test of the empty barrier) and issues
-    // the TMA loads when the slot is free.  The physical block ids of a lane's
-    // next two tiles are kept in registers, loaded two tiles ahead.
+    // Lane w feeds consumer warp w: first its unit's own chunk, then the
+    // balancing chunks it claims.  Lanes never wait for each other: each polls
+    // its own next ring slot (non-blocking test of the empty barrier) and
+    // issues the TMA loads when the slot is free.  The next two tiles are
+    // resolved ahead.  Nothing fetched from global memory is used in the
+    // iteration that fetches it: a physical block id is checked when its tile
+    // is issued, and the claim of the next chunk is sent kClaimAhead tiles
+    // before the current chunk's end and read at its last tile, so the warp
+    // (whose lanes run in step) never waits on an L2 round trip.
     const int u = blockIdx.x * kConsumerWarps + lane;
-    int pending = 0;
     Walk wn;
+    bool walking = false;
     if (lane < kConsumerWarps && u < U) {
-      const int k0 = unit_begin(u, T, U), k1 = unit_begin(u + 1, T, U);
-      if (walk_begin(wn, prefix, ctxs, B, k0, k1)) pending = k1 - k0;
+      int k0, k1;
+      chunk_bounds(sc, u * (M + 1), k0, k1);
+      walking = walk_begin(wn, prefix, ctxs, B, k0, k1);
     }
-    auto load_phys = [&](const Walk& w) -> int {
-      int ph = __ldg(p.block_tables + static_cast<size_t>(w.b) * p.max_blocks_per_seq + w.j);
-      if (ph < 0 || ph >= p.num_blocks) {
-        flag_error(PKV_DEVERR_BLOCK_ID);
-        ph = 0;
-      }
-      return ph;
+    int ticket = -1;
+    bool claimed = false;
+    struct Ahead {
+      int phys, kvh;
+      int4 info;  // {next chunk, its first tile, its end, 0} on a chunk's last tile, else next chunk -2
+      bool valid;
     };
-    auto advance = [&](Walk& w) {
-      if (w.k + 1 < w.k_end) walk_next(w, prefix, ctxs, B, p.ng);
-      else w.k = w.k_end;
-    };
-    int q0_phys = 0, q0_kvh = 0, q1_phys = 0, q1_kvh = 0;
-    if (pending > 0) {
-      q0_phys = load_phys(wn);
-      q0_kvh = (wn.hg * p.gp) / p.group;
-      advance(wn);
-      if (wn.k < wn.k_end) {
-        q1_phys = load_phys(wn);
-        q1_kvh = (wn.hg * p.gp) / p.group;
-        advance(wn);
+    auto resolve = [&](Ahead& t) {
+      t.valid = walking;
+      if (!walking) return;
+      t.phys = __ldg(p.block_tables + static_cast<size_t>(wn.b) * p.max_blocks_per_seq + wn.j);
+      t.kvh = (wn.hg * p.gp) / p.group;
+      t.info = make_int4(-2, 0, 0, 0);
+      if (M > 0 && !claimed && wn.k + kClaimAhead >= wn.k_end) {
+        ticket = atomicAdd(p.sched, 1);
+        claimed = true;
       }
-    }
+      if (wn.k + 1 < wn.k_end) {
+        walk_next(wn, prefix, ctxs, B, p.ng);
+        return;
+      }
+      walking = false;
+      t.info.x = -1;
+      if (claimed && ticket >= 0 && ticket < U * M) {
+        // All units' largest balancing chunks first.
+        const int c = (ticket % U) * (M + 1) + 1 + ticket / U;
+        int k0, k1;
+        chunk_bounds(sc, c, k0, k1);
+        t.info = make_int4(c, k0, k1, 0);
+        walking = walk_begin(wn, prefix, ctxs, B, k0, k1);
+      }
+      claimed = false;
+    };
+    Ahead t0, t1;
+    resolve(t0);
+    resolve(t1);
     int stage = 0, issued = 0;
     uint32_t phase = 0;
     uint64_t idle_since = 0;
-    while (__any_sync(0xffffffffu, pending > 0)) {
+    while (__any_sync(0xffffffffu, t0.valid)) {
       bool progressed = false;
-      if (pending > 0) {
+      if (t0.valid) {
         const int slot = lane * p.stages + stage;
         if (mbar_test_wait(&empty_bar[slot], phase ^ 1u)) {
+          int ph = t0.phys;
+          if (ph < 0 || ph >= p.num_blocks) {
+            flag_error(PKV_DEVERR_BLOCK_ID);
+            ph = 0;
+          }
+          asm volatile("st.shared.v4.s32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(&slot_info[slot])), "r"(t0.info.x),
+                       "r"(t0.info.y), "r"(t0.info.z), "r"(t0.info.w)
+                       : "memory");  // published to the consumer by the arrive below
           mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
           uint8_t* sk = ring + static_cast<size_t>(slot) * kStageBytes;
 #pragma unroll
           for (int y = 0; y < Y; ++y)
-            tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, q0_kvh, q0_phys);
+            tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, t0.kvh, ph);
 #pragma unroll
           for (int y = 0; y < Y; ++y)
-            tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, q0_kvh, q0_phys);
+            tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, t0.kvh, ph);
           ++issued;
-          --pending;
           if (++stage == p.stages) {
             stage = 0;
             phase ^= 1u;
           }
-          q0_phys = q1_phys;
-          q0_kvh = q1_kvh;
-          if (wn.k < wn.k_end) {
-            q1_phys = load_phys(wn);
-            q1_kvh = (wn.hg * p.gp) / p.group;
-            advance(wn);
-          }
+          t0 = t1;
+          resolve(t1);
           progressed = true;
         }
       }
@@ -980,9 +1090,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int s = 0; s < p.stages && s < issued; ++s) {
         const int cnt = (issued - s + p.stages - 1) / p.stages;
         const uint32_t par = static_cast<uint32_t>((cnt - 1) & 1);
-        const uint64_t t0 = global_timer_ns();
+        const uint64_t t0s = global_timer_ns();
         while (!mbar_try_wait(&full_bar[lane * p.stages + s], par)) {
-          if (global_timer_ns() - t0 > kWaitLimitNs) {
+          if (global_timer_ns() - t0s > kWaitLimitNs) {
             flag_error(kDevErrTimeout);
             break;
           }
@@ -994,11 +1104,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const int u = blockIdx.x * kConsumerWarps + warp;
     if (u < U) {
       uint8_t* qbuf = qbufs + warp * kQBufBytes;
-      const int k0 = unit_begin(u, T, U), k1 = unit_begin(u + 1, T, U);
+      int chunk = u * (M + 1);
+      int k0, k1;
+      chunk_bounds(sc, chunk, k0, k1);
       Walk wk;
       bool have = walk_begin(wk, prefix, ctxs, B, k0, k1);
       Consumer cs;
       int first_seg = -1, cur_seg = -1, cur_b = 0, cur_hg = 0, seg_start = 0, seg_end = 0;
+      int4 my_meta = make_int4(-1, 0, 0, 0);  // split segment whose first piece this chunk holds
       int stage = 0;
       uint32_t phase = 0;
       bool aborted = false;
@@ -1010,9 +1123,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           cs.finish(p, cur_b, cur_hg, nullptr, lane);
         } else {
           const int slot_idx = (cur_seg == first_seg) ? 0 : 1;
-          float* rec = p.records + (static_cast<size_t>(u) * 2 + slot_idx) * p.rec_floats;
+          float* rec = p.records + (static_cast<size_t>(chunk) * 2 + slot_idx) * p.rec_floats;
           cs.finish(p, cur_b, cur_hg, rec, lane);
-          if (starts_here) my_meta = make_int4(cur_seg, unit_of_tile(seg_end - 1, T, U), slot_idx, T);
+          if (starts_here) my_meta = make_int4(cur_seg, chunk_of_tile(sc, seg_end - 1), slot_idx, 0);
         }
       };
 
@@ -1034,9 +1147,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           __syncwarp();
           q_ready = false;
         }
-        // The last tile of a segment, with more tiles to come: start copying
-        // the next segment's Q now, so that it is in place when it is needed.
-        if (wk.j == wk.nb - 1 && wk.k + 1 < wk.k_end) {
+        const bool last = wk.k + 1 >= wk.k_end;
+        // The last tile of a segment, with more tiles to come in this chunk:
+        // start copying the next segment's Q now, so that it is in place when
+        // it is needed.
+        if (wk.j == wk.nb - 1 && !last) {
           Walk nx = wk;
           walk_next(nx, prefix, ctxs, B, p.ng);
           q_fetch<ES, D>(qbuf, p.q, p.n_q_heads, nx.b, nx.hg, p.gp, lane);
@@ -1047,6 +1162,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           aborted = true;
           break;
         }
+        int next_chunk = -1, n0 = 0, n1 = 0;
+        if (last) {
+          // The chunk this warp runs next, as claimed by its producer lane:
+          // start copying the Q of its first segment.
+          int4 info;
+          asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(info.x), "=r"(info.y), "=r"(info.z), "=r"(info.w)
+                       : "r"(smem_u32(&slot_info[slot])));
+          next_chunk = info.x;
+          n0 = info.y;
+          n1 = info.z;
+          Walk nw;
+          if (next_chunk >= 0 && walk_begin(nw, prefix, ctxs, B, n0, n1)) {
+            q_fetch<ES, D>(qbuf, p.q, p.n_q_heads, nw.b, nw.hg, p.gp, lane);
+            q_ready = true;
+          } else {
+            next_chunk = -1;
+          }
+        }
         const int nv = min(kBlockTokens, wk.ctx - wk.j * kBlockTokens);
         cs.tile(smem_u32(ring + static_cast<size_t>(slot) * kStageBytes), nv, p.scale_log2, lane);
         __syncwarp();
@@ -1055,40 +1189,65 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           stage = 0;
           phase ^= 1u;
         }
-        if (wk.k + 1 < wk.k_end) walk_next(wk, prefix, ctxs, B, p.ng);
-        else have = false;
+        if (!last) {
+          walk_next(wk, prefix, ctxs, B, p.ng);
+          continue;
+        }
+        // End of a chunk: close its open segment and publish its metadata.
+        finish_segment();
+        if (lane == 0) p.meta[chunk] = my_meta;
+        have = next_chunk >= 0;
+        if (have) {
+          chunk = next_chunk;
+          k0 = n0;
+          k1 = n1;
+          walk_begin(wk, prefix, ctxs, B, k0, k1);
+          first_seg = cur_seg = -1;
+          my_meta = make_int4(-1, 0, 0, 0);
+        }
       }
       cp_async_wait_all();
-      if (!aborted && cur_seg >= 0) finish_segment();
-      if (aborted) my_meta = make_int4(-1, 0, 0, T);
-      if (lane == 0) p.meta[u] = my_meta;
+      if (aborted && lane == 0) p.meta[chunk] = make_int4(-1, 0, 0, 0);
     }
   }
 
   // ---------------- phase 2: merge split segments ----------------
-  // Every warp of the grid takes (unit, query head) items; the items of units
-  // that hold the first piece of a split segment merge that head.
+  // Every warp of the grid takes (chunk, query head) items; the items of
+  // chunks that hold the first piece of a split segment merge that head.
   cooperative_groups::this_grid().sync();
   {
     constexpr int kWarps = kConsumerWarps + 1;
     const int gw = blockIdx.x * kWarps + warp, n_warps = gridDim.x * kWarps;
-    const int items = U * p.gp;
-    // At most 32 items per warp (U <= kConsumerWarps per CTA, gp <= 16):
-    // load their
-    // metadata in one round, lane t for the warp's t-th item.
-    int4 my_item = make_int4(-1, 0, 0, 0);
-    {
-      const int i = gw + lane * n_warps;
-      if (i < items) my_item = __ldcg(p.meta + i / p.gp);
+    const int items = n_chunks * p.gp;
+    const int n_segs = B * p.ng;
+    // Item metadata is loaded 32 items at a time, lane t for the round's
+    // t-th item of this warp.
+    for (int base = gw; base < items; base += 32 * n_warps) {
+      int4 my_item = make_int4(-1, 0, 0, 0);
+      const int i_lane = base + lane * n_warps;
+      if (i_lane < items) my_item = __ldcg(p.meta + i_lane / p.gp);
+      for (int t = 0; t < 32 && base + t * n_warps < items; ++t) {
+        const int i = base + t * n_warps;
+        const int c = i / p.gp;
+        int4 mt;
+        mt.x = __shfl_sync(0xffffffffu, my_item.x, t);
+        mt.y = __shfl_sync(0xffffffffu, my_item.y, t);
+        mt.z = __shfl_sync(0xffffffffu, my_item.z, t);
+        // Entries of chunks that an aborted launch never reached may be
+        // stale: only well-formed ones are merged.
+        if (mt.x >= 0 && mt.x < n_segs && mt.y > c && mt.y < n_chunks && (mt.z == 0 || mt.z == 1))
+          merge_head<DT, D>(p, c, mt, i % p.gp, lane);
+      }
     }
-    for (int t = 0; gw + t * n_warps < items; ++t) {
-      const int i = gw + t * n_warps;
-      int4 mt;
-      mt.x = __shfl_sync(0xffffffffu, my_item.x, t);
-      mt.y = __shfl_sync(0xffffffffu, my_item.y, t);
-      mt.z = __shfl_sync(0xffffffffu, my_item.z, t);
-      mt.w = __shfl_sync(0xffffffffu, my_item.w, t);
-      if (mt.x >= 0) merge_head<DT, D>(p, i / p.gp, mt, i % p.gp, lane);
+    // The claim counter must have seen every balancing chunk plus one failed
+    // claim per unit; anything else means it was not zero at launch (the
+    // workspace was not cleared before its first use).  Leave it at zero.
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      const int expect = M > 0 ? U * M + U : 0;
+      const int seen = *reinterpret_cast<volatile int*>(p.sched);
+      if (seen != expect && (*reinterpret_cast<volatile uint32_t*>(&g_device_error) & kDevErrTimeout) == 0)
+        flag_error(PKV_DEVERR_SCHEDULE);
+      if (seen != 0) *reinterpret_cast<volatile int*>(p.sched) = 0;
     }
     // Sequences with no tokens get a zero output row, or, when an initial
     // state is given for them, that state normalised.

@@ -25,14 +25,15 @@ def bits(t: torch.Tensor) -> torch.Tensor:
 
 
 def run_gpu(w, num_units: int = 0, force_simt: bool = False, check_errors: bool = True,
-            return_cache: bool = False, workspace=None):
+            return_cache: bool = False, workspace=None, balance_chunks: int = 0, static_permille: int = 0):
     dev = torch.device("cuda")
     kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
     if w.appended:
         pkv.paged_kv_append(w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev), kc, vc)
     out = pkv.paged_attention_decode(w.q.to(dev), kc, vc, w.block_tables.to(dev), w.context_lens.to(dev),
                                      w.scale, num_units=num_units, force_simt=force_simt,
-                                     workspace=workspace)
+                                     workspace=workspace, balance_chunks=balance_chunks,
+                                     static_permille=static_permille)
     torch.cuda.synchronize()
     if check_errors:
         assert pkv.pkv_get_device_error() == 0

@@ -32,7 +32,7 @@ def test_header_declares_expected_entry_points():
     names = set(declared_functions())
     assert {"paged_kv_append", "paged_attention_decode", "paged_attention_decode_ex",
             "paged_attention_workspace_size", "pkv_get_device_error", "pkv_status_string",
-            "pkv_version", "paged_kv_copy_blocks", "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_hash_blocks",
+            "pkv_version", "paged_kv_copy_blocks", "paged_attention_workspace_size_ex", "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_hash_blocks",
             "pkv_bm_add_sequence", "pkv_bm_fork", "pkv_bm_append", "pkv_bm_free", "pkv_bm_get_tables",
             "pkv_bm_stats", "pkv_bm_refcount"} <= names
 
@@ -81,11 +81,12 @@ def test_decode_ex_rejects_bad_options(lib):
     st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
                                        None, 0, None, ctypes.byref(opts))
     assert st == INVALID
-    opts = pkv._Options()
-    opts.reserved[2] = 1
-    st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
-                                       None, 0, None, ctypes.byref(opts))
-    assert st == INVALID
+    for bad in (dict(reserved=(ctypes.c_int32 * 4)(0, 0, 1, 0)), dict(balance_chunks=5), dict(balance_chunks=-1),
+                dict(static_permille=100), dict(static_permille=1000)):
+        opts = pkv._Options(**bad)
+        st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
+                                           None, 0, None, ctypes.byref(opts))
+        assert st == INVALID, bad
 
 
 def test_append_host_validation(lib):

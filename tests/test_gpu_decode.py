@@ -90,6 +90,48 @@ def test_split_count_invariance():
     assert torch.equal(bits(run_gpu(w, num_units=7)), bits(outs[7]))
 
 
+# Balancing chunks: the last part of every unit's tile range is cut into
+# chunks that the first warps to run out of work claim at run time.  The
+# workloads here give each unit enough tiles (few units) for the chunks to be
+# used.
+BALANCE = [(64, 3, 0), (64, 4, 500), (64, 1, 999), (200, 2, 0), (37, 0, 0), (150, 3, 700)]
+
+
+@pytest.mark.parametrize("units,balance,permille", BALANCE, ids=[f"u{u}-c{c}-s{s}" for u, c, s in BALANCE])
+def test_balancing_chunks_match_oracle_and_repeat_bitwise(units, balance, permille):
+    w = W.uniform_gqa(batch=10, len_lo=100, len_hi=3000, seed=13)
+    ref, _, _ = oracle.workload_decode(w)
+    ws = pkv.new_workspace(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
+                                                              w.dtype, balance_chunks=balance))
+    kw = dict(num_units=units, balance_chunks=balance, static_permille=permille, workspace=ws)
+    out = run_gpu(w, **kw)
+    assert_close(out, ref, w.dtype, what=str(kw))
+    for _ in range(3):   # which warp runs a chunk varies; the bits do not
+        assert torch.equal(bits(run_gpu(w, **kw)), bits(out))
+
+
+@pytest.mark.parametrize("simt", [False, True])
+def test_balancing_chunks_on_mha_and_simt_paths(simt):
+    w = W.lognormal_mha(batch=24, seed=31)
+    ref, _, _ = oracle.workload_decode(w)
+    for units, balance in ((48, 4), (48, 0)):
+        out = run_gpu(w, num_units=units, balance_chunks=balance, force_simt=simt)
+        assert_close(out, ref, w.dtype, what=f"mha units={units} balance={balance} simt={simt}")
+
+
+def test_workspace_not_cleared_is_flagged_then_reset():
+    w = W.uniform_gqa(batch=10, len_lo=100, len_hi=3000, seed=13)
+    ref, _, _ = oracle.workload_decode(w)
+    need = pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype,
+                                              balance_chunks=3)
+    for fill in (0x7F, 0xFF):   # a large positive and a negative claim counter
+        ws = torch.full((need,), fill, dtype=torch.uint8, device="cuda")
+        run_gpu(w, num_units=64, workspace=ws, check_errors=False, balance_chunks=3)
+        assert pkv.pkv_get_device_error() & pkv.DEVERR_SCHEDULE
+        out = run_gpu(w, num_units=64, workspace=ws, balance_chunks=3)   # the launch left the counter at zero
+        assert_close(out, ref, w.dtype, what=f"after fill {fill:#x}")
+
+
 def test_one_unit_no_split_matches_oracle_on_every_path():
     for simt in (False, True):
         w = W.build_workload("one", [3, 40, 517], 8, 2, 128, torch.bfloat16, seed=14)
@@ -220,7 +262,7 @@ def test_maximum_batch():
 def test_explicit_workspace_and_too_small_workspace():
     w = W.uniform_gqa(batch=8, len_lo=500, len_hi=3000, seed=24)
     need = pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.dtype)
-    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ws = pkv.new_workspace(need)
     a = run_gpu(w, workspace=ws)
     b = run_gpu(w)
     assert torch.equal(bits(a), bits(b))
