@@ -244,6 +244,170 @@ int oracle_paged_decode(const void* q, const void* k_cache, const void* v_cache,
   return status;
 }
 
+/*
+ * ---------------------------------------------------------------------------
+ * INT8 paged KV cache (quantised KV: "Transformer anatomy" ch. 15 §15.7, INT8
+ * KV quantisation trades a small accuracy loss for half the bytes).
+ *
+ * Format (a reading: the pages fix neither granularity nor layout):
+ *   k8      int8 [num_blocks][n_kv][block_size][head_dim]
+ *   v8      int8 [num_blocks][n_kv][head_dim][block_size]; within a row, token
+ *           j of the block sits at byte position
+ *             vpos(j) = 4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2)
+ *   k_scale, v_scale  fp32 [num_blocks][n_kv][block_size]
+ * Each (token, kv head) row x of K or V is quantised symmetrically:
+ *   amax = max_e |x_e|, scale = amax / 127 (binary32 division),
+ *   code_e = clamp(rint(x_e / scale), -127, 127) (binary32 division, rounding
+ *   half to even; all codes 0 when amax = 0),
+ * and read back as scale * code.  The binary32 steps are what decide the
+ * integer codes, so they are done here in binary32 exactly as stated.
+ * ---------------------------------------------------------------------------
+ */
+static int vpos(int j) { return 4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2); }
+
+static void quantise_row(const void* src, size_t idx0, int dtype, int32_t d, int8_t* codes, float* scale_out) {
+  float amax = 0.0f;
+  for (int32_t e = 0; e < d; ++e) {
+    float x = (float)load_elem(src, idx0 + e, dtype); /* exact: 16-bit values widen exactly */
+    float a = fabsf(x);
+    if (a > amax) amax = a;
+  }
+  float scale = amax / 127.0f;
+  for (int32_t e = 0; e < d; ++e) {
+    float x = (float)load_elem(src, idx0 + e, dtype);
+    float c = amax == 0.0f ? 0.0f : rintf(x / scale);
+    if (c > 127.0f) c = 127.0f;
+    if (c < -127.0f) c = -127.0f;
+    codes[e] = (int8_t)c;
+  }
+  *scale_out = scale;
+}
+
+/* Append into the INT8 cache (the block-size must be 16: vpos is defined for it). */
+int oracle_kv_append_int8(const void* k, const void* v, int32_t dtype, const int64_t* slot_mapping,
+                          int32_t num_tokens, int8_t* k8, int8_t* v8, float* k_scale, float* v_scale,
+                          int32_t num_blocks, int32_t block_size, int32_t n_kv_heads, int32_t head_dim) {
+  if (!elem_bytes(dtype) || num_tokens < 0 || num_blocks <= 0 || block_size != 16 || n_kv_heads <= 0 ||
+      head_dim <= 0)
+    return ORC_EINVAL;
+  int8_t* codes = (int8_t*)malloc((size_t)head_dim);
+  if (!codes) return ORC_ENOMEM;
+  int64_t n_slots = (int64_t)num_blocks * block_size;
+  for (int32_t i = 0; i < num_tokens; ++i) {
+    int64_t s = slot_mapping[i];
+    if (s < 0) continue;
+    if (s >= n_slots) {
+      free(codes);
+      return ORC_ESLOT;
+    }
+    int64_t blk = s / block_size, off = s % block_size;
+    for (int32_t h = 0; h < n_kv_heads; ++h) {
+      size_t src = ((size_t)i * n_kv_heads + h) * head_dim;
+      size_t bh = (size_t)blk * n_kv_heads + h;
+      float sc;
+      quantise_row(k, src, dtype, head_dim, codes, &sc);
+      memcpy(k8 + (bh * block_size + off) * head_dim, codes, (size_t)head_dim);
+      k_scale[bh * block_size + off] = sc;
+      quantise_row(v, src, dtype, head_dim, codes, &sc);
+      for (int32_t e = 0; e < head_dim; ++e) v8[(bh * head_dim + e) * block_size + vpos((int)off)] = codes[e];
+      v_scale[bh * block_size + off] = sc;
+    }
+  }
+  free(codes);
+  return ORC_OK;
+}
+
+/* The same single-query attention as decode_row, over the dequantised INT8
+ * cache (every value scale * code, exact in double). */
+static int decode_row_int8(const void* q, int dtype, const int8_t* k8, const int8_t* v8, const float* k_scale,
+                           const float* v_scale, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t num_blocks, double scale, int32_t n_q,
+                           int32_t n_kv, int32_t d, int32_t bs, int32_t b, int32_t h, double* out_row) {
+  int32_t group = n_q / n_kv;
+  int32_t kvh = h / group;
+  int32_t ctx = context_lens[b];
+  if (ctx < 0 || (int64_t)ctx > (int64_t)max_blocks_per_seq * bs) return ORC_ECTX;
+  for (int32_t e = 0; e < d; ++e) out_row[e] = 0.0;
+  if (ctx == 0) return ORC_OK;
+  double* K = (double*)malloc(sizeof(double) * (size_t)ctx * d);
+  double* V = (double*)malloc(sizeof(double) * (size_t)ctx * d);
+  double* s = (double*)malloc(sizeof(double) * (size_t)ctx);
+  double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+  if (!K || !V || !s || !qv) {
+    free(K); free(V); free(s); free(qv);
+    return ORC_ENOMEM;
+  }
+  for (int32_t j = 0; j < ctx; ++j) {
+    int32_t phys = block_tables[(size_t)b * max_blocks_per_seq + j / bs];
+    if (phys < 0 || phys >= num_blocks) {
+      free(K); free(V); free(s); free(qv);
+      return ORC_EBLOCK;
+    }
+    size_t bh = (size_t)phys * n_kv + kvh;
+    int32_t off = j % bs;
+    double ks = (double)k_scale[bh * bs + off], vs = (double)v_scale[bh * bs + off];
+    for (int32_t e = 0; e < d; ++e) {
+      K[(size_t)j * d + e] = ks * (double)k8[(bh * bs + off) * d + e];
+      V[(size_t)j * d + e] = vs * (double)v8[(bh * d + e) * bs + vpos(off)];
+    }
+  }
+  for (int32_t e = 0; e < d; ++e) qv[e] = load_elem(q, ((size_t)b * n_q + h) * d + e, dtype);
+  for (int32_t j = 0; j < ctx; ++j) {
+    double acc = 0.0;
+    for (int32_t e = 0; e < d; ++e) acc += qv[e] * K[(size_t)j * d + e];
+    s[j] = scale * acc;
+  }
+  double m = s[0];
+  for (int32_t j = 1; j < ctx; ++j)
+    if (s[j] > m) m = s[j];
+  double denom = 0.0;
+  for (int32_t j = 0; j < ctx; ++j) {
+    s[j] = exp(s[j] - m);
+    denom += s[j];
+  }
+  for (int32_t j = 0; j < ctx; ++j)
+    for (int32_t e = 0; e < d; ++e) out_row[e] += s[j] * V[(size_t)j * d + e];
+  for (int32_t e = 0; e < d; ++e) out_row[e] /= denom;
+  free(K); free(V); free(s); free(qv);
+  return ORC_OK;
+}
+
+int oracle_paged_decode_int8(const void* q, int32_t dtype, const int8_t* k8, const int8_t* v8,
+                             const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
+                             int32_t num_blocks, double scale, int32_t n_q_heads, int32_t n_kv_heads,
+                             int32_t head_dim, int32_t block_size, double* out, const int32_t* rows,
+                             int32_t n_rows, int32_t n_threads) {
+  if (!elem_bytes(dtype) || batch < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0 ||
+      head_dim <= 0 || block_size != 16 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return ORC_EINVAL;
+  int64_t total = rows ? (int64_t)n_rows : (int64_t)batch * n_q_heads;
+  int status = ORC_OK;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+  (void)n_threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < total; ++r) {
+    int32_t b = rows ? rows[2 * r] : (int32_t)(r / n_q_heads);
+    int32_t h = rows ? rows[2 * r + 1] : (int32_t)(r % n_q_heads);
+    int rc;
+    if (b < 0 || b >= batch || h < 0 || h >= n_q_heads) {
+      rc = ORC_EINVAL;
+    } else {
+      rc = decode_row_int8(q, dtype, k8, v8, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
+                           num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, b, h,
+                           out + ((size_t)b * n_q_heads + h) * head_dim);
+    }
+    if (rc != ORC_OK) {
+#pragma omp critical
+      status = rc;
+    }
+  }
+  return status;
+}
+
 /* Number of threads an OpenMP region would use (for reporting). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

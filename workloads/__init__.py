@@ -267,6 +267,37 @@ def cascade_view(w: DecodeWorkload) -> CascadeView:
                        torch.tensor(lens, dtype=torch.int32))
 
 
+def cached_token_rows(w: DecodeWorkload):
+    """Every slot that holds a token before this step's append, once each
+    (shared blocks are listed once): ``(k_rows, v_rows, slots)`` with rows
+    ``[n, n_kv, d]`` copied from the caches and int64 slots.  Used to fill a
+    cache of another format with the same tokens."""
+    bs = w.block_size
+    slots = set()
+    for b, n in enumerate(w.lens()):
+        held = n - 1 if w.appended else n
+        for j in range(held):
+            slots.add(int(w.block_tables[b, j // bs]) * bs + j % bs)
+    sl = torch.tensor(sorted(slots), dtype=torch.int64)
+    blk, off = sl // bs, sl % bs
+    k_rows = w.k_cache[blk, :, off, :].contiguous()
+    v_rows = w.v_cache[blk, :, off, :].contiguous()
+    return k_rows, v_rows, sl
+
+
+def int8_cache_buffers(w: DecodeWorkload):
+    """Empty INT8 cache buffers for the pool of ``w``: codes ``k8``
+    ``[blocks, n_kv, 16, d]`` and ``v8`` ``[blocks, n_kv, d, 16]`` zeroed, and
+    per-token fp32 scales ``[blocks, n_kv, 16]`` set to NaN, so that a read of
+    a slot that holds no token poisons the result."""
+    nb, nkv, bs, d = w.k_cache.shape
+    k8 = torch.zeros((nb, nkv, bs, d), dtype=torch.int8)
+    v8 = torch.zeros((nb, nkv, d, bs), dtype=torch.int8)
+    ks = torch.full((nb, nkv, bs), float("nan"), dtype=torch.float32)
+    vs = torch.full((nb, nkv, bs), float("nan"), dtype=torch.float32)
+    return k8, v8, ks, vs
+
+
 # ---------------------------------------------------------------------------
 # The five workload shapes (Llama-class, block size 16).
 # ---------------------------------------------------------------------------
