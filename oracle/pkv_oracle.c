@@ -323,24 +323,23 @@ static int decode_row_int8(const void* q, int dtype, const int8_t* k8, const int
                            const float* v_scale, const int32_t* block_tables, int32_t max_blocks_per_seq,
                            const int32_t* context_lens, int32_t num_blocks, double scale, int32_t n_q,
                            int32_t n_kv, int32_t d, int32_t bs, int32_t b, int32_t h, double* out_row) {
-  int32_t group = n_q / n_kv;
-  int32_t kvh = h / group;
-  int32_t ctx = context_lens[b];
+  int32_t kvh = h / (n_q / n_kv);
+  const int32_t ctx = *(context_lens + b);
   if (ctx < 0 || (int64_t)ctx > (int64_t)max_blocks_per_seq * bs) return ORC_ECTX;
   for (int32_t e = 0; e < d; ++e) out_row[e] = 0.0;
   if (ctx == 0) return ORC_OK;
   double* K = (double*)malloc(sizeof(double) * (size_t)ctx * d);
   double* V = (double*)malloc(sizeof(double) * (size_t)ctx * d);
-  double* s = (double*)malloc(sizeof(double) * (size_t)ctx);
+  double* w = (double*)malloc(sizeof(double) * (size_t)ctx);
   double* qv = (double*)malloc(sizeof(double) * (size_t)d);
-  if (!K || !V || !s || !qv) {
-    free(K); free(V); free(s); free(qv);
+  if (!K || !V || !w || !qv) {
+    free(K); free(V); free(w); free(qv);
     return ORC_ENOMEM;
   }
   for (int32_t j = 0; j < ctx; ++j) {
-    int32_t phys = block_tables[(size_t)b * max_blocks_per_seq + j / bs];
+    int32_t phys = block_tables[(size_t)b * max_blocks_per_seq + (size_t)(j / bs)];
     if (phys < 0 || phys >= num_blocks) {
-      free(K); free(V); free(s); free(qv);
+      free(K); free(V); free(w); free(qv);
       return ORC_EBLOCK;
     }
     size_t bh = (size_t)phys * n_kv + kvh;
@@ -351,24 +350,24 @@ static int decode_row_int8(const void* q, int dtype, const int8_t* k8, const int
       V[(size_t)j * d + e] = vs * (double)v8[(bh * d + e) * bs + vpos(off)];
     }
   }
-  for (int32_t e = 0; e < d; ++e) qv[e] = load_elem(q, ((size_t)b * n_q + h) * d + e, dtype);
+  for (int32_t e = 0; e < d; ++e) qv[e] = load_elem(q, (size_t)(b * n_q + h) * d + e, dtype);
+  /* Scores, softmax with the maximum subtracted, weighted sum of V. */
   for (int32_t j = 0; j < ctx; ++j) {
-    double acc = 0.0;
-    for (int32_t e = 0; e < d; ++e) acc += qv[e] * K[(size_t)j * d + e];
-    s[j] = scale * acc;
+    double dot = 0.0;
+    for (int32_t e = 0; e < d; ++e) dot += qv[e] * K[(size_t)j * d + e];
+    w[j] = dot * scale;
   }
-  double m = s[0];
-  for (int32_t j = 1; j < ctx; ++j)
-    if (s[j] > m) m = s[j];
-  double denom = 0.0;
+  double wmax = w[0];
+  for (int32_t j = 1; j < ctx; ++j) wmax = w[j] > wmax ? w[j] : wmax;
+  double total = 0.0;
   for (int32_t j = 0; j < ctx; ++j) {
-    s[j] = exp(s[j] - m);
-    denom += s[j];
+    w[j] = exp(w[j] - wmax);
+    total += w[j];
   }
   for (int32_t j = 0; j < ctx; ++j)
-    for (int32_t e = 0; e < d; ++e) out_row[e] += s[j] * V[(size_t)j * d + e];
-  for (int32_t e = 0; e < d; ++e) out_row[e] /= denom;
-  free(K); free(V); free(s); free(qv);
+    for (int32_t e = 0; e < d; ++e) out_row[e] += w[j] * V[(size_t)j * d + e];
+  for (int32_t e = 0; e < d; ++e) out_row[e] = out_row[e] / total;
+  free(K); free(V); free(w); free(qv);
   return ORC_OK;
 }
 
