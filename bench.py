@@ -184,7 +184,11 @@ def run_ours(args) -> None:
     make, desc = WORKLOADS[args.workload]
     w = make(args.seed)
     es = w.k_cache.element_size()
-    tr = layout.decode_traffic(w.block_tables, w.context_lens, w.n_q_heads, w.n_kv_heads, w.head_dim, es)
+    int8 = args.kv == "int8"
+    if int8 and args.cascade:
+        raise SystemExit("--kv int8 and --cascade cannot be combined")
+    tr = layout.decode_traffic(w.block_tables, w.context_lens, w.n_q_heads, w.n_kv_heads, w.head_dim, es,
+                               kv_int8=int8)
     kv_bytes = tr["kv_unique"]
     decode_bytes = tr["total_unique"]
 
@@ -193,6 +197,13 @@ def run_ours(args) -> None:
     q, k_new, v_new = w.q.to(dev), w.k_new.to(dev), w.v_new.to(dev)
     slots, bt, cl = w.slot_mapping.to(dev), w.block_tables.to(dev), w.context_lens.to(dev)
     out = torch.empty_like(q)
+    if int8:
+        # The same tokens quantised into the INT8 cache (untimed set-up).
+        k8, v8, ks8, vs8 = pkv.int8_cache(w.num_blocks, w.n_kv_heads, w.head_dim, device=dev)
+        kr, vr, sl = W.cached_token_rows(w)
+        pkv.paged_kv_append_int8(kr.to(dev), vr.to(dev), sl.to(dev), k8, v8, ks8, vs8)
+        del kc, vc, kr, vr
+        torch.cuda.synchronize(dev)
     if args.cascade:
         # Shared prefixes attended once per group and kv head, then the suffixes.
         cv = W.cascade_view(w)
@@ -204,8 +215,17 @@ def run_ours(args) -> None:
         ws = torch.zeros(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
                                                             w.dtype), dtype=torch.uint8, device=dev)
 
+    def append(stream_=None):
+        if int8:
+            pkv.paged_kv_append_int8(k_new, v_new, slots, k8, v8, ks8, vs8, stream=stream_)
+        else:
+            pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream_)
+
     def decode(stream_=None):
-        if args.cascade:
+        if int8:
+            pkv.paged_attention_decode_int8(q, k8, v8, ks8, vs8, bt, cl, w.scale, out=out, workspace=ws,
+                                            stream=stream_)
+        elif args.cascade:
             pkv.paged_attention_decode_cascade(q, kc, vc, c_pt, c_pl, c_sg, c_bt, c_cl, w.scale, out=out,
                                                workspace=ws, stream=stream_)
         else:
@@ -214,7 +234,7 @@ def run_ours(args) -> None:
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
+        append(stream)
         decode(stream)
 
     # Warm-up: W steps, continued until 0.3 s have passed so that the SM
@@ -243,7 +263,7 @@ def run_ours(args) -> None:
             cap.wait_stream(stream)
             with torch.cuda.graph(g, stream=cap):
                 ev_a.record()
-                pkv.paged_kv_append(k_new, v_new, slots, kc, vc)
+                append()
                 ev_b.record()
                 decode()
                 ev_c.record()
@@ -273,7 +293,7 @@ def run_ours(args) -> None:
             else:
                 a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
                 a.record(stream)
-                pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
+                append(stream)
                 b.record(stream)
                 decode(stream)
                 c.record(stream)
@@ -310,7 +330,7 @@ def run_ours(args) -> None:
     def e2e_step():
         for d, h in zip(d_in, h_in):
             d.copy_(h, non_blocking=True)
-        pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream)
+        append(stream)
         decode(stream)
         h_out.copy_(out, non_blocking=True)
 
@@ -334,32 +354,40 @@ def run_ours(args) -> None:
 
     traffic = None
     try:
-        prof = json.loads(PROFILE_TRAFFIC.read_text())
-        if prof.get("kernel_hash") == kernel_hash() and prof.get("workload") == args.workload:
-            traffic = prof.get("dram_bytes_per_launch")
+        entries = json.loads(PROFILE_TRAFFIC.read_text())
+        for prof in (entries if isinstance(entries, list) else [entries]):
+            if (prof.get("kernel_hash") == kernel_hash() and prof.get("workload") == args.workload
+                    and prof.get("kv", "16-bit") == ("int8" if int8 else "16-bit") and not args.cascade):
+                traffic = prof.get("dram_bytes_per_launch")
     except Exception:
         traffic = None
 
     result = None
     if rank == 0:
-        cpu = cpu_baseline(w, kv_bytes, budget_s=args.cpu_budget) if (world == 1 and not args.no_cpu) else None
+        cpu = (cpu_baseline(w, kv_bytes, budget_s=args.cpu_budget)
+               if (world == 1 and not args.no_cpu and not int8) else None)
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(max_step_s / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": W.DTYPE_NAMES[w.dtype], "data": "synthetic (seeded N(0,1) q/K/V, random block placement)",
+            "dtype": ("int8 KV / " if int8 else "") + W.DTYPE_NAMES[w.dtype],
+            "data": "synthetic (seeded N(0,1) q/K/V, random block placement)",
             "config": {"workload": desc, "global_batch": w.batch * world, "seq_len": "ragged",
                        "mean_context": round(tr["tokens"] / w.batch, 1), "parallelism": f"replicas x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed)", "seed": args.seed,
                        "warmup_steps_run": warm_steps,
                        "launch": launch_note,
-                       "decode": "cascade (shared prefix once per group)" if args.cascade else "paged decode"},
+                       "decode": "cascade (shared prefix once per group)" if args.cascade else "paged decode",
+                       "kv_cache": ("INT8 codes + fp32 scale per (token, kv head)" if int8
+                                    else W.DTYPE_NAMES[w.dtype])},
             "tokens_per_s_per_layer": round(tokens_per_s, 1),
             "kv_bytes_per_step": kv_bytes,
             "roofline": {"bound": "hbm",
                          "kernel": ("paged_attention_decode_cascade (pkv_prefix_kernel + pkv_decode_kernel)"
-                                    if args.cascade else "paged_attention_decode (pkv_decode_kernel)"),
+                                    if args.cascade else
+                                    "paged_attention_decode_int8 (pkv_decode_kernel, INT8)" if int8
+                                    else "paged_attention_decode (pkv_decode_kernel)"),
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": decode_bytes,
@@ -471,6 +499,8 @@ def main(argv=None) -> None:
     ap.add_argument("--cascade", action="store_true",
                     help="decode shared-prefix workloads with paged_attention_decode_cascade")
     ap.add_argument("--ref-seqs", type=int, default=0, help="sequences per reference-arm step (0: all)")
+    ap.add_argument("--kv", choices=["16-bit", "int8"], default="16-bit",
+                    help="cache format: the workload's 16-bit dtype, or INT8 codes with per-token scales")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -67,6 +67,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_widen.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_paged_decode_mq.argtypes = [p, p, p, i32, p, i32, p, i32, i32, ctypes.c_double, i32, i32, i32, i32,
+                                           i32, p, i32]
+    lib.oracle_paged_decode_mq.restype = ctypes.c_int
     lib.oracle_kv_append_int8.argtypes = [p, p, i32, p, i32, p, p, p, p, i32, i32, i32, i32]
     lib.oracle_kv_append_int8.restype = ctypes.c_int
     lib.oracle_paged_decode_int8.argtypes = [p, i32, p, p, p, p, p, i32, p, i32, i32, ctypes.c_double,
@@ -141,6 +144,36 @@ def workload_decode(w, rows=None, n_threads: int = 0, lib=None):
         kv_append(w.k_new, w.v_new, w.slot_mapping, kc, vc, w.block_size, lib=lib)
     out = paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=rows,
                        n_threads=n_threads, lib=lib)
+    return out, kc, vc
+
+
+def paged_decode_mq(q, k_cache, v_cache, block_tables, context_lens, scale: float, n_threads: int = 0,
+                    lib=None) -> torch.Tensor:
+    """fp64 ``[batch, q_len, n_q, d]`` multi-query attention: query i of a
+    sequence sees its context up to position ``ctx - q_len + i``."""
+    lib = lib or load()
+    B, q_len, n_q, d = q.shape
+    num_blocks, n_kv, bs, d2 = k_cache.shape
+    assert d2 == d and k_cache.dtype == q.dtype == v_cache.dtype
+    q = q.contiguous()
+    bt = block_tables.to(torch.int32).contiguous()
+    cl = context_lens.to(torch.int32).contiguous()
+    out = torch.full((B, q_len, n_q, d), float("nan"), dtype=torch.float64)
+    _check(lib.oracle_paged_decode_mq(_ptr(q), _ptr(k_cache), _ptr(v_cache), ORC_DTYPE[q.dtype], _ptr(bt),
+                                      bt.shape[1], _ptr(cl), B, num_blocks, float(scale), n_q, n_kv, d, bs, q_len,
+                                      _ptr(out), int(n_threads)))
+    return out
+
+
+def workload_decode_mq(w, n_threads: int = 0, lib=None):
+    """Oracle for a multi-query workload: append its q_len new tokens per
+    sequence, then the causal multi-query decode.  Returns
+    ``(out_fp64 [B, q_len, n_q, d], k_cache_after, v_cache_after)``."""
+    kc, vc = w.k_cache.clone(), w.v_cache.clone()
+    if w.appended:
+        kv_append(w.k_new, w.v_new, w.slot_mapping, kc, vc, w.block_size, lib=lib)
+    q = w.q if w.q.dim() == 4 else w.q.unsqueeze(1)
+    out = paged_decode_mq(q, kc, vc, w.block_tables, w.context_lens, w.scale, n_threads=n_threads, lib=lib)
     return out, kc, vc
 
 

@@ -245,6 +245,56 @@ int oracle_paged_decode(const void* q, const void* k_cache, const void* v_cache,
 }
 
 /*
+ * Multi-query decode (several new tokens per sequence: a draft to verify,
+ * "LLM Primer VI" ch. 8, speculative decoding; or a prefill chunk).  q and
+ * out are [batch][q_len][n_q][head_dim]; the q_len new tokens are the last
+ * q_len of the sequence's context (already in the cache), and query i sees
+ * the cache up to and including its own position:
+ *   ctx_i = context_lens[b] - q_len + i + 1.
+ * Each row is the single-query attention above over that prefix (causal
+ * among the new tokens).  context_lens[b] < q_len is an error.
+ */
+int oracle_paged_decode_mq(const void* q, const void* k_cache, const void* v_cache, int32_t dtype,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                           int32_t batch, int32_t num_blocks, double scale, int32_t n_q_heads,
+                           int32_t n_kv_heads, int32_t head_dim, int32_t block_size, int32_t q_len, double* out,
+                           int32_t n_threads) {
+  int es = elem_bytes(dtype);
+  if (!es || batch < 0 || q_len <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0 ||
+      head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return ORC_EINVAL;
+  int64_t total = (int64_t)batch * q_len * n_q_heads;
+  int status = ORC_OK;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+  (void)n_threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < total; ++r) {
+    int32_t h = (int32_t)(r % n_q_heads);
+    int32_t i = (int32_t)((r / n_q_heads) % q_len);
+    int32_t b = (int32_t)(r / ((int64_t)n_q_heads * q_len));
+    int32_t ctx_i = context_lens[b] - q_len + i + 1;
+    int rc;
+    if (context_lens[b] < q_len) {
+      rc = ORC_ECTX;
+    } else {
+      /* Query i of sequence b as a one-sequence single-query problem. */
+      const char* q_row = (const char*)q + ((size_t)b * q_len + i) * n_q_heads * head_dim * es;
+      rc = decode_row(q_row, k_cache, v_cache, dtype, block_tables + (size_t)b * max_blocks_per_seq,
+                      max_blocks_per_seq, &ctx_i, num_blocks, scale, n_q_heads, n_kv_heads, head_dim,
+                      block_size, 0, h, out + (size_t)r * head_dim);
+    }
+    if (rc != ORC_OK) {
+#pragma omp critical
+      status = rc;
+    }
+  }
+  return status;
+}
+
+/*
  * ---------------------------------------------------------------------------
  * INT8 paged KV cache (quantised KV: "Transformer anatomy" ch. 15 §15.7, INT8
  * KV quantisation trades a small accuracy loss for half the bytes).

@@ -140,10 +140,10 @@ pkv_status encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dt, i
 
 // The decode kernel is launched cooperatively: its CTAs (at most one per SM)
 // are guaranteed to be co-resident, which its grid-wide barrier needs.
-template <int DT, int D, int GPAD>
+template <int DT, int D, int GPAD, bool kI8 = false>
 pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid, size_t smem,
                          cudaStream_t stream) {
-  auto kern = pkv_decode_kernel<DT, D, GPAD>;
+  auto kern = pkv_decode_kernel<DT, D, GPAD, kI8>;
   // Opt in to the largest dynamic shared memory once per device (the launch
   // itself passes the size it needs).
   static bool opted_in[kMaxDevices] = {};
@@ -190,6 +190,35 @@ pkv_status dispatch_dim(int head_dim, int gpad, const CUtensorMap& mk, const CUt
   return head_dim == 64 ? dispatch_gpad<DT, 64>(gpad, mk, mv, p, grid, smem, stream)
                         : dispatch_gpad<DT, 128>(gpad, mk, mv, p, grid, smem, stream);
 }
+
+// INT8 cache (head_dim 128, tensor-core consumer for every head group).
+template <int DT>
+pkv_status dispatch_i8(int gpad, const CUtensorMap& mk, const DecodeParams& p, int grid, size_t smem,
+                       cudaStream_t stream) {
+  return gpad == 8 ? launch_decode<DT, 128, 8, true>(mk, mk, p, grid, smem, stream)
+                   : launch_decode<DT, 128, 16, true>(mk, mk, p, grid, smem, stream);
+}
+
+// TMA view of the INT8 K codes: [block][kv head][token][dim] bytes, one
+// 128-byte x 16-row box per tile, 128B swizzle.
+pkv_status encode_i8_key_map(CUtensorMap* map, const void* k8, int num_blocks, int n_kv, int head_dim) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(kBlockTokens),
+                              static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim);
+  const cuuint64_t strides[3] = {row, row * kBlockTokens, row * kBlockTokens * n_kv};
+  const cuuint32_t box[4] = {128, static_cast<cuuint32_t>(kBlockTokens), 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(k8), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
+// Scale rows and transposed V codes of the INT8 cache (null for 16-bit caches).
+struct KvI8 {
+  const float* k_scale;
+  const float* v_scale;
+};
 
 // Shared-memory ring of the prefix kernel: three stages of 64 tokens of K and V.
 constexpr int kPrefixStages = 3;
@@ -299,6 +328,53 @@ pkv_status paged_kv_copy_blocks(void* k_cache, void* v_cache, const int32_t* src
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+pkv_status paged_kv_append_int8(const void* k, const void* v, pkv_dtype dtype, const int64_t* slot_mapping,
+                                int32_t num_tokens, int8_t* k_cache, int8_t* v_cache, float* k_scale, float* v_scale,
+                                int32_t num_blocks, int32_t block_size, int32_t n_kv_heads, int32_t head_dim,
+                                void* stream) {
+  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || n_kv_heads <= 0 || head_dim <= 0)
+    return PKV_ERR_INVALID_ARG;
+  if (elem_bytes(dtype) == 0 || block_size != kBlockTokens || (head_dim != 64 && head_dim != 128))
+    return PKV_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u) || (reinterpret_cast<uintptr_t>(k) & 3u) ||
+      (reinterpret_cast<uintptr_t>(v) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+    return PKV_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  AppendI8Params p;
+  p.k = k;
+  p.v = v;
+  p.slot_mapping = slot_mapping;
+  p.k8 = k_cache;
+  p.v8 = v_cache;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  p.num_tokens = num_tokens;
+  p.n_kv_heads = n_kv_heads;
+  const int64_t warps = static_cast<int64_t>(num_tokens) * n_kv_heads;
+  const int64_t want = (warps + 7) / 8;  // 8 warps per 256-thread CTA
+  const int grid = static_cast<int>(want < int64_t(di.sm_count) * 8 ? want : int64_t(di.sm_count) * 8);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool d128 = head_dim == 128;
+  switch (dtype) {
+    case PKV_F32:
+      d128 ? pkv_append_i8_kernel<kF32, 128><<<grid, 256, 0, s>>>(p) : pkv_append_i8_kernel<kF32, 64><<<grid, 256, 0, s>>>(p);
+      break;
+    case PKV_F16:
+      d128 ? pkv_append_i8_kernel<kF16, 128><<<grid, 256, 0, s>>>(p) : pkv_append_i8_kernel<kF16, 64><<<grid, 256, 0, s>>>(p);
+      break;
+    default:
+      d128 ? pkv_append_i8_kernel<kBF16, 128><<<grid, 256, 0, s>>>(p)
+           : pkv_append_i8_kernel<kBF16, 64><<<grid, 256, 0, s>>>(p);
+      break;
+  }
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 pkv_status paged_attention_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                           pkv_dtype dtype, size_t* bytes) {
   return paged_attention_workspace_size_ex(batch, n_q_heads, n_kv_heads, head_dim, dtype, nullptr, bytes);
@@ -331,10 +407,16 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
                        float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
                        void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes, void* stream,
                        const pkv_decode_options* options, const float* init, const int32_t* seq_group,
-                       int32_t n_groups) {
+                       int32_t n_groups, const KvI8* i8 = nullptr) {
   pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                     num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
-  if (st != PKV_OK || batch == 0) return st;
+  if (st != PKV_OK) return st;
+  if (i8) {
+    if (dtype == PKV_F32 || head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (!i8->k_scale || !i8->v_scale || !aligned16(i8->k_scale) || !aligned16(i8->v_scale))
+      return PKV_ERR_INVALID_ARG;
+  }
+  if (batch == 0) return st;
   pkv_decode_options opt = {};
   if (options) {
     opt = *options;
@@ -352,8 +434,9 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   const int group = n_q_heads / n_kv_heads;
-  const int gp = heads_per_segment(group, dtype, opt.force_simt == 1);
-  const int gpad = gp == 1 ? 0 : (gp <= 8 ? 8 : 16);
+  const int gp = heads_per_segment(group, dtype, opt.force_simt == 1 && !i8);
+  // The INT8 cache always takes the tensor-core consumer (8 rows at least).
+  const int gpad = (gp == 1 && !i8) ? 0 : (gp <= 8 ? 8 : 16);
   // One CTA per SM at most (the kernel's grid barrier needs every CTA
   // resident), so the unit count is capped at one per consumer warp of
   // every SM.
@@ -364,7 +447,9 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   // Ring depth: as many slots per consumer warp as shared memory allows
   // (at most 4; 2 with ten consumer warps and 8 KiB tiles).
   const int es = elem_bytes(dtype);
-  const size_t stage_bytes = static_cast<size_t>(2) * (head_dim * es / 128) * kBoxBytes;
+  // INT8: K codes (16 x head_dim bytes) plus transposed V codes and 2 x 16 scales.
+  const size_t stage_bytes = i8 ? static_cast<size_t>(2) * head_dim * kBlockTokens + 2 * kBlockTokens * 4
+                                : static_cast<size_t>(2) * (head_dim * es / 128) * kBoxBytes;
   // 1 KiB alignment slack, abort word, prefix sums and clamped lengths, and
   // 256 bytes for the kernel's static shared memory.
   const size_t qbuf_bytes = static_cast<size_t>(gpad == 0 ? 1 : gpad) * head_dim * es;
@@ -391,10 +476,18 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   }
 
   CUtensorMap mk, mv;
-  st = encode_cache_map(&mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
-  if (st == PKV_OK) st = encode_cache_map(&mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+  if (i8) {
+    st = encode_i8_key_map(&mk, k_cache, num_blocks, n_kv_heads, head_dim);
+  } else {
+    st = encode_cache_map(&mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
+    if (st == PKV_OK) st = encode_cache_map(&mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+  }
 
   DecodeParams p;
+  p.v_i8 = i8 ? static_cast<const int8_t*>(v_cache) : nullptr;
+  p.k_scale = i8 ? i8->k_scale : nullptr;
+  p.v_scale = i8 ? i8->v_scale : nullptr;
+  p.n_kv_heads = n_kv_heads;
   p.q = q;
   p.out = out;
   p.block_tables = block_tables;
@@ -421,7 +514,9 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   p.seq_group = seq_group;
   p.n_groups = n_groups;
 
-  if (st == PKV_OK) {
+  if (st == PKV_OK && i8) {
+    st = dtype == PKV_F16 ? dispatch_i8<kF16>(gpad, mk, p, grid, smem, s) : dispatch_i8<kBF16>(gpad, mk, p, grid, smem, s);
+  } else if (st == PKV_OK) {
     switch (dtype) {
       case PKV_F32: st = dispatch_dim<kF32>(head_dim, gpad, mk, mv, p, grid, smem, s); break;
       case PKV_F16: st = dispatch_dim<kF16>(head_dim, gpad, mk, mv, p, grid, smem, s); break;
@@ -456,6 +551,18 @@ pkv_status paged_attention_decode(const void* q, const void* k_cache, const void
   return paged_attention_decode_ex(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                    num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype,
                                    workspace, workspace_bytes, stream, nullptr);
+}
+
+pkv_status paged_attention_decode_int8(const void* q, const int8_t* k_cache, const int8_t* v_cache,
+                                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                       int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
+                                       int32_t num_blocks, float scale, int32_t n_q_heads, int32_t n_kv_heads,
+                                       int32_t head_dim, int32_t block_size, void* out, pkv_dtype dtype,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  const KvI8 i8 = {k_scale, v_scale};
+  return decode_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
+                     n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, workspace, workspace_bytes, stream,
+                     nullptr, nullptr, nullptr, 0, &i8);
 }
 
 // ---------------------------------------------------------------------------

@@ -110,6 +110,16 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Contiguous bulk copy global -> this CTA's shared memory, completing on an
+// mbarrier (both addresses 16-byte aligned, bytes a multiple of 16).  No
+// multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // cp.async (16-byte global -> shared copies) and bulk L2 prefetch
 // ---------------------------------------------------------------------------
@@ -182,6 +192,26 @@ __device__ __forceinline__ void unpack2(uint32_t v, float& lo, float& hi) {
     unsigned short l = static_cast<unsigned short>(v & 0xffffu), h = static_cast<unsigned short>(v >> 16);
     asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(l));
     asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(h));
+  }
+}
+
+// Two signed 8-bit codes (bytes 2*half and 2*half + 1 of w) to a packed
+// 16-bit pair, exactly.  The code b is offset to b + 128 (flip of the sign
+// bit) and placed in the mantissa of a float whose value is then 2^23 +
+// b + 128 (bf16: through fp32), or of a half whose value is 1024 + b + 128
+// (f16); subtracting the bias leaves b.
+template <bool kBf16>
+__device__ __forceinline__ uint32_t i8x2_to_16x2(uint32_t w, int half) {
+  const uint32_t u = w ^ 0x80808080u;
+  if constexpr (kBf16) {
+    const float lo = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u + 2 * half)) - 8388736.0f;
+    const float hi = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541u + 2 * half)) - 8388736.0f;
+    return pack2<true>(lo, hi);
+  } else {
+    const uint32_t h2 = __byte_perm(u, 0x64646464u, half == 0 ? 0x5140u : 0x5342u);
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h2), "r"(0x64806480u));
+    return r;
   }
 }
 

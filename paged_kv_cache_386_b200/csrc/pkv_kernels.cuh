@@ -1,6 +1,7 @@
 // pkv_kernels.cuh -- sm_100a kernels of the paged KV cache:
 //   pkv_append_kernel   scatter of new K/V rows into their slots
 //   pkv_copy_blocks_kernel  whole-block copies for copy-on-write
+//   pkv_append_i8_kernel    quantising append into the INT8 cache
 //   pkv_decode_kernel   persistent split-KV paged decode attention, with the
 //                       log-sum-exp merge of split contexts after a grid-wide
 //                       barrier
@@ -159,6 +160,99 @@ __global__ void __launch_bounds__(256) pkv_copy_blocks_kernel(const CopyParams p
 }
 
 // ---------------------------------------------------------------------------
+// INT8 cache append (quantised KV)
+// ---------------------------------------------------------------------------
+// Byte position of block offset j in a transposed V row: the four tokens a
+// tensor-core lane t needs for one P V step (2t, 2t + 1, 2t + 8, 2t + 9) are
+// bytes 4t .. 4t + 3.
+__host__ __device__ __forceinline__ int vpos_i8(int j) { return 4 * ((j & 7) >> 1) + 2 * (j >> 3) + (j & 1); }
+
+struct AppendI8Params {
+  const void* k;
+  const void* v;
+  const int64_t* slot_mapping;
+  int8_t* k8;       // [num_blocks][n_kv][16][D]
+  int8_t* v8;       // [num_blocks][n_kv][D][16], token order vpos_i8
+  float* k_scale;   // [num_blocks][n_kv][16]
+  float* v_scale;
+  int64_t num_slots;
+  int32_t num_tokens;
+  int32_t n_kv_heads;
+};
+
+// Symmetric quantisation of one row held D / 32 elements per lane (lane owns
+// dims [lane * EPL, lane * EPL + EPL)): scale = amax / 127, codes
+// rint(x / scale), both in binary32 (IEEE division: the build uses no fast
+// math).
+template <int EPL>
+__device__ __forceinline__ float quantise_row(const float (&x)[EPL], int8_t (&c)[EPL]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float scale = amax / 127.0f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    float q = amax == 0.f ? 0.f : rintf(x[e] / scale);
+    q = fminf(fmaxf(q, -127.f), 127.f);
+    c[e] = static_cast<int8_t>(q);
+  }
+  return scale;
+}
+
+template <int DT, int D>
+__global__ void __launch_bounds__(256) pkv_append_i8_kernel(const AppendI8Params p) {
+  using T = typename DTypeInfo<DT>::T;
+  constexpr int EPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t n_rows = static_cast<int64_t>(p.num_tokens) * p.n_kv_heads;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < n_rows;
+       r += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int64_t i = r / p.n_kv_heads;
+    const int h = static_cast<int>(r % p.n_kv_heads);
+    const int64_t s = __ldg(p.slot_mapping + i);
+    if (s < 0) continue;  // padding token
+    if (s >= p.num_slots) {
+      if (lane == 0 && h == 0) flag_error(PKV_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t blk = s / kBlockTokens;
+    const int off = static_cast<int>(s % kBlockTokens);
+    const size_t bh = static_cast<size_t>(blk) * p.n_kv_heads + h;
+    const size_t src = static_cast<size_t>(r) * D + lane * EPL;
+    float xk[EPL], xv[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      if constexpr (DT == kF32) {
+        xk[e] = __ldg(static_cast<const float*>(p.k) + src + e);
+        xv[e] = __ldg(static_cast<const float*>(p.v) + src + e);
+      } else {
+        const uint16_t bk = __ldg(reinterpret_cast<const unsigned short*>(p.k) + src + e);
+        const uint16_t bv = __ldg(reinterpret_cast<const unsigned short*>(p.v) + src + e);
+        float lo, hi;
+        unpack2<DT == kBF16>(static_cast<uint32_t>(bk) | (static_cast<uint32_t>(bv) << 16), lo, hi);
+        xk[e] = lo;
+        xv[e] = hi;
+      }
+    }
+    int8_t ck[EPL], cv[EPL];
+    const float sk = quantise_row<EPL>(xk, ck);
+    const float sv = quantise_row<EPL>(xv, cv);
+    int8_t* krow = p.k8 + (bh * kBlockTokens + off) * D + lane * EPL;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) krow[e] = ck[e];
+    const int vp = vpos_i8(off);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) p.v8[(bh * D + lane * EPL + e) * kBlockTokens + vp] = cv[e];
+    if (lane == 0) {
+      p.k_scale[bh * kBlockTokens + off] = sk;
+      p.v_scale[bh * kBlockTokens + off] = sv;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Decode
 // ---------------------------------------------------------------------------
 struct DecodeParams {
@@ -167,6 +261,11 @@ struct DecodeParams {
   const int32_t* block_tables;
   const int32_t* context_lens;
   float* records;  // [chunks][2][rec_floats]: O[gp][D], m[gp], l[gp]
+  // INT8 cache only: transposed V codes and the per-token scales.
+  const int8_t* v_i8;
+  const float* k_scale;
+  const float* v_scale;
+  int32_t n_kv_heads;
   int4* meta;      // [chunks]: split segment whose first piece the chunk holds
   int* sched;      // [0]: claim counter of the balancing chunks (0 between launches)
   // Optional initial softmax state per (sequence, query head) -- the shared
@@ -404,8 +503,7 @@ struct MmaConsumer {
     }
   }
 
-  __device__ __forceinline__ void tile(uint32_t kbase, int nv, float scale_log2, int lane) {
-    const uint32_t vbase = kbase + (D / (128 / ES)) * kBoxBytes;
+  __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, int nv, float scale_log2, int lane) {
     const int t = lane & 3;
     const int mi = lane >> 3, rr = lane & 7;
 
@@ -621,8 +719,7 @@ struct SimtConsumer {
     l = tp == 0 ? __ldg(p.init + nqb * D + nqb + rowi) : 0.f;
   }
 
-  __device__ __forceinline__ void tile(uint32_t kbase, int nv, float scale_log2, int lane) {
-    const uint32_t vbase = kbase + (D / (128 / ES)) * kBoxBytes;
+  __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, int nv, float scale_log2, int lane) {
     const int tp = lane & 7, sub = lane >> 3;
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
@@ -733,13 +830,184 @@ struct SimtConsumer {
   }
 };
 
-template <int DT, int D, int GPAD>
+// ---- tensor-core consumer over the INT8 cache (head_dim 128) ----
+// K tile: 16 rows of 128 one-byte codes, TMA 128B swizzle (16-byte chunk c of
+// row r at chunk c ^ (r % 8)).  V tile: 128 rows (dims) of 16 bytes (tokens,
+// in vpos_i8 order).  Then 16 fp32 K scales and 16 V scales (token order).
+// The dot product over the head dim does not depend on the order of the
+// dims, so lane t owns dims [32t, 32t + 32) for every k-step: k-step ks
+// takes dims 32t + 4ks + {0, 1} as the fragment's columns 2t, 2t + 1 and
+// 32t + 4ks + {2, 3} as columns 2t + 8, 2t + 9, for Q and K alike.  A lane's
+// K codes of one row are then two 16-byte loads that the swizzle keeps free of
+// bank conflicts.  Codes become exact 16-bit values (i8x2_to_16x2); the K
+// scale multiplies the score columns, the V scale the probabilities.
+template <int DT, int GPAD>
+struct MmaConsumerI8 : MmaConsumer<DT, 128, GPAD> {
+  using Base = MmaConsumer<DT, 128, GPAD>;
+  using T = typename Base::T;
+  static constexpr bool kBf16 = Base::kBf16;
+  static constexpr int D = 128;
+  static constexpr int KS = D / 16;
+  static constexpr int NT = D / 8;
+  using Base::l;
+  using Base::m;
+  using Base::o;
+  using Base::qa;
+
+  __device__ __forceinline__ void begin(const uint8_t* qbuf, int gp, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const T* qb = reinterpret_cast<const T*>(qbuf);
+    const bool r0 = g < gp;
+    const bool r1 = (GPAD == 16) && (g + 8 < gp);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int c = 32 * t + 4 * ks;
+      const uint2 x0 = r0 ? *reinterpret_cast<const uint2*>(qb + g * D + c) : make_uint2(0u, 0u);
+      const uint2 x1 = r1 ? *reinterpret_cast<const uint2*>(qb + (g + 8) * D + c) : make_uint2(0u, 0u);
+      qa[ks][0] = x0.x;
+      qa[ks][2] = x0.y;
+      qa[ks][1] = x1.x;
+      qa[ks][3] = x1.y;
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, int nv, float scale_log2, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t sbase = vbase + D * kBlockTokens;  // K scales, then V scales
+
+    // S = Q K^T for tokens g (n-tile 0) and g + 8 (n-tile 1).
+    float s[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      const int row = nt * 8 + g;
+      uint4 c0, c1;
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w)
+                   : "r"(kbase + row * 128 + (((2 * t) ^ (row & 7)) << 4)));
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
+                   : "r"(kbase + row * 128 + (((2 * t + 1) ^ (row & 7)) << 4)));
+      const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks)
+        mma_16816<kBf16>(s[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], i8x2_to_16x2<kBf16>(w[ks], 0),
+                         i8x2_to_16x2<kBf16>(w[ks], 1));
+    }
+    // K scales of this lane's score columns: tokens 2t, 2t + 1 and 2t + 8, 2t + 9.
+    float2 ks0, ks1;
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(ks0.x), "=f"(ks0.y) : "r"(sbase + 8 * t));
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(ks1.x), "=f"(ks1.y) : "r"(sbase + 32 + 8 * t));
+    s[0][0] *= ks0.x;
+    s[0][1] *= ks0.y;
+    s[0][2] *= ks0.x;
+    s[0][3] *= ks0.y;
+    s[1][0] *= ks1.x;
+    s[1][1] *= ks1.y;
+    s[1][2] *= ks1.x;
+    s[1][3] *= ks1.y;
+
+    // Online softmax (as in the 16-bit consumer).
+    constexpr int kRows = (GPAD == 16) ? 2 : 1;
+    float pr[2][2][2];
+    bool grow = false;
+    float alpha[2] = {1.f, 1.f};
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      float x[2][2];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tok = nt * 8 + 2 * t + e;
+          x[nt][e] = (tok < nv) ? s[nt][2 * r + e] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[nt][e]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mn = fmaxf(m[r], mx);
+      if (mn > m[r]) {
+        grow = true;
+        alpha[r] = exp2f(m[r] - mn);
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          pr[r][nt][e] = exp2f(x[nt][e] - mn);
+          sum += pr[r][nt][e];
+        }
+      l[r] = l[r] * alpha[r] + sum;
+      m[r] = mn;
+    }
+    if (__any_sync(0xffffffffu, grow)) {
+      const float a_lo = alpha[0];
+      const float a_hi = (GPAD == 16) ? alpha[1] : alpha[0];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] *= a_lo;
+        o[n][1] *= a_lo;
+        o[n][2] *= a_hi;
+        o[n][3] *= a_hi;
+      }
+    }
+
+    // V scales folded into the probabilities; tokens past the context (whose
+    // scales may be anything, NaN included) get 0.
+    float2 vs0, vs1;
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(vs0.x), "=f"(vs0.y) : "r"(sbase + 64 + 8 * t));
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(vs1.x), "=f"(vs1.y) : "r"(sbase + 96 + 8 * t));
+    const float vsc[2][2] = {{vs0.x, vs0.y}, {vs1.x, vs1.y}};
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) pr[r][nt][e] = (nt * 8 + 2 * t + e < nv) ? pr[r][nt][e] * vsc[nt][e] : 0.f;
+
+    uint32_t pa0 = pack2<kBf16>(pr[0][0][0], pr[0][0][1]);
+    uint32_t pa2 = pack2<kBf16>(pr[0][1][0], pr[0][1][1]);
+    uint32_t pa1, pa3;
+    if constexpr (GPAD == 16) {
+      pa1 = pack2<kBf16>(pr[1][0][0], pr[1][0][1]);
+      pa3 = pack2<kBf16>(pr[1][1][0], pr[1][1][1]);
+    } else {
+      float h00, h01, h10, h11;
+      unpack2<kBf16>(pa0, h00, h01);
+      unpack2<kBf16>(pa2, h10, h11);
+      pa1 = pack2<kBf16>(pr[0][0][0] - h00, pr[0][0][1] - h01);
+      pa3 = pack2<kBf16>(pr[0][1][0] - h10, pr[0][1][1] - h11);
+    }
+
+    // O += P V: V^T row 8n + g holds dim 8n + g of all 16 tokens; bytes 4t ..
+    // 4t + 3 are tokens 2t, 2t + 1, 2t + 8, 2t + 9 (codes are finite, so the
+    // rows past the context need no mask: their probabilities are 0).
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      uint32_t w;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(vbase + (8 * n + g) * kBlockTokens + 4 * t));
+      mma_16816<kBf16>(o[n], pa0, pa1, pa2, pa3, i8x2_to_16x2<kBf16>(w, 0), i8x2_to_16x2<kBf16>(w, 1));
+    }
+  }
+};
+
+template <int DT, int D, int GPAD, bool kI8 = false>
 struct ConsumerFor {
   using type = MmaConsumer<DT, D, GPAD>;
 };
 template <int DT, int D>
-struct ConsumerFor<DT, D, 0> {
+struct ConsumerFor<DT, D, 0, false> {
   using type = SimtConsumer<DT, D>;
+};
+template <int DT, int GPAD>
+struct ConsumerFor<DT, 128, GPAD, true> {
+  using type = MmaConsumerI8<DT, GPAD>;
 };
 
 // Four fp32 values rounded to the output dtype and stored together.
@@ -896,7 +1164,8 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
 // producer/consumer pipeline; a grid-wide barrier follows (every wait before
 // it is bounded, so every thread reaches it); phase 2 merges split segments
 // and zero-fills the rows of empty sequences.
-template <int DT, int D, int GPAD>
+// kI8: the cache holds INT8 codes and per-token scales (MmaConsumerI8).
+template <int DT, int D, int GPAD, bool kI8>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     pkv_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeParams p) {
@@ -904,16 +1173,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   constexpr int X = 128 / ES;                      // elements per swizzle row
   constexpr int Y = D / X;                         // boxes per tile
   constexpr int kTileBytes = Y * kBoxBytes;
-  constexpr int kStageBytes = 2 * kTileBytes;
+  // Ring slots: the K region (1 KiB aligned for the swizzle) and, for INT8,
+  // a second region with the transposed V codes and the two scale rows.
+  constexpr int kRingStride = kI8 ? D * kBlockTokens : 2 * kTileBytes;
+  constexpr int kVStride = kI8 ? D * kBlockTokens + 2 * kBlockTokens * 4 : 0;
+  constexpr int kStageBytes = kI8 ? kRingStride + kVStride : 2 * kTileBytes;  // bytes landing per slot
   constexpr int kQBufBytes = (GPAD == 0 ? 1 : GPAD) * D * ES;
-  using Consumer = typename ConsumerFor<DT, D, GPAD>::type;
+  using Consumer = typename ConsumerFor<DT, D, GPAD, kI8>::type;
   using OutT = typename DTypeInfo<DT>::T;
+  static_assert(!kI8 || (D == 128 && GPAD != 0), "INT8 cache: head_dim 128, tensor-core consumer");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const int n_slots = kConsumerWarps * p.stages;
-  uint8_t* qbufs = ring + static_cast<size_t>(n_slots) * kStageBytes;  // [warps][kQBufBytes]
+  uint8_t* vring = ring + static_cast<size_t>(n_slots) * kRingStride;                 // INT8: [slots][kVStride]
+  uint8_t* qbufs = vring + static_cast<size_t>(n_slots) * kVStride;  // [warps][kQBufBytes]
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(qbufs + kConsumerWarps * kQBufBytes);
   uint64_t* empty_bar = full_bar + n_slots;
   int4* slot_info = reinterpret_cast<int4*>(empty_bar + n_slots);  // [n_slots]: next chunk, from the producer
@@ -1052,13 +1327,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                        "r"(t0.info.y), "r"(t0.info.z), "r"(t0.info.w)
                        : "memory");  // published to the consumer by the arrive below
           mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
-          uint8_t* sk = ring + static_cast<size_t>(slot) * kStageBytes;
+          uint8_t* sk = ring + static_cast<size_t>(slot) * kRingStride;
+          if constexpr (kI8) {
+            const size_t bh = static_cast<size_t>(ph) * p.n_kv_heads + t0.kvh;
+            uint8_t* sv = vring + static_cast<size_t>(slot) * kVStride;
+            tma_load_4d(sk, &tm_k, &full_bar[slot], 0, 0, t0.kvh, ph);
+            bulk_load(sv, p.v_i8 + bh * D * kBlockTokens, D * kBlockTokens, &full_bar[slot]);
+            bulk_load(sv + D * kBlockTokens, p.k_scale + bh * kBlockTokens, kBlockTokens * 4, &full_bar[slot]);
+            bulk_load(sv + D * kBlockTokens + kBlockTokens * 4, p.v_scale + bh * kBlockTokens, kBlockTokens * 4,
+                      &full_bar[slot]);
+          } else {
 #pragma unroll
-          for (int y = 0; y < Y; ++y)
-            tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, t0.kvh, ph);
+            for (int y = 0; y < Y; ++y)
+              tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, t0.kvh, ph);
 #pragma unroll
-          for (int y = 0; y < Y; ++y)
-            tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, t0.kvh, ph);
+            for (int y = 0; y < Y; ++y)
+              tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, t0.kvh, ph);
+          }
           ++issued;
           if (++stage == p.stages) {
             stage = 0;
@@ -1182,7 +1467,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           }
         }
         const int nv = min(kBlockTokens, wk.ctx - wk.j * kBlockTokens);
-        cs.tile(smem_u32(ring + static_cast<size_t>(slot) * kStageBytes), nv, p.scale_log2, lane);
+        const uint32_t kaddr = smem_u32(ring + static_cast<size_t>(slot) * kRingStride);
+        const uint32_t vaddr = kI8 ? smem_u32(vring + static_cast<size_t>(slot) * kVStride) : kaddr + kTileBytes;
+        cs.tile(kaddr, vaddr, nv, p.scale_log2, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[slot]);
         if (++stage == p.stages) {

@@ -10,6 +10,8 @@
   entries read and the context lengths.  A physical block shared by several
   sequences counts once ("unique"); the per-sequence sum is the "logical"
   traffic a kernel without reuse would pay.
+  With ``kv_int8`` a tile is the INT8 cache's: one-byte codes and one fp32
+  scale per token.
 * :func:`append_traffic` counts the bytes of one ``paged_kv_append`` call.
 """
 
@@ -30,7 +32,9 @@ def blocks_for(n_tokens: int, block_size: int = BLOCK_SIZE) -> int:
 
 def decode_traffic(block_tables: torch.Tensor, context_lens: torch.Tensor, n_q_heads: int,
                    n_kv_heads: int, head_dim: int, elem_bytes: int,
-                   block_size: int = BLOCK_SIZE) -> dict:
+                   block_size: int = BLOCK_SIZE, kv_int8: bool = False) -> dict:
+    """``elem_bytes`` is the element size of q and out; with ``kv_int8`` the
+    cache holds one-byte codes plus one fp32 scale per token for K and V."""
     lens = [int(x) for x in context_lens.tolist()]
     bt = block_tables.cpu()
     used = []
@@ -41,7 +45,8 @@ def decode_traffic(block_tables: torch.Tensor, context_lens: torch.Tensor, n_q_h
         if nb:
             used.append(bt[b, :nb])
     unique_blocks = int(torch.unique(torch.cat(used)).numel()) if used else 0
-    tile = block_size * head_dim * elem_bytes  # one kv head of one block, K or V
+    # One kv head of one block, K or V (INT8: codes plus a scale per token).
+    tile = block_size * (head_dim + 4) if kv_int8 else block_size * head_dim * elem_bytes
     kv_unique = unique_blocks * n_kv_heads * tile * 2
     kv_logical = logical_blocks * n_kv_heads * tile * 2
     batch = len(lens)

@@ -58,6 +58,7 @@ class DecodeWorkload:
     distinct_blocks: int
     appended: bool
     meta: dict = field(default_factory=dict)
+    q_len: int = 1  # new tokens (queries) per sequence; q is [B, q_len, n_q, d] when > 1
 
     @property
     def batch(self) -> int:
@@ -107,6 +108,7 @@ def build_workload(
     scale: float | None = None,
     block_size: int = BLOCK_SIZE,
     max_blocks_per_seq: int | None = None,
+    q_len: int = 1,
 ) -> DecodeWorkload:
     """Lay out ``len(lens)`` sequences in a shuffled pool of physical blocks.
 
@@ -116,7 +118,13 @@ def build_workload(
     ch. 15 §15.6 and "LLM Primer VI" ch. 8 §8.1).  ``prefix`` must be a
     multiple of ``block_size`` and shorter than every member's context, so
     that the appended token lands in a private block.
+
+    ``q_len`` > 1 makes the last ``q_len`` tokens of every context new (their
+    slots start at the fill value and ``k_new``/``v_new`` hold them, sequence
+    major), with ``q`` of shape ``[B, q_len, n_q, d]``: several queries per
+    sequence, as for verifying a draft or a prefill chunk.
     """
+    assert q_len >= 1 and (q_len == 1 or (append and not sink_tokens))
     B = len(lens)
     g_struct = torch.Generator().manual_seed(seed)
     g_data = torch.Generator().manual_seed(seed + 7919)
@@ -164,7 +172,7 @@ def build_workload(
     # in the cache (the appended token's slot stays at the fill value).
     valid = torch.zeros(pool_blocks, dtype=torch.int64)
     for b in range(B):
-        have = lens[b] - 1 if append else lens[b]
+        have = lens[b] - q_len if append else lens[b]
         for j, dblk in enumerate(seq_blocks[b]):
             n = min(block_size, have - j * block_size)
             if n <= 0:
@@ -192,20 +200,21 @@ def build_workload(
                 n = min(sink_tokens, lens[b] - (1 if append else 0))
                 k_cache[p, :, :n, :] *= sink_scale
 
-    q = _randn((B, n_q_heads, head_dim), dtype, g_data)
-    k_new = _randn((B, n_kv_heads, head_dim), dtype, g_data)
-    v_new = _randn((B, n_kv_heads, head_dim), dtype, g_data)
+    q = _randn((B, n_q_heads, head_dim) if q_len == 1 else (B, q_len, n_q_heads, head_dim), dtype, g_data)
+    k_new = _randn((B * q_len, n_kv_heads, head_dim), dtype, g_data)
+    v_new = _randn((B * q_len, n_kv_heads, head_dim), dtype, g_data)
     if append and sink_tokens:
         for b in range(B):
             if lens[b] - 1 < sink_tokens:
                 k_new[b] *= sink_scale
 
-    slot = torch.full((B,), -1, dtype=torch.int64)
+    slot = torch.full((B * q_len,), -1, dtype=torch.int64)
     if append:
         for b in range(B):
-            t = lens[b] - 1
-            if t >= 0:
-                slot[b] = int(block_tables[b, t // block_size]) * block_size + t % block_size
+            for i in range(q_len):
+                t = lens[b] - q_len + i
+                if t >= 0:
+                    slot[b * q_len + i] = int(block_tables[b, t // block_size]) * block_size + t % block_size
 
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
@@ -216,6 +225,7 @@ def build_workload(
         head_dim=head_dim, block_size=block_size, distinct_blocks=n_distinct, appended=append,
         meta={"seed": seed, "placement": placement, "pool_blocks": pool_blocks,
               "shared_blocks": shared_of, "groups": groups or []},
+        q_len=q_len,
     )
 
 
@@ -275,7 +285,7 @@ def cached_token_rows(w: DecodeWorkload):
     bs = w.block_size
     slots = set()
     for b, n in enumerate(w.lens()):
-        held = n - 1 if w.appended else n
+        held = n - w.q_len if w.appended else n
         for j in range(held):
             slots.add(int(w.block_tables[b, j // bs]) * bs + j % bs)
     sl = torch.tensor(sorted(slots), dtype=torch.int64)
