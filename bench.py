@@ -199,9 +199,9 @@ def run_ours(args) -> None:
     out = torch.empty_like(q)
     if int8:
         # The same tokens quantised into the INT8 cache (untimed set-up).
-        k8, v8, ks8, vs8 = pkv.int8_cache(w.num_blocks, w.n_kv_heads, w.head_dim, device=dev)
+        kv8 = pkv.int8_cache(w.num_blocks, w.n_kv_heads, w.head_dim, device=dev)
         kr, vr, sl = W.cached_token_rows(w)
-        pkv.paged_kv_append_int8(kr.to(dev), vr.to(dev), sl.to(dev), k8, v8, ks8, vs8)
+        pkv.paged_kv_append_int8(kr.to(dev), vr.to(dev), sl.to(dev), kv8)
         del kc, vc, kr, vr
         torch.cuda.synchronize(dev)
     if args.cascade:
@@ -217,14 +217,13 @@ def run_ours(args) -> None:
 
     def append(stream_=None):
         if int8:
-            pkv.paged_kv_append_int8(k_new, v_new, slots, k8, v8, ks8, vs8, stream=stream_)
+            pkv.paged_kv_append_int8(k_new, v_new, slots, kv8, stream=stream_)
         else:
             pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream_)
 
     def decode(stream_=None):
         if int8:
-            pkv.paged_attention_decode_int8(q, k8, v8, ks8, vs8, bt, cl, w.scale, out=out, workspace=ws,
-                                            stream=stream_)
+            pkv.paged_attention_decode_int8(q, kv8, bt, cl, w.scale, out=out, workspace=ws, stream=stream_)
         elif args.cascade:
             pkv.paged_attention_decode_cascade(q, kc, vc, c_pt, c_pl, c_sg, c_bt, c_cl, w.scale, out=out,
                                                workspace=ws, stream=stream_)
@@ -379,7 +378,8 @@ def run_ours(args) -> None:
                        "warmup_steps_run": warm_steps,
                        "launch": launch_note,
                        "decode": "cascade (shared prefix once per group)" if args.cascade else "paged decode",
-                       "kv_cache": ("INT8 codes + fp32 scale per (token, kv head)" if int8
+                       "kv_cache": ("INT8 codes + fp32 scale per (token, kv head), one 4224-byte record per "
+                                    "(block, kv head)" if int8
                                     else W.DTYPE_NAMES[w.dtype])},
             "tokens_per_s_per_layer": round(tokens_per_s, 1),
             "kv_bytes_per_step": kv_bytes,

@@ -385,39 +385,46 @@ pkv_status pkv_bm_refcount(const pkv_block_manager* bm, int32_t block, int32_t* 
  * INT8 paged KV cache (quantised KV, "Transformer anatomy" ch. 15 §15.7:
  * 8-bit K and V halve the cache bytes for a small loss of accuracy).
  *
- * Format (block_size 16):
- *   k_cache  int8 [num_blocks][n_kv_heads][16][head_dim]
- *   v_cache  int8 [num_blocks][n_kv_heads][head_dim][16]; in every row the
- *            token at block offset j sits at byte
- *              4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2)
- *   k_scale, v_scale  fp32 [num_blocks][n_kv_heads][16]
+ * Format (block_size 16, head dim d = 64 or 128): one byte array
+ * kv_cache[num_blocks][n_kv_heads][R], R = 32 * d + 128 (4224 at d = 128),
+ * holding one record per (block, kv head):
+ *   bytes [0, 16 d)        K codes: row j (block offset j) of d bytes; its
+ *                          16-byte chunk c is stored at chunk position
+ *                          c ^ (j % min(8, d / 16));
+ *   bytes [16 d, 32 d)     V codes, transposed: row e (dim e) of 16 bytes;
+ *                          the token at block offset j is at byte
+ *                          4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2);
+ *   bytes [32 d, 32 d + 64)        16 fp32 K scales, by block offset;
+ *   bytes [32 d + 64, 32 d + 128)  16 fp32 V scales.
  * A (token, kv head) row x of K or V is stored as codes
  *   c_e = rint(x_e / s), s = max_e |x_e| / 127 (binary32 division, round half
  *   to even; all codes 0 when the row is 0), and read as s * c_e.
+ * The record is laid out so that a decode moves it with one contiguous copy
+ * and reads it from shared memory without bank conflicts.
  * ------------------------------------------------------------------------ */
 
 /*
  * paged_kv_append_int8 -- quantise and write the K/V of new tokens into
- * their slots of the INT8 cache (slot semantics as paged_kv_append; the
- * codes and scales are bit-exact with the definition above).
+ * their slots of the INT8 cache (slot semantics as paged_kv_append; codes and
+ * scales are bit-exact with the definition above).
  *
- *   k, v    : device, [num_tokens][n_kv_heads][head_dim], `dtype` (f32, f16, bf16)
- *   head_dim: 64 or 128
+ *   k, v     : device, [num_tokens][n_kv_heads][head_dim], `dtype` (f32, f16, bf16)
+ *   kv_cache : device, 16-byte aligned, layout above; written in place
  */
 pkv_status paged_kv_append_int8(const void* k, const void* v, pkv_dtype dtype, const int64_t* slot_mapping,
-                                int32_t num_tokens, int8_t* k_cache, int8_t* v_cache, float* k_scale,
-                                float* v_scale, int32_t num_blocks, int32_t block_size, int32_t n_kv_heads,
-                                int32_t head_dim, void* stream);
+                                int32_t num_tokens, uint8_t* kv_cache, int32_t num_blocks, int32_t block_size,
+                                int32_t n_kv_heads, int32_t head_dim, void* stream);
 
 /*
  * paged_attention_decode_int8 -- paged_attention_decode over the INT8 cache:
- * the same attention with K_j = k_scale_j * k_code_j and V_j likewise.  q and
- * out are f16 or bf16 (`dtype`), head_dim 128; every head group runs on the
- * tensor cores.  Workspace as paged_attention_decode (same size function).
- * Tolerance against the fp64 oracle on the same codes: as the 16-bit decode.
+ * the same attention with K_j = s_j * (K codes) and V_j likewise.  q and out
+ * are f16 or bf16 (`dtype`), head_dim 128.  Q K^T runs on the integer tensor
+ * cores with every Q row put on a 14-bit grid (scale max|q| / 8191, two signed
+ * 8-bit halves); P V runs in f16.  Workspace as paged_attention_decode (same
+ * size function).  Tolerance against the fp64 oracle on the same codes: as
+ * the 16-bit decode.
  */
-pkv_status paged_attention_decode_int8(const void* q, const int8_t* k_cache, const int8_t* v_cache,
-                                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
+pkv_status paged_attention_decode_int8(const void* q, const uint8_t* kv_cache, const int32_t* block_tables,
                                        int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
                                        int32_t num_blocks, float scale, int32_t n_q_heads, int32_t n_kv_heads,
                                        int32_t head_dim, int32_t block_size, void* out, pkv_dtype dtype,

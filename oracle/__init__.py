@@ -70,10 +70,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_paged_decode_mq.argtypes = [p, p, p, i32, p, i32, p, i32, i32, ctypes.c_double, i32, i32, i32, i32,
                                            i32, p, i32]
     lib.oracle_paged_decode_mq.restype = ctypes.c_int
-    lib.oracle_kv_append_int8.argtypes = [p, p, i32, p, i32, p, p, p, p, i32, i32, i32, i32]
+    lib.oracle_kv_append_int8.argtypes = [p, p, i32, p, i32, p, i32, i32, i32, i32]
     lib.oracle_kv_append_int8.restype = ctypes.c_int
-    lib.oracle_paged_decode_int8.argtypes = [p, i32, p, p, p, p, p, i32, p, i32, i32, ctypes.c_double,
-                                             i32, i32, i32, i32, p, p, i32, i32]
+    lib.oracle_paged_decode_int8.argtypes = [p, i32, p, p, i32, p, i32, i32, ctypes.c_double, i32, i32, i32, i32,
+                                             p, p, i32, i32]
     lib.oracle_paged_decode_int8.restype = ctypes.c_int
     return lib
 
@@ -177,26 +177,26 @@ def workload_decode_mq(w, n_threads: int = 0, lib=None):
     return out, kc, vc
 
 
-def kv_append_int8(k, v, slot_mapping, k8, v8, k_scale, v_scale, lib=None) -> None:
-    """In-place quantising append into the INT8 cache (CPU tensors):
-    ``k8`` int8 ``[blocks, n_kv, 16, d]``, ``v8`` int8 ``[blocks, n_kv, d, 16]``
-    (token order within a row as documented in pkv_oracle.c), scales fp32
-    ``[blocks, n_kv, 16]``."""
+def kv_append_int8(k, v, slot_mapping, cache, lib=None) -> None:
+    """In-place quantising append into the INT8 cache, a CPU uint8 tensor
+    ``[blocks, n_kv, 32 * d + 128]`` of records (layout in pkv_oracle.c)."""
     lib = lib or load()
-    num_blocks, n_kv, bs, d = k8.shape
+    num_blocks, n_kv, rb = cache.shape
+    d = k.shape[-1]
+    assert rb == 32 * d + 128 and cache.dtype == torch.uint8
     k, v = k.contiguous(), v.contiguous()
     sm = slot_mapping.to(torch.int64).contiguous()
-    _check(lib.oracle_kv_append_int8(_ptr(k), _ptr(v), ORC_DTYPE[k.dtype], _ptr(sm), k.shape[0], _ptr(k8),
-                                     _ptr(v8), _ptr(k_scale), _ptr(v_scale), num_blocks, bs, n_kv, d))
+    _check(lib.oracle_kv_append_int8(_ptr(k), _ptr(v), ORC_DTYPE[k.dtype], _ptr(sm), k.shape[0], _ptr(cache),
+                                     num_blocks, 16, n_kv, d))
 
 
-def paged_decode_int8(q, k8, v8, k_scale, v_scale, block_tables, context_lens, scale: float, rows=None,
-                      n_threads: int = 0, lib=None) -> torch.Tensor:
+def paged_decode_int8(q, cache, block_tables, context_lens, scale: float, rows=None, n_threads: int = 0,
+                      lib=None) -> torch.Tensor:
     """fp64 ``[batch, n_q, d]`` attention over the dequantised INT8 cache."""
     lib = lib or load()
     B, n_q, d = q.shape
-    num_blocks, n_kv, bs, d2 = k8.shape
-    assert d2 == d
+    num_blocks, n_kv, rb = cache.shape
+    assert rb == 32 * d + 128
     q = q.contiguous()
     bt = block_tables.to(torch.int32).contiguous()
     cl = context_lens.to(torch.int32).contiguous()
@@ -206,9 +206,8 @@ def paged_decode_int8(q, k8, v8, k_scale, v_scale, block_tables, context_lens, s
     if rows is not None:
         r = torch.as_tensor(rows, dtype=torch.int32).reshape(-1, 2).contiguous()
         n_rows = r.shape[0]
-    _check(lib.oracle_paged_decode_int8(_ptr(q), ORC_DTYPE[q.dtype], _ptr(k8), _ptr(v8), _ptr(k_scale),
-                                        _ptr(v_scale), _ptr(bt), bt.shape[1], _ptr(cl), B, num_blocks,
-                                        float(scale), n_q, n_kv, d, bs, _ptr(out),
+    _check(lib.oracle_paged_decode_int8(_ptr(q), ORC_DTYPE[q.dtype], _ptr(cache), _ptr(bt), bt.shape[1], _ptr(cl),
+                                        B, num_blocks, float(scale), n_q, n_kv, d, 16, _ptr(out),
                                         _ptr(r) if r is not None else None, n_rows, n_threads))
     return out
 
@@ -216,16 +215,16 @@ def paged_decode_int8(q, k8, v8, k_scale, v_scale, block_tables, context_lens, s
 def workload_decode_int8(w, rows=None, n_threads: int = 0, lib=None):
     """Oracle for a workload held in the INT8 cache: every cached token and
     the appended one go through the quantising append, then the decode runs
-    over the dequantised cache.  Returns ``(out_fp64, k8, v8, k_scale, v_scale)``."""
+    over the dequantised cache.  Returns ``(out_fp64, cache)``."""
     import workloads as W
-    k8, v8, ks, vs = W.int8_cache_buffers(w)
+    cache = W.int8_cache_buffers(w)
     kr, vr, slots = W.cached_token_rows(w)
-    kv_append_int8(kr, vr, slots, k8, v8, ks, vs, lib=lib)
+    kv_append_int8(kr, vr, slots, cache, lib=lib)
     if w.appended:
-        kv_append_int8(w.k_new, w.v_new, w.slot_mapping, k8, v8, ks, vs, lib=lib)
-    out = paged_decode_int8(w.q, k8, v8, ks, vs, w.block_tables, w.context_lens, w.scale, rows=rows,
-                            n_threads=n_threads, lib=lib)
-    return out, k8, v8, ks, vs
+        kv_append_int8(w.k_new, w.v_new, w.slot_mapping, cache, lib=lib)
+    out = paged_decode_int8(w.q, cache, w.block_tables, w.context_lens, w.scale, rows=rows, n_threads=n_threads,
+                            lib=lib)
+    return out, cache
 
 
 def cpu_cores() -> int:

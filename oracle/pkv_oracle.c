@@ -299,12 +299,17 @@ int oracle_paged_decode_mq(const void* q, const void* k_cache, const void* v_cac
  * INT8 paged KV cache (quantised KV: "Transformer anatomy" ch. 15 §15.7, INT8
  * KV quantisation trades a small accuracy loss for half the bytes).
  *
- * Format (a reading: the pages fix neither granularity nor layout):
- *   k8      int8 [num_blocks][n_kv][block_size][head_dim]
- *   v8      int8 [num_blocks][n_kv][head_dim][block_size]; within a row, token
- *           j of the block sits at byte position
- *             vpos(j) = 4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2)
- *   k_scale, v_scale  fp32 [num_blocks][n_kv][block_size]
+ * Format (a reading: the pages fix neither granularity nor layout).  The
+ * cache is one byte array [num_blocks][n_kv][R], R = 32 * d + 128 for block
+ * size 16 and head dim d; the record of (block, kv head) holds
+ *   bytes [0, 16 d)        K codes: row j (block offset j) of d bytes, whose
+ *                          16-byte chunk c sits at chunk position c ^ (j % 8)
+ *                          (c ^ (j % 4) for d = 64);
+ *   bytes [16 d, 32 d)     V codes transposed: row e (dim e) of 16 bytes, the
+ *                          token at block offset j at byte vpos(j) =
+ *                          4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2);
+ *   bytes [32 d, 32 d + 64)       16 fp32 K scales (block offset order);
+ *   bytes [32 d + 64, 32 d + 128) 16 fp32 V scales.
  * Each (token, kv head) row x of K or V is quantised symmetrically:
  *   amax = max_e |x_e|, scale = amax / 127 (binary32 division),
  *   code_e = clamp(rint(x_e / scale), -127, 127) (binary32 division, rounding
@@ -314,6 +319,15 @@ int oracle_paged_decode_mq(const void* q, const void* k_cache, const void* v_cac
  * ---------------------------------------------------------------------------
  */
 static int vpos(int j) { return 4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2); }
+
+static size_t rec_bytes(int32_t d) { return (size_t)32 * d + 128; }
+
+/* Byte of K code (offset j, dim e) inside a record. */
+static size_t kpos(int j, int e, int32_t d) {
+  int chunks = d / 16;
+  int c = e / 16;
+  return (size_t)j * d + (size_t)((c ^ (j % (chunks < 8 ? chunks : 8))) * 16 + e % 16);
+}
 
 static void quantise_row(const void* src, size_t idx0, int dtype, int32_t d, int8_t* codes, float* scale_out) {
   float amax = 0.0f;
@@ -333,12 +347,12 @@ static void quantise_row(const void* src, size_t idx0, int dtype, int32_t d, int
   *scale_out = scale;
 }
 
-/* Append into the INT8 cache (the block-size must be 16: vpos is defined for it). */
+/* Append into the INT8 cache (block size 16, head dim 64 or 128). */
 int oracle_kv_append_int8(const void* k, const void* v, int32_t dtype, const int64_t* slot_mapping,
-                          int32_t num_tokens, int8_t* k8, int8_t* v8, float* k_scale, float* v_scale,
-                          int32_t num_blocks, int32_t block_size, int32_t n_kv_heads, int32_t head_dim) {
+                          int32_t num_tokens, uint8_t* cache, int32_t num_blocks, int32_t block_size,
+                          int32_t n_kv_heads, int32_t head_dim) {
   if (!elem_bytes(dtype) || num_tokens < 0 || num_blocks <= 0 || block_size != 16 || n_kv_heads <= 0 ||
-      head_dim <= 0)
+      (head_dim != 64 && head_dim != 128))
     return ORC_EINVAL;
   int8_t* codes = (int8_t*)malloc((size_t)head_dim);
   if (!codes) return ORC_ENOMEM;
@@ -350,17 +364,18 @@ int oracle_kv_append_int8(const void* k, const void* v, int32_t dtype, const int
       free(codes);
       return ORC_ESLOT;
     }
-    int64_t blk = s / block_size, off = s % block_size;
+    int64_t blk = s / block_size;
+    int off = (int)(s % block_size);
     for (int32_t h = 0; h < n_kv_heads; ++h) {
       size_t src = ((size_t)i * n_kv_heads + h) * head_dim;
-      size_t bh = (size_t)blk * n_kv_heads + h;
+      uint8_t* rec = cache + ((size_t)blk * n_kv_heads + h) * rec_bytes(head_dim);
       float sc;
       quantise_row(k, src, dtype, head_dim, codes, &sc);
-      memcpy(k8 + (bh * block_size + off) * head_dim, codes, (size_t)head_dim);
-      k_scale[bh * block_size + off] = sc;
+      for (int32_t e = 0; e < head_dim; ++e) rec[kpos(off, e, head_dim)] = (uint8_t)codes[e];
+      memcpy(rec + (size_t)32 * head_dim + 4 * off, &sc, 4);
       quantise_row(v, src, dtype, head_dim, codes, &sc);
-      for (int32_t e = 0; e < head_dim; ++e) v8[(bh * head_dim + e) * block_size + vpos((int)off)] = codes[e];
-      v_scale[bh * block_size + off] = sc;
+      for (int32_t e = 0; e < head_dim; ++e) rec[(size_t)16 * head_dim + (size_t)e * 16 + vpos(off)] = (uint8_t)codes[e];
+      memcpy(rec + (size_t)32 * head_dim + 64 + 4 * off, &sc, 4);
     }
   }
   free(codes);
@@ -369,10 +384,10 @@ int oracle_kv_append_int8(const void* k, const void* v, int32_t dtype, const int
 
 /* The same single-query attention as decode_row, over the dequantised INT8
  * cache (every value scale * code, exact in double). */
-static int decode_row_int8(const void* q, int dtype, const int8_t* k8, const int8_t* v8, const float* k_scale,
-                           const float* v_scale, const int32_t* block_tables, int32_t max_blocks_per_seq,
-                           const int32_t* context_lens, int32_t num_blocks, double scale, int32_t n_q,
-                           int32_t n_kv, int32_t d, int32_t bs, int32_t b, int32_t h, double* out_row) {
+static int decode_row_int8(const void* q, int dtype, const uint8_t* cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t num_blocks,
+                           double scale, int32_t n_q, int32_t n_kv, int32_t d, int32_t bs, int32_t b, int32_t h,
+                           double* out_row) {
   int32_t kvh = h / (n_q / n_kv);
   const int32_t ctx = *(context_lens + b);
   if (ctx < 0 || (int64_t)ctx > (int64_t)max_blocks_per_seq * bs) return ORC_ECTX;
@@ -392,12 +407,14 @@ static int decode_row_int8(const void* q, int dtype, const int8_t* k8, const int
       free(K); free(V); free(w); free(qv);
       return ORC_EBLOCK;
     }
-    size_t bh = (size_t)phys * n_kv + kvh;
-    int32_t off = j % bs;
-    double ks = (double)k_scale[bh * bs + off], vs = (double)v_scale[bh * bs + off];
+    const uint8_t* rec = cache + ((size_t)phys * n_kv + kvh) * rec_bytes(d);
+    int off = j % bs;
+    float ksf, vsf;
+    memcpy(&ksf, rec + (size_t)32 * d + 4 * off, 4);
+    memcpy(&vsf, rec + (size_t)32 * d + 64 + 4 * off, 4);
     for (int32_t e = 0; e < d; ++e) {
-      K[(size_t)j * d + e] = ks * (double)k8[(bh * bs + off) * d + e];
-      V[(size_t)j * d + e] = vs * (double)v8[(bh * d + e) * bs + vpos(off)];
+      K[(size_t)j * d + e] = (double)ksf * (double)(int8_t)rec[kpos(off, e, d)];
+      V[(size_t)j * d + e] = (double)vsf * (double)(int8_t)rec[(size_t)16 * d + (size_t)e * 16 + vpos(off)];
     }
   }
   for (int32_t e = 0; e < d; ++e) qv[e] = load_elem(q, (size_t)(b * n_q + h) * d + e, dtype);
@@ -421,14 +438,13 @@ static int decode_row_int8(const void* q, int dtype, const int8_t* k8, const int
   return ORC_OK;
 }
 
-int oracle_paged_decode_int8(const void* q, int32_t dtype, const int8_t* k8, const int8_t* v8,
-                             const float* k_scale, const float* v_scale, const int32_t* block_tables,
+int oracle_paged_decode_int8(const void* q, int32_t dtype, const uint8_t* cache, const int32_t* block_tables,
                              int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
                              int32_t num_blocks, double scale, int32_t n_q_heads, int32_t n_kv_heads,
                              int32_t head_dim, int32_t block_size, double* out, const int32_t* rows,
                              int32_t n_rows, int32_t n_threads) {
   if (!elem_bytes(dtype) || batch < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0 ||
-      head_dim <= 0 || block_size != 16 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+      (head_dim != 64 && head_dim != 128) || block_size != 16 || num_blocks <= 0 || max_blocks_per_seq <= 0)
     return ORC_EINVAL;
   int64_t total = rows ? (int64_t)n_rows : (int64_t)batch * n_q_heads;
   int status = ORC_OK;
@@ -445,8 +461,8 @@ int oracle_paged_decode_int8(const void* q, int32_t dtype, const int8_t* k8, con
     if (b < 0 || b >= batch || h < 0 || h >= n_q_heads) {
       rc = ORC_EINVAL;
     } else {
-      rc = decode_row_int8(q, dtype, k8, v8, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
-                           num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, b, h,
+      rc = decode_row_int8(q, dtype, cache, block_tables, max_blocks_per_seq, context_lens, num_blocks, scale,
+                           n_q_heads, n_kv_heads, head_dim, block_size, b, h,
                            out + ((size_t)b * n_q_heads + h) * head_dim);
     }
     if (rc != ORC_OK) {

@@ -102,9 +102,9 @@ def _load() -> ctypes.CDLL:
     lib.pkv_version.restype = ctypes.c_int32
     lib.paged_kv_copy_blocks.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p]
     lib.paged_kv_copy_blocks.restype = ctypes.c_int
-    lib.paged_kv_append_int8.argtypes = [p, p, ctypes.c_int, p, i32, p, p, p, p, i32, i32, i32, i32, p]
+    lib.paged_kv_append_int8.argtypes = [p, p, ctypes.c_int, p, i32, p, i32, i32, i32, i32, p]
     lib.paged_kv_append_int8.restype = ctypes.c_int
-    lib.paged_attention_decode_int8.argtypes = [p, p, p, p, p, p, i32, p, i32, i32, f32, i32, i32, i32, i32, p,
+    lib.paged_attention_decode_int8.argtypes = [p, p, p, i32, p, i32, i32, f32, i32, i32, i32, i32, p,
                                                 ctypes.c_int, p, sz, p]
     lib.paged_attention_decode_int8.restype = ctypes.c_int
     i64, u64 = ctypes.c_int64, ctypes.c_uint64
@@ -403,40 +403,33 @@ class BlockManager:
 
 
 def int8_cache(num_blocks: int, n_kv_heads: int, head_dim: int, device="cuda"):
-    """Empty INT8 cache tensors ``(k_cache, v_cache, k_scale, v_scale)``:
-    codes ``[num_blocks, n_kv, 16, d]`` and ``[num_blocks, n_kv, d, 16]``
-    (int8), per-token scales ``[num_blocks, n_kv, 16]`` (fp32)."""
-    k = torch.zeros((num_blocks, n_kv_heads, 16, head_dim), dtype=torch.int8, device=device)
-    v = torch.zeros((num_blocks, n_kv_heads, head_dim, 16), dtype=torch.int8, device=device)
-    ks = torch.zeros((num_blocks, n_kv_heads, 16), dtype=torch.float32, device=device)
-    vs = torch.zeros((num_blocks, n_kv_heads, 16), dtype=torch.float32, device=device)
-    return k, v, ks, vs
+    """An empty INT8 cache: uint8 ``[num_blocks, n_kv, 32 * head_dim + 128]``,
+    one record per (block, kv head) (layout in include/pagedkv.h)."""
+    return torch.zeros((num_blocks, n_kv_heads, 32 * head_dim + 128), dtype=torch.uint8, device=device)
 
 
-def paged_kv_append_int8(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale, stream=None) -> None:
+def paged_kv_append_int8(k, v, slot_mapping, kv_cache, block_size: int = 16, stream=None) -> None:
     """Quantise ``k[i]``, ``v[i]`` into slot ``slot_mapping[i]`` of the INT8 cache (in place)."""
     lib = _load()
-    num_blocks, n_kv, bs, d = k_cache.shape
-    if (k_cache.dtype != torch.int8 or v_cache.dtype != torch.int8 or tuple(v_cache.shape) != (num_blocks, n_kv, d, bs)
-            or tuple(k_scale.shape) != (num_blocks, n_kv, bs) or tuple(v_scale.shape) != (num_blocks, n_kv, bs)
-            or k_scale.dtype != torch.float32 or v_scale.dtype != torch.float32):
-        raise ValueError("INT8 cache tensors disagree")
+    num_blocks, n_kv, rb = kv_cache.shape
+    d = k.shape[-1]
+    if kv_cache.dtype != torch.uint8 or rb != 32 * d + 128 or k.shape[1] != n_kv:
+        raise ValueError("INT8 cache shape disagrees with k")
     if v.dtype != k.dtype or slot_mapping.dtype != torch.int64:
         raise ValueError("dtype mismatch (slot_mapping must be int64)")
     _check(lib.paged_kv_append_int8(_dev(k, "k"), _dev(v, "v"), _DTYPE[k.dtype], _dev(slot_mapping, "slot_mapping"),
-                                    k.shape[0], _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-                                    _dev(k_scale, "k_scale"), _dev(v_scale, "v_scale"), num_blocks, bs, n_kv, d,
+                                    k.shape[0], _dev(kv_cache, "kv_cache"), num_blocks, block_size, n_kv, d,
                                     _stream(stream)), "paged_kv_append_int8")
 
 
-def paged_attention_decode_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale: float,
-                                out=None, workspace=None, stream=None):
+def paged_attention_decode_int8(q, kv_cache, block_tables, context_lens, scale: float, out=None, workspace=None,
+                                block_size: int = 16, stream=None):
     """paged_attention_decode over the INT8 cache; returns ``out`` (dtype of q)."""
     lib = _load()
     B, n_q, d = q.shape
-    num_blocks, n_kv, bs, d2 = k_cache.shape
-    if d2 != d or tuple(v_cache.shape) != (num_blocks, n_kv, d, bs):
-        raise ValueError("shape mismatch")
+    num_blocks, n_kv, rb = kv_cache.shape
+    if rb != 32 * d + 128 or kv_cache.dtype != torch.uint8:
+        raise ValueError("INT8 cache shape disagrees with q")
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise ValueError("block_tables and context_lens must be int32")
     if out is None:
@@ -445,8 +438,7 @@ def paged_attention_decode_int8(q, k_cache, v_cache, k_scale, v_scale, block_tab
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
     _check(lib.paged_attention_decode_int8(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(k_scale, "k_scale"),
-        _dev(v_scale, "v_scale"), _dev(block_tables, "block_tables"), block_tables.shape[1],
-        _dev(context_lens, "context_lens"), B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"),
+        _dev(q, "q"), _dev(kv_cache, "kv_cache"), _dev(block_tables, "block_tables"), block_tables.shape[1],
+        _dev(context_lens, "context_lens"), B, num_blocks, float(scale), n_q, n_kv, d, block_size, _dev(out, "out"),
         _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream)), "paged_attention_decode_int8")
     return out

@@ -199,25 +199,9 @@ pkv_status dispatch_i8(int gpad, const CUtensorMap& mk, const DecodeParams& p, i
                    : launch_decode<DT, 128, 16, true>(mk, mk, p, grid, smem, stream);
 }
 
-// TMA view of the INT8 K codes: [block][kv head][token][dim] bytes, one
-// 128-byte x 16-row box per tile, 128B swizzle.
-pkv_status encode_i8_key_map(CUtensorMap* map, const void* k8, int num_blocks, int n_kv, int head_dim) {
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(kBlockTokens),
-                              static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(num_blocks)};
-  const cuuint64_t row = static_cast<cuuint64_t>(head_dim);
-  const cuuint64_t strides[3] = {row, row * kBlockTokens, row * kBlockTokens * n_kv};
-  const cuuint32_t box[4] = {128, static_cast<cuuint32_t>(kBlockTokens), 1, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(k8), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
-}
-
-// Scale rows and transposed V codes of the INT8 cache (null for 16-bit caches).
+// The INT8 cache (one record per (block, kv head); null for 16-bit caches).
 struct KvI8 {
-  const float* k_scale;
-  const float* v_scale;
+  const uint8_t* records;
 };
 
 // Shared-memory ring of the prefix kernel: three stages of 64 tokens of K and V.
@@ -329,18 +313,15 @@ pkv_status paged_kv_copy_blocks(void* k_cache, void* v_cache, const int32_t* src
 }
 
 pkv_status paged_kv_append_int8(const void* k, const void* v, pkv_dtype dtype, const int64_t* slot_mapping,
-                                int32_t num_tokens, int8_t* k_cache, int8_t* v_cache, float* k_scale, float* v_scale,
-                                int32_t num_blocks, int32_t block_size, int32_t n_kv_heads, int32_t head_dim,
-                                void* stream) {
+                                int32_t num_tokens, uint8_t* kv_cache, int32_t num_blocks, int32_t block_size,
+                                int32_t n_kv_heads, int32_t head_dim, void* stream) {
   if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || n_kv_heads <= 0 || head_dim <= 0)
     return PKV_ERR_INVALID_ARG;
   if (elem_bytes(dtype) == 0 || block_size != kBlockTokens || (head_dim != 64 && head_dim != 128))
     return PKV_ERR_UNSUPPORTED;
   if (num_tokens == 0) return PKV_OK;
-  if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale ||
-      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u) || (reinterpret_cast<uintptr_t>(k) & 3u) ||
-      (reinterpret_cast<uintptr_t>(v) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
-      (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+  if (!k || !v || !slot_mapping || !kv_cache || !aligned16(kv_cache) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7u) ||
+      (reinterpret_cast<uintptr_t>(k) & 3u) || (reinterpret_cast<uintptr_t>(v) & 3u))
     return PKV_ERR_INVALID_ARG;
   DeviceInfo di;
   if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
@@ -348,10 +329,7 @@ pkv_status paged_kv_append_int8(const void* k, const void* v, pkv_dtype dtype, c
   p.k = k;
   p.v = v;
   p.slot_mapping = slot_mapping;
-  p.k8 = k_cache;
-  p.v8 = v_cache;
-  p.k_scale = k_scale;
-  p.v_scale = v_scale;
+  p.cache = kv_cache;
   p.num_slots = static_cast<int64_t>(num_blocks) * block_size;
   p.num_tokens = num_tokens;
   p.n_kv_heads = n_kv_heads;
@@ -411,11 +389,7 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                     num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
   if (st != PKV_OK) return st;
-  if (i8) {
-    if (dtype == PKV_F32 || head_dim != 128) return PKV_ERR_UNSUPPORTED;
-    if (!i8->k_scale || !i8->v_scale || !aligned16(i8->k_scale) || !aligned16(i8->v_scale))
-      return PKV_ERR_INVALID_ARG;
-  }
+  if (i8 && (dtype == PKV_F32 || head_dim != 128)) return PKV_ERR_UNSUPPORTED;
   if (batch == 0) return st;
   pkv_decode_options opt = {};
   if (options) {
@@ -447,8 +421,8 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   // Ring depth: as many slots per consumer warp as shared memory allows
   // (at most 4; 2 with ten consumer warps and 8 KiB tiles).
   const int es = elem_bytes(dtype);
-  // INT8: K codes (16 x head_dim bytes) plus transposed V codes and 2 x 16 scales.
-  const size_t stage_bytes = i8 ? static_cast<size_t>(2) * head_dim * kBlockTokens + 2 * kBlockTokens * 4
+  // INT8: one record (K and transposed V codes, 2 x 16 scales).
+  const size_t stage_bytes = i8 ? static_cast<size_t>(i8_record_bytes(head_dim))
                                 : static_cast<size_t>(2) * (head_dim * es / 128) * kBoxBytes;
   // 1 KiB alignment slack, abort word, prefix sums and clamped lengths, and
   // 256 bytes for the kernel's static shared memory.
@@ -475,18 +449,14 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
     return PKV_ERR_WORKSPACE;
   }
 
-  CUtensorMap mk, mv;
-  if (i8) {
-    st = encode_i8_key_map(&mk, k_cache, num_blocks, n_kv_heads, head_dim);
-  } else {
+  CUtensorMap mk = {}, mv = {};
+  if (!i8) {
     st = encode_cache_map(&mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
     if (st == PKV_OK) st = encode_cache_map(&mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
   }
 
   DecodeParams p;
-  p.v_i8 = i8 ? static_cast<const int8_t*>(v_cache) : nullptr;
-  p.k_scale = i8 ? i8->k_scale : nullptr;
-  p.v_scale = i8 ? i8->v_scale : nullptr;
+  p.kv_i8 = i8 ? i8->records : nullptr;
   p.n_kv_heads = n_kv_heads;
   p.q = q;
   p.out = out;
@@ -553,14 +523,13 @@ pkv_status paged_attention_decode(const void* q, const void* k_cache, const void
                                    workspace, workspace_bytes, stream, nullptr);
 }
 
-pkv_status paged_attention_decode_int8(const void* q, const int8_t* k_cache, const int8_t* v_cache,
-                                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
+pkv_status paged_attention_decode_int8(const void* q, const uint8_t* kv_cache, const int32_t* block_tables,
                                        int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
                                        int32_t num_blocks, float scale, int32_t n_q_heads, int32_t n_kv_heads,
                                        int32_t head_dim, int32_t block_size, void* out, pkv_dtype dtype,
                                        void* workspace, size_t workspace_bytes, void* stream) {
-  const KvI8 i8 = {k_scale, v_scale};
-  return decode_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
+  const KvI8 i8 = {kv_cache};
+  return decode_impl(q, kv_cache, kv_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
                      n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, workspace, workspace_bytes, stream,
                      nullptr, nullptr, nullptr, 0, &i8);
 }

@@ -170,6 +170,17 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
   }
 }
 
+// D += A B on the integer tensor-core path: A 16 x 32 and B 32 x 8 signed
+// 8-bit (four per register), D 16 x 8 int32.
+__device__ __forceinline__ void mma_16832_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Pack two fp32 into a 16-bit pair (lo in bits 0..15), round to nearest even.
 template <bool kBf16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {

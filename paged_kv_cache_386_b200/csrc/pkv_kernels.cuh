@@ -167,14 +167,17 @@ __global__ void __launch_bounds__(256) pkv_copy_blocks_kernel(const CopyParams p
 // bytes 4t .. 4t + 3.
 __host__ __device__ __forceinline__ int vpos_i8(int j) { return 4 * ((j & 7) >> 1) + 2 * (j >> 3) + (j & 1); }
 
+// One record per (block, kv head) of the INT8 cache, head dim D: K codes
+// (16 rows of D bytes, 16-byte chunk c of row j stored at chunk c ^ (j %
+// min(8, D / 16))), transposed V codes (D rows of 16 bytes, token order
+// vpos_i8), 16 fp32 K scales, 16 fp32 V scales.
+__host__ __device__ constexpr int i8_record_bytes(int D) { return 32 * D + 128; }
+
 struct AppendI8Params {
   const void* k;
   const void* v;
   const int64_t* slot_mapping;
-  int8_t* k8;       // [num_blocks][n_kv][16][D]
-  int8_t* v8;       // [num_blocks][n_kv][D][16], token order vpos_i8
-  float* k_scale;   // [num_blocks][n_kv][16]
-  float* v_scale;
+  uint8_t* cache;  // [num_blocks][n_kv][i8_record_bytes(D)]
   int64_t num_slots;
   int32_t num_tokens;
   int32_t n_kv_heads;
@@ -219,7 +222,7 @@ __global__ void __launch_bounds__(256) pkv_append_i8_kernel(const AppendI8Params
     }
     const int64_t blk = s / kBlockTokens;
     const int off = static_cast<int>(s % kBlockTokens);
-    const size_t bh = static_cast<size_t>(blk) * p.n_kv_heads + h;
+    uint8_t* rec = p.cache + (static_cast<size_t>(blk) * p.n_kv_heads + h) * i8_record_bytes(D);
     const size_t src = static_cast<size_t>(r) * D + lane * EPL;
     float xk[EPL], xv[EPL];
 #pragma unroll
@@ -239,15 +242,18 @@ __global__ void __launch_bounds__(256) pkv_append_i8_kernel(const AppendI8Params
     int8_t ck[EPL], cv[EPL];
     const float sk = quantise_row<EPL>(xk, ck);
     const float sv = quantise_row<EPL>(xv, cv);
-    int8_t* krow = p.k8 + (bh * kBlockTokens + off) * D + lane * EPL;
+    // This lane's EPL dims sit inside one 16-byte chunk of the K row.
+    constexpr int kSwz = (D / 16) < 8 ? (D / 16) : 8;
+    const int c = (lane * EPL) / 16;
+    uint8_t* krow = rec + off * D + ((c ^ (off % kSwz)) * 16) + (lane * EPL) % 16;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) krow[e] = ck[e];
+    for (int e = 0; e < EPL; ++e) krow[e] = static_cast<uint8_t>(ck[e]);
     const int vp = vpos_i8(off);
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) p.v8[(bh * D + lane * EPL + e) * kBlockTokens + vp] = cv[e];
+    for (int e = 0; e < EPL; ++e) rec[16 * D + (lane * EPL + e) * kBlockTokens + vp] = static_cast<uint8_t>(cv[e]);
     if (lane == 0) {
-      p.k_scale[bh * kBlockTokens + off] = sk;
-      p.v_scale[bh * kBlockTokens + off] = sv;
+      reinterpret_cast<float*>(rec + 32 * D)[off] = sk;
+      reinterpret_cast<float*>(rec + 32 * D + 64)[off] = sv;
     }
   }
 }
@@ -261,10 +267,7 @@ struct DecodeParams {
   const int32_t* block_tables;
   const int32_t* context_lens;
   float* records;  // [chunks][2][rec_floats]: O[gp][D], m[gp], l[gp]
-  // INT8 cache only: transposed V codes and the per-token scales.
-  const int8_t* v_i8;
-  const float* k_scale;
-  const float* v_scale;
+  const uint8_t* kv_i8;  // INT8 cache only: one record per (block, kv head)
   int32_t n_kv_heads;
   int4* meta;      // [chunks]: split segment whose first piece the chunk holds
   int* sched;      // [0]: claim counter of the balancing chunks (0 between launches)
@@ -834,56 +837,96 @@ struct SimtConsumer {
 // K tile: 16 rows of 128 one-byte codes, TMA 128B swizzle (16-byte chunk c of
 // row r at chunk c ^ (r % 8)).  V tile: 128 rows (dims) of 16 bytes (tokens,
 // in vpos_i8 order).  Then 16 fp32 K scales and 16 V scales (token order).
+//
+// S = Q K^T runs on the integer tensor-core path (mma m16n8k32 s8): each Q
+// row is put on a 14-bit grid once per segment, q ~ sq * (128 hi + lo) with
+// sq = max|q| / 8191 and hi, lo signed 8-bit, so that S = sq * sk * (128
+// (hi . k) + (lo . k)) with exact int32 dot products over the K codes (the
+// grid's rounding, at most sq / 2 per element, is the only approximation).
 // The dot product over the head dim does not depend on the order of the
-// dims, so lane t owns dims [32t, 32t + 32) for every k-step: k-step ks
-// takes dims 32t + 4ks + {0, 1} as the fragment's columns 2t, 2t + 1 and
-// 32t + 4ks + {2, 3} as columns 2t + 8, 2t + 9, for Q and K alike.  A lane's
-// K codes of one row are then two 16-byte loads that the swizzle keeps free of
-// bank conflicts.  Codes become exact 16-bit values (i8x2_to_16x2); the K
-// scale multiplies the score columns, the V scale the probabilities.
+// dims, so lane t owns dims [32t, 32t + 32): k-step kk takes dims 32t + 8kk
+// + [0, 4) as the fragment's columns 4t.. and 32t + 8kk + [4, 8) as columns
+// 16 + 4t.., for Q and K alike; a lane's K codes of one row are two 16-byte
+// loads that the swizzle keeps free of bank conflicts.
+//
+// O += P V runs in f16 with V codes turned into exact f16 values.  The V
+// scale of token t enters through the probabilities, p * vs_t / c, where c
+// is the largest V scale seen so far by the warp: the factors stay in [0, 1]
+// (f16 range), O is rescaled when c grows, and O * c is the true sum.
 template <int DT, int GPAD>
 struct MmaConsumerI8 : MmaConsumer<DT, 128, GPAD> {
   using Base = MmaConsumer<DT, 128, GPAD>;
   using T = typename Base::T;
   static constexpr bool kBf16 = Base::kBf16;
   static constexpr int D = 128;
-  static constexpr int KS = D / 16;
   static constexpr int NT = D / 8;
   using Base::l;
   using Base::m;
   using Base::o;
-  using Base::qa;
+  using Base::qa;  // qa[kk] = hi, qa[4 + kk] = lo, k-steps kk = 0..3
+  float qs[2];     // grid step of rows g and g + 8
+  float cv;        // largest V scale seen (0 before the first tile)
+  float inv_cv;    // 1 / cv (0 while cv is 0)
+
+  // Q row `row` (this lane's 32 dims) on the 14-bit grid.
+  __device__ __forceinline__ void split_row(const T* qr, bool live, int t, int slot) {
+    float x[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t w = live ? *reinterpret_cast<const uint32_t*>(qr + 32 * t + 2 * i) : 0u;
+      unpack2<kBf16>(w, x[2 * i], x[2 * i + 1]);
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(x[i]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float inv = mx > 0.f ? 8191.f / mx : 0.f;
+    qs[slot] = mx / 8191.f;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t h[2] = {0u, 0u}, lo[2] = {0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int qi = __float2int_rn(x[8 * kk + j] * inv);  // |qi| <= 8191
+        const int hi = (qi + 64) >> 7;                        // [-64, 64]
+        const int lw = qi - (hi << 7);                        // [-64, 63]
+        h[j >> 2] |= (static_cast<uint32_t>(hi) & 0xffu) << (8 * (j & 3));
+        lo[j >> 2] |= (static_cast<uint32_t>(lw) & 0xffu) << (8 * (j & 3));
+      }
+      // a0 / a2 carry row g (columns 4t.. and 16 + 4t..); a1 / a3 row g + 8.
+      qa[kk][slot] = h[0];
+      qa[kk][2 + slot] = h[1];
+      qa[4 + kk][slot] = lo[0];
+      qa[4 + kk][2 + slot] = lo[1];
+    }
+  }
 
   __device__ __forceinline__ void begin(const uint8_t* qbuf, int gp, int lane) {
     const int g = lane >> 2, t = lane & 3;
     const T* qb = reinterpret_cast<const T*>(qbuf);
-    const bool r0 = g < gp;
-    const bool r1 = (GPAD == 16) && (g + 8 < gp);
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int c = 32 * t + 4 * ks;
-      const uint2 x0 = r0 ? *reinterpret_cast<const uint2*>(qb + g * D + c) : make_uint2(0u, 0u);
-      const uint2 x1 = r1 ? *reinterpret_cast<const uint2*>(qb + (g + 8) * D + c) : make_uint2(0u, 0u);
-      qa[ks][0] = x0.x;
-      qa[ks][2] = x0.y;
-      qa[ks][1] = x1.x;
-      qa[ks][3] = x1.y;
+    split_row(qb + g * D, g < gp, t, 0);
+    if constexpr (GPAD == 16) {
+      split_row(qb + (g + 8) * D, g + 8 < gp, t, 1);
+    } else {
+      qs[1] = 0.f;
     }
 #pragma unroll
     for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     m[0] = m[1] = -INFINITY;
     l[0] = l[1] = 0.f;
+    cv = 0.f;
+    inv_cv = 0.f;
   }
 
   __device__ __forceinline__ void tile(uint32_t kbase, uint32_t vbase, int nv, float scale_log2, int lane) {
     const int g = lane >> 2, t = lane & 3;
     const uint32_t sbase = vbase + D * kBlockTokens;  // K scales, then V scales
 
-    // S = Q K^T for tokens g (n-tile 0) and g + 8 (n-tile 1).
+    // Integer S for tokens g (n-tile 0) and g + 8 (n-tile 1).
     float s[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
       const int row = nt * 8 + g;
       uint4 c0, c1;
       asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -893,23 +936,31 @@ struct MmaConsumerI8 : MmaConsumer<DT, 128, GPAD> {
                    : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
                    : "r"(kbase + row * 128 + (((2 * t + 1) ^ (row & 7)) << 4)));
       const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks)
-        mma_16816<kBf16>(s[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], i8x2_to_16x2<kBf16>(w[ks], 0),
-                         i8x2_to_16x2<kBf16>(w[ks], 1));
+      for (int kk = 0; kk < 4; ++kk) {
+        // With at most 8 rows, rows 8..15 of A are zero (literal zeros: no registers held).
+        const uint32_t h1 = GPAD == 16 ? qa[kk][1] : 0u, h3 = GPAD == 16 ? qa[kk][3] : 0u;
+        const uint32_t l1 = GPAD == 16 ? qa[4 + kk][1] : 0u, l3 = GPAD == 16 ? qa[4 + kk][3] : 0u;
+        mma_16832_s8(ah, qa[kk][0], h1, qa[kk][2], h3, w[2 * kk], w[2 * kk + 1]);
+        mma_16832_s8(al, qa[4 + kk][0], l1, qa[4 + kk][2], l3, w[2 * kk], w[2 * kk + 1]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nt][e] = static_cast<float>(ah[e] * 128 + al[e]);
     }
-    // K scales of this lane's score columns: tokens 2t, 2t + 1 and 2t + 8, 2t + 9.
+    // Scales: the row's grid step and the K scale of this lane's columns
+    // (tokens 2t, 2t + 1 and 2t + 8, 2t + 9).
     float2 ks0, ks1;
     asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(ks0.x), "=f"(ks0.y) : "r"(sbase + 8 * t));
     asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(ks1.x), "=f"(ks1.y) : "r"(sbase + 32 + 8 * t));
-    s[0][0] *= ks0.x;
-    s[0][1] *= ks0.y;
-    s[0][2] *= ks0.x;
-    s[0][3] *= ks0.y;
-    s[1][0] *= ks1.x;
-    s[1][1] *= ks1.y;
-    s[1][2] *= ks1.x;
-    s[1][3] *= ks1.y;
+    s[0][0] *= qs[0] * ks0.x;
+    s[0][1] *= qs[0] * ks0.y;
+    s[0][2] *= qs[1] * ks0.x;
+    s[0][3] *= qs[1] * ks0.y;
+    s[1][0] *= qs[0] * ks1.x;
+    s[1][1] *= qs[0] * ks1.y;
+    s[1][2] *= qs[1] * ks1.x;
+    s[1][3] *= qs[1] * ks1.y;
 
     // Online softmax (as in the 16-bit consumer).
     constexpr int kRows = (GPAD == 16) ? 2 : 1;
@@ -946,9 +997,35 @@ struct MmaConsumerI8 : MmaConsumer<DT, 128, GPAD> {
       l[r] = l[r] * alpha[r] + sum;
       m[r] = mn;
     }
-    if (__any_sync(0xffffffffu, grow)) {
-      const float a_lo = alpha[0];
-      const float a_hi = (GPAD == 16) ? alpha[1] : alpha[0];
+
+    // V scales of this lane's tokens; the largest over the tile's live tokens
+    // (scales past the context may be anything, NaN included).
+    float2 vs0, vs1;
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(vs0.x), "=f"(vs0.y) : "r"(sbase + 64 + 8 * t));
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(vs1.x), "=f"(vs1.y) : "r"(sbase + 96 + 8 * t));
+    float vsc[2][2] = {{vs0.x, vs0.y}, {vs1.x, vs1.y}};
+    float vmax = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool live = nt * 8 + 2 * t + e < nv;
+        vsc[nt][e] = live ? vsc[nt][e] : 0.f;
+        vmax = fmaxf(vmax, vsc[nt][e]);
+      }
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 1));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
+    const float cn = fmaxf(cv, vmax);
+    const bool cgrow = cn > cv;  // warp-uniform (cv, vmax are)
+    float rc = 1.f;
+    if (cgrow) {
+      rc = cv / cn;  // 0 on the first tile (O is 0 then)
+      inv_cv = 1.f / cn;
+      cv = cn;
+    }
+    if (__any_sync(0xffffffffu, grow || cgrow)) {
+      const float a_lo = alpha[0] * rc;
+      const float a_hi = ((GPAD == 16) ? alpha[1] : alpha[0]) * rc;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         o[n][0] *= a_lo;
@@ -957,43 +1034,52 @@ struct MmaConsumerI8 : MmaConsumer<DT, 128, GPAD> {
         o[n][3] *= a_hi;
       }
     }
-
-    // V scales folded into the probabilities; tokens past the context (whose
-    // scales may be anything, NaN included) get 0.
-    float2 vs0, vs1;
-    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(vs0.x), "=f"(vs0.y) : "r"(sbase + 64 + 8 * t));
-    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(vs1.x), "=f"(vs1.y) : "r"(sbase + 96 + 8 * t));
-    const float vsc[2][2] = {{vs0.x, vs0.y}, {vs1.x, vs1.y}};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) vsc[nt][e] *= inv_cv;
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) pr[r][nt][e] = (nt * 8 + 2 * t + e < nv) ? pr[r][nt][e] * vsc[nt][e] : 0.f;
+        for (int e = 0; e < 2; ++e) pr[r][nt][e] *= vsc[nt][e];
 
-    uint32_t pa0 = pack2<kBf16>(pr[0][0][0], pr[0][0][1]);
-    uint32_t pa2 = pack2<kBf16>(pr[0][1][0], pr[0][1][1]);
+    uint32_t pa0 = pack2<false>(pr[0][0][0], pr[0][0][1]);
+    uint32_t pa2 = pack2<false>(pr[0][1][0], pr[0][1][1]);
     uint32_t pa1, pa3;
     if constexpr (GPAD == 16) {
-      pa1 = pack2<kBf16>(pr[1][0][0], pr[1][0][1]);
-      pa3 = pack2<kBf16>(pr[1][1][0], pr[1][1][1]);
+      pa1 = pack2<false>(pr[1][0][0], pr[1][0][1]);
+      pa3 = pack2<false>(pr[1][1][0], pr[1][1][1]);
     } else {
       float h00, h01, h10, h11;
-      unpack2<kBf16>(pa0, h00, h01);
-      unpack2<kBf16>(pa2, h10, h11);
-      pa1 = pack2<kBf16>(pr[0][0][0] - h00, pr[0][0][1] - h01);
-      pa3 = pack2<kBf16>(pr[0][1][0] - h10, pr[0][1][1] - h11);
+      unpack2<false>(pa0, h00, h01);
+      unpack2<false>(pa2, h10, h11);
+      pa1 = pack2<false>(pr[0][0][0] - h00, pr[0][0][1] - h01);
+      pa3 = pack2<false>(pr[0][1][0] - h10, pr[0][1][1] - h11);
     }
 
-    // O += P V: V^T row 8n + g holds dim 8n + g of all 16 tokens; bytes 4t ..
-    // 4t + 3 are tokens 2t, 2t + 1, 2t + 8, 2t + 9 (codes are finite, so the
-    // rows past the context need no mask: their probabilities are 0).
+    // O += P V in f16: V^T row 8n + g holds dim 8n + g of all 16 tokens; bytes
+    // 4t .. 4t + 3 are tokens 2t, 2t + 1, 2t + 8, 2t + 9 (codes are finite, so
+    // the rows past the context need no mask: their factors are 0).
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       uint32_t w;
       asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(vbase + (8 * n + g) * kBlockTokens + 4 * t));
-      mma_16816<kBf16>(o[n], pa0, pa1, pa2, pa3, i8x2_to_16x2<kBf16>(w, 0), i8x2_to_16x2<kBf16>(w, 1));
+      mma_16816<false>(o[n], pa0, pa1, pa2, pa3, i8x2_to_16x2<false>(w, 0), i8x2_to_16x2<false>(w, 1));
     }
+  }
+
+  // O in true units (times c) before the 16-bit consumer's epilogue.
+  __device__ __forceinline__ void finish(const DecodeParams& p, int b, int hg, float* rec, int lane) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      o[n][0] *= cv;
+      o[n][1] *= cv;
+      o[n][2] *= cv;
+      o[n][3] *= cv;
+    }
+    Base::finish(p, b, hg, rec, lane);
   }
 };
 
@@ -1173,11 +1259,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   constexpr int X = 128 / ES;                      // elements per swizzle row
   constexpr int Y = D / X;                         // boxes per tile
   constexpr int kTileBytes = Y * kBoxBytes;
-  // Ring slots: the K region (1 KiB aligned for the swizzle) and, for INT8,
-  // a second region with the transposed V codes and the two scale rows.
-  constexpr int kRingStride = kI8 ? D * kBlockTokens : 2 * kTileBytes;
-  constexpr int kVStride = kI8 ? D * kBlockTokens + 2 * kBlockTokens * 4 : 0;
-  constexpr int kStageBytes = kI8 ? kRingStride + kVStride : 2 * kTileBytes;  // bytes landing per slot
+  // Ring slots (1 KiB aligned for the swizzle; INT8 records on 128-byte
+  // multiples, which keeps their pre-swizzled K rows conflict-free).
+  constexpr int kRingStride = kI8 ? i8_record_bytes(D) : 2 * kTileBytes;
+  constexpr int kStageBytes = kRingStride;  // bytes landing per slot
   constexpr int kQBufBytes = (GPAD == 0 ? 1 : GPAD) * D * ES;
   using Consumer = typename ConsumerFor<DT, D, GPAD, kI8>::type;
   using OutT = typename DTypeInfo<DT>::T;
@@ -1187,8 +1272,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ring = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const int n_slots = kConsumerWarps * p.stages;
-  uint8_t* vring = ring + static_cast<size_t>(n_slots) * kRingStride;                 // INT8: [slots][kVStride]
-  uint8_t* qbufs = vring + static_cast<size_t>(n_slots) * kVStride;  // [warps][kQBufBytes]
+  uint8_t* qbufs = ring + static_cast<size_t>(n_slots) * kRingStride;  // [warps][kQBufBytes]
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(qbufs + kConsumerWarps * kQBufBytes);
   uint64_t* empty_bar = full_bar + n_slots;
   int4* slot_info = reinterpret_cast<int4*>(empty_bar + n_slots);  // [n_slots]: next chunk, from the producer
@@ -1214,7 +1298,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if ((reinterpret_cast<uintptr_t>(p.block_tables) & 15u) == 0)
       prefetch_slice_l2(p.block_tables, static_cast<size_t>(B) * p.max_blocks_per_seq * sizeof(int32_t) & ~size_t(15));
   }
-  if (warp == kConsumerWarps && lane == 0) {
+  if (!kI8 && warp == kConsumerWarps && lane == 0) {  // the INT8 cache uses no tensor map
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
@@ -1329,13 +1413,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
           uint8_t* sk = ring + static_cast<size_t>(slot) * kRingStride;
           if constexpr (kI8) {
+            // The whole record in one contiguous request.
             const size_t bh = static_cast<size_t>(ph) * p.n_kv_heads + t0.kvh;
-            uint8_t* sv = vring + static_cast<size_t>(slot) * kVStride;
-            tma_load_4d(sk, &tm_k, &full_bar[slot], 0, 0, t0.kvh, ph);
-            bulk_load(sv, p.v_i8 + bh * D * kBlockTokens, D * kBlockTokens, &full_bar[slot]);
-            bulk_load(sv + D * kBlockTokens, p.k_scale + bh * kBlockTokens, kBlockTokens * 4, &full_bar[slot]);
-            bulk_load(sv + D * kBlockTokens + kBlockTokens * 4, p.v_scale + bh * kBlockTokens, kBlockTokens * 4,
-                      &full_bar[slot]);
+            bulk_load(sk, p.kv_i8 + bh * kRingStride, kRingStride, &full_bar[slot]);
           } else {
 #pragma unroll
             for (int y = 0; y < Y; ++y)
@@ -1468,7 +1548,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
         const int nv = min(kBlockTokens, wk.ctx - wk.j * kBlockTokens);
         const uint32_t kaddr = smem_u32(ring + static_cast<size_t>(slot) * kRingStride);
-        const uint32_t vaddr = kI8 ? smem_u32(vring + static_cast<size_t>(slot) * kVStride) : kaddr + kTileBytes;
+        const uint32_t vaddr = kI8 ? kaddr + D * kBlockTokens : kaddr + kTileBytes;
         cs.tile(kaddr, vaddr, nv, p.scale_log2, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[slot]);

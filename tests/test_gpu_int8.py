@@ -17,19 +17,18 @@ def _gpu_cache(w):
     """Fill an INT8 cache on the GPU with every cached token of `w` and its
     appended token, through the GPU append."""
     dev = torch.device("cuda")
-    k8, v8, ks, vs = (t.to(dev) for t in W.int8_cache_buffers(w))
+    cache = W.int8_cache_buffers(w).to(dev)
     kr, vr, slots = W.cached_token_rows(w)
-    pkv.paged_kv_append_int8(kr.to(dev), vr.to(dev), slots.to(dev), k8, v8, ks, vs)
+    pkv.paged_kv_append_int8(kr.to(dev), vr.to(dev), slots.to(dev), cache)
     if w.appended:
-        pkv.paged_kv_append_int8(w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev), k8, v8, ks, vs)
-    return k8, v8, ks, vs
+        pkv.paged_kv_append_int8(w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev), cache)
+    return cache
 
 
 def _decode(w, cache):
     dev = torch.device("cuda")
-    k8, v8, ks, vs = cache
-    out = pkv.paged_attention_decode_int8(w.q.to(dev), k8, v8, ks, vs, w.block_tables.to(dev),
-                                          w.context_lens.to(dev), w.scale)
+    out = pkv.paged_attention_decode_int8(w.q.to(dev), cache, w.block_tables.to(dev), w.context_lens.to(dev),
+                                          w.scale)
     torch.cuda.synchronize()
     assert pkv.pkv_get_device_error() == 0
     return out.cpu()
@@ -37,10 +36,8 @@ def _decode(w, cache):
 
 def _check(w, rows=None):
     cache = _gpu_cache(w)
-    ref, ok8, ov8, oks, ovs = oracle.workload_decode_int8(w, rows=rows)
-    k8, v8, ks, vs = (t.cpu() for t in cache)
-    assert torch.equal(k8, ok8) and torch.equal(v8, ov8), "INT8 codes differ from the oracle"
-    assert torch.equal(bits(ks), bits(oks)) and torch.equal(bits(vs), bits(ovs)), "INT8 scales differ"
+    ref, ocache = oracle.workload_decode_int8(w, rows=rows)
+    assert torch.equal(cache.cpu(), ocache), "INT8 records (codes and scale bits) differ from the oracle"
     out = _decode(w, cache)
     return assert_close(out, ref, w.dtype, rows=rows, what=w.name)
 
@@ -82,19 +79,14 @@ def test_int8_append_bit_exact(src, d):
     k[3] = 0                                                    # all-zero rows: scale 0, codes 0
     slots = torch.randperm(nb * 16, generator=g)[:n].to(torch.int64)
     slots[5] = -1                                               # padding token: skipped
-    ok8 = torch.zeros((nb, n_kv, 16, d), dtype=torch.int8)
-    ov8 = torch.zeros((nb, n_kv, d, 16), dtype=torch.int8)
-    oks = torch.full((nb, n_kv, 16), float("nan"))
-    ovs = torch.full((nb, n_kv, 16), float("nan"))
-    oracle.kv_append_int8(k, v, slots, ok8, ov8, oks, ovs)
-    dev = torch.device("cuda")
-    k8, v8, ks, vs = ok8.new_zeros(ok8.shape).to(dev), ov8.new_zeros(ov8.shape).to(dev), \
-        torch.full_like(oks, float("nan")).to(dev), torch.full_like(ovs, float("nan")).to(dev)
-    pkv.paged_kv_append_int8(k.to(dev), v.to(dev), slots.to(dev), k8, v8, ks, vs)
+    ocache = torch.zeros((nb, n_kv, 32 * d + 128), dtype=torch.uint8)
+    ocache[:, :, 32 * d:].view(torch.float32).fill_(float("nan"))
+    cache = ocache.clone().cuda()
+    oracle.kv_append_int8(k, v, slots, ocache)
+    pkv.paged_kv_append_int8(k.cuda(), v.cuda(), slots.cuda(), cache)
     torch.cuda.synchronize()
     assert pkv.pkv_get_device_error() == 0
-    assert torch.equal(k8.cpu(), ok8) and torch.equal(v8.cpu(), ov8)
-    assert torch.equal(bits(ks.cpu()), bits(oks)) and torch.equal(bits(vs.cpu()), bits(ovs))
+    assert torch.equal(cache.cpu(), ocache)
 
 
 def test_int8_placement_bit_exact_and_deterministic():
@@ -105,9 +97,8 @@ def test_int8_placement_bit_exact_and_deterministic():
     # The same tokens with every physical block moved elsewhere.
     perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(5))
     dev = torch.device("cuda")
-    moved = [torch.empty_like(t) for t in cache]
-    for src, dst in zip(cache, moved):
-        dst[perm.to(dev)] = src
+    moved = torch.empty_like(cache)
+    moved[perm.to(dev)] = cache
     m = W.uniform_gqa(batch=8, len_lo=30, len_hi=1200, seed=63)
     m.block_tables = torch.where(w.block_tables >= 0, perm[w.block_tables.clamp(min=0).long()].int(), w.block_tables)
     b = _decode(m, moved)
@@ -120,11 +111,10 @@ def test_int8_empty_and_unsupported():
     cache = _gpu_cache(w)
     out = _decode(w, cache)
     assert torch.equal(out[0], torch.zeros_like(out[0]))
-    ref, *_ = oracle.workload_decode_int8(w)
+    ref, _ = oracle.workload_decode_int8(w)
     assert_close(out, ref, w.dtype, what="i8 empty")
     dev = torch.device("cuda")
-    k8, v8, ks, vs = cache
     with pytest.raises(pkv.PagedKVError) as e:   # fp32 queries are not supported on the INT8 cache
-        pkv.paged_attention_decode_int8(w.q.float().to(dev), k8, v8, ks, vs, w.block_tables.to(dev),
+        pkv.paged_attention_decode_int8(w.q.float().to(dev), cache, w.block_tables.to(dev),
                                         w.context_lens.to(dev), w.scale)
     assert e.value.status == 2

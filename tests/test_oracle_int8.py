@@ -23,12 +23,12 @@ MUTANTS = [
     ("round_half_away", "rintf(x / scale)", "roundf(x / scale)"),
     ("vpos_swapped_halves", "return 4 * ((j % 8) / 2) + 2 * (j / 8) + (j % 2);",
      "return 2 * ((j % 8) / 2) + 8 * (j / 8) + (j % 2);"),
-    ("v_not_transposed_on_read", "V[(size_t)j * d + e] = vs * (double)v8[(bh * d + e) * bs + vpos(off)];",
-     "V[(size_t)j * d + e] = vs * (double)v8[(bh * bs + off) * d + e];"),
-    ("k_scale_for_v", "double ks = (double)k_scale[bh * bs + off], vs = (double)v_scale[bh * bs + off];",
-     "double ks = (double)k_scale[bh * bs + off], vs = (double)k_scale[bh * bs + off];"),
-    ("k_row_offset", "memcpy(k8 + (bh * block_size + off) * head_dim", "memcpy(k8 + (bh * block_size + (off ^ 1)) * head_dim"),
+    ("k_not_swizzled", "return (size_t)j * d + (size_t)((c ^ (j % (chunks < 8 ? chunks : 8))) * 16 + e % 16);",
+     "return (size_t)j * d + (size_t)(c * 16 + e % 16);"),
+    ("v_scale_from_k", "memcpy(&vsf, rec + (size_t)32 * d + 64 + 4 * off, 4);", "memcpy(&vsf, rec + (size_t)32 * d + 4 * off, 4);"),
     ("amax_signed", "float a = fabsf(x);", "float a = x;"),
+    ("v_row_stride", "rec[(size_t)16 * head_dim + (size_t)e * 16 + vpos(off)] = (uint8_t)codes[e];",
+     "rec[(size_t)16 * head_dim + (size_t)e * 8 + vpos(off)] = (uint8_t)codes[e];"),
 ]
 
 

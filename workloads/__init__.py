@@ -296,16 +296,14 @@ def cached_token_rows(w: DecodeWorkload):
 
 
 def int8_cache_buffers(w: DecodeWorkload):
-    """Empty INT8 cache buffers for the pool of ``w``: codes ``k8``
-    ``[blocks, n_kv, 16, d]`` and ``v8`` ``[blocks, n_kv, d, 16]`` zeroed, and
-    per-token fp32 scales ``[blocks, n_kv, 16]`` set to NaN, so that a read of
-    a slot that holds no token poisons the result."""
+    """An empty INT8 cache for the pool of ``w``: uint8 records
+    ``[blocks, n_kv, 32 * d + 128]`` with zero codes and NaN scales (the last
+    128 bytes of each record), so that a read of a slot that holds no token
+    poisons the result."""
     nb, nkv, bs, d = w.k_cache.shape
-    k8 = torch.zeros((nb, nkv, bs, d), dtype=torch.int8)
-    v8 = torch.zeros((nb, nkv, d, bs), dtype=torch.int8)
-    ks = torch.full((nb, nkv, bs), float("nan"), dtype=torch.float32)
-    vs = torch.full((nb, nkv, bs), float("nan"), dtype=torch.float32)
-    return k8, v8, ks, vs
+    cache = torch.zeros((nb, nkv, 32 * d + 128), dtype=torch.uint8)
+    cache[:, :, 32 * d:].view(torch.float32).fill_(float("nan"))
+    return cache
 
 
 # ---------------------------------------------------------------------------
