@@ -381,6 +381,31 @@ pkv_status pkv_bm_stats(const pkv_block_manager* bm, pkv_bm_stats_t* out);
 /* Refcount of one block. */
 pkv_status pkv_bm_refcount(const pkv_block_manager* bm, int32_t block, int32_t* refcount);
 
+/*
+ * paged_attention_decode_mq -- several queries per sequence: the last q_len
+ * tokens of every context are new (already written with paged_kv_append, for
+ * instance a draft to verify: "LLM Primer VI" ch. 8, speculative decoding, or
+ * a prefill chunk) and each attends to the context up to its own position:
+ *   query i of sequence b sees tokens j < context_lens[b] - q_len + i + 1.
+ * Otherwise as paged_attention_decode.
+ *
+ *   q, out   : device, [batch][q_len][n_q_heads][head_dim], f16 or bf16
+ *   q_len    : 1 .. 16
+ *   context_lens[b] : >= q_len (0 gives zero rows; 0 < n < q_len is clamped
+ *              to 0 and sets PKV_DEVERR_CONTEXT)
+ *   workspace: paged_attention_mq_workspace_size() bytes, or NULL
+ * Each (sequence, group of kv-head-sharing query heads) runs as one set of
+ * up to 16 (query, head) rows on the tensor cores.
+ */
+pkv_status paged_attention_mq_workspace_size(int32_t batch, int32_t q_len, int32_t n_q_heads, int32_t n_kv_heads,
+                                             int32_t head_dim, pkv_dtype dtype, size_t* bytes);
+pkv_status paged_attention_decode_mq(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t batch, int32_t q_len, int32_t num_blocks,
+                                     float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                     int32_t block_size, void* out, pkv_dtype dtype, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * INT8 paged KV cache (quantised KV, "Transformer anatomy" ch. 15 §15.7:
  * 8-bit K and V halve the cache bytes for a small loss of accuracy).

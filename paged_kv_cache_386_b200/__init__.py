@@ -26,6 +26,7 @@ __all__ = [
     "paged_attention_decode_cascade", "paged_attention_cascade_workspace_size",
     "paged_attention_workspace_size", "paged_kv_copy_blocks", "BlockManager", "pkv_bm_hash_blocks",
     "paged_kv_append_int8", "paged_attention_decode_int8", "int8_cache",
+    "paged_attention_decode_mq", "paged_attention_mq_workspace_size",
     "pkv_get_device_error", "pkv_status_string", "pkv_version", "PagedKVError", "library_path",
     "DEVERR_BLOCK_ID", "DEVERR_CONTEXT", "DEVERR_SLOT", "DEVERR_TIMEOUT", "DEVERR_SCHEDULE", "new_workspace",
 ]
@@ -102,6 +103,11 @@ def _load() -> ctypes.CDLL:
     lib.pkv_version.restype = ctypes.c_int32
     lib.paged_kv_copy_blocks.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p]
     lib.paged_kv_copy_blocks.restype = ctypes.c_int
+    lib.paged_attention_mq_workspace_size.argtypes = [i32, i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(sz)]
+    lib.paged_attention_mq_workspace_size.restype = ctypes.c_int
+    lib.paged_attention_decode_mq.argtypes = [p, p, p, p, i32, p, i32, i32, i32, f32, i32, i32, i32, i32, p,
+                                              ctypes.c_int, p, sz, p]
+    lib.paged_attention_decode_mq.restype = ctypes.c_int
     lib.paged_kv_append_int8.argtypes = [p, p, ctypes.c_int, p, i32, p, i32, i32, i32, i32, p]
     lib.paged_kv_append_int8.restype = ctypes.c_int
     lib.paged_attention_decode_int8.argtypes = [p, p, p, i32, p, i32, i32, f32, i32, i32, i32, i32, p,
@@ -441,4 +447,36 @@ def paged_attention_decode_int8(q, kv_cache, block_tables, context_lens, scale: 
         _dev(q, "q"), _dev(kv_cache, "kv_cache"), _dev(block_tables, "block_tables"), block_tables.shape[1],
         _dev(context_lens, "context_lens"), B, num_blocks, float(scale), n_q, n_kv, d, block_size, _dev(out, "out"),
         _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream)), "paged_attention_decode_int8")
+    return out
+
+
+def paged_attention_mq_workspace_size(batch: int, q_len: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                                      dtype: torch.dtype) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_load().paged_attention_mq_workspace_size(batch, q_len, n_q_heads, n_kv_heads, head_dim, _DTYPE[dtype],
+                                                     ctypes.byref(out)), "paged_attention_mq_workspace_size")
+    return int(out.value)
+
+
+def paged_attention_decode_mq(q, k_cache, v_cache, block_tables, context_lens, scale: float, out=None,
+                              workspace=None, block_size: int = 16, stream=None):
+    """Several queries per sequence: ``q`` ``[batch, q_len, n_q, d]``; query i
+    of a sequence sees its context up to position ``ctx - q_len + i``.
+    Returns ``out`` (shape and dtype of q)."""
+    lib = _load()
+    B, q_len, n_q, d = q.shape
+    num_blocks, n_kv, bs, d2 = k_cache.shape
+    if d2 != d or bs != block_size or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if out is None:
+        out = torch.empty_like(q)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    _check(lib.paged_attention_decode_mq(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables"),
+        block_tables.shape[1], _dev(context_lens, "context_lens"), B, q_len, num_blocks, float(scale), n_q, n_kv, d,
+        bs, _dev(out, "out"), _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream)), "paged_attention_decode_mq")
     return out

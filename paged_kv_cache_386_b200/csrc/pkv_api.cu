@@ -140,10 +140,10 @@ pkv_status encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dt, i
 
 // The decode kernel is launched cooperatively: its CTAs (at most one per SM)
 // are guaranteed to be co-resident, which its grid-wide barrier needs.
-template <int DT, int D, int GPAD, bool kI8 = false>
+template <int DT, int D, int GPAD, bool kI8 = false, bool kMQ = false>
 pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid, size_t smem,
                          cudaStream_t stream) {
-  auto kern = pkv_decode_kernel<DT, D, GPAD, kI8>;
+  auto kern = pkv_decode_kernel<DT, D, GPAD, kI8, kMQ>;
   // Opt in to the largest dynamic shared memory once per device (the launch
   // itself passes the size it needs).
   static bool opted_in[kMaxDevices] = {};
@@ -197,6 +197,25 @@ pkv_status dispatch_i8(int gpad, const CUtensorMap& mk, const DecodeParams& p, i
                        cudaStream_t stream) {
   return gpad == 8 ? launch_decode<DT, 128, 8, true>(mk, mk, p, grid, smem, stream)
                    : launch_decode<DT, 128, 16, true>(mk, mk, p, grid, smem, stream);
+}
+
+// Several queries per sequence (16-bit data, tensor-core consumer).
+template <int DT>
+pkv_status dispatch_mq(int head_dim, int gpad, const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p,
+                       int grid, size_t smem, cudaStream_t stream) {
+  if (head_dim == 64)
+    return gpad == 8 ? launch_decode<DT, 64, 8, false, true>(mk, mv, p, grid, smem, stream)
+                     : launch_decode<DT, 64, 16, false, true>(mk, mv, p, grid, smem, stream);
+  return gpad == 8 ? launch_decode<DT, 128, 8, false, true>(mk, mv, p, grid, smem, stream)
+                   : launch_decode<DT, 128, 16, false, true>(mk, mv, p, grid, smem, stream);
+}
+
+// Heads per segment with q_len queries: the largest divisor of the head group
+// whose rows (heads x queries) fit the 16 rows of a tensor-core tile.
+int heads_per_segment_mq(int group, int q_len) {
+  for (int gp = 16 / q_len; gp >= 1; --gp)
+    if (group % gp == 0) return gp;
+  return 1;
 }
 
 // The INT8 cache (one record per (block, kv head); null for 16-bit caches).
@@ -385,11 +404,13 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
                        float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
                        void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes, void* stream,
                        const pkv_decode_options* options, const float* init, const int32_t* seq_group,
-                       int32_t n_groups, const KvI8* i8 = nullptr) {
+                       int32_t n_groups, const KvI8* i8 = nullptr, int32_t q_len = 1) {
   pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                     num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
   if (st != PKV_OK) return st;
   if (i8 && (dtype == PKV_F32 || head_dim != 128)) return PKV_ERR_UNSUPPORTED;
+  if (q_len < 1) return PKV_ERR_INVALID_ARG;
+  if (q_len > 1 && (q_len > 16 || dtype == PKV_F32 || i8 || init)) return PKV_ERR_UNSUPPORTED;
   if (batch == 0) return st;
   pkv_decode_options opt = {};
   if (options) {
@@ -408,9 +429,11 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   const int group = n_q_heads / n_kv_heads;
-  const int gp = heads_per_segment(group, dtype, opt.force_simt == 1 && !i8);
-  // The INT8 cache always takes the tensor-core consumer (8 rows at least).
-  const int gpad = (gp == 1 && !i8) ? 0 : (gp <= 8 ? 8 : 16);
+  const bool mq = q_len > 1;
+  const int gp = mq ? heads_per_segment_mq(group, q_len) : heads_per_segment(group, dtype, opt.force_simt == 1 && !i8);
+  const int rows = gp * q_len;
+  // The INT8 cache and several queries always take the tensor-core consumer.
+  const int gpad = (rows == 1 && !i8 && !mq) ? 0 : (rows <= 8 ? 8 : 16);
   // One CTA per SM at most (the kernel's grid barrier needs every CTA
   // resident), so the unit count is capped at one per consumer warp of
   // every SM.
@@ -435,7 +458,7 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   if (stages > 4) stages = 4;
   const size_t smem = fixed - 256 + stages * per_round;
 
-  const size_t need = workspace_for(units, sub_chunks, gp, head_dim);
+  const size_t need = workspace_for(units, sub_chunks, rows, head_dim);
   void* ws = workspace;
   bool own = false;
   if (ws == nullptr) {
@@ -477,14 +500,19 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   p.sub_chunks = sub_chunks;
   p.static_permille = static_permille;
   p.stages = stages;
-  p.rec_floats = record_floats(gp, head_dim);
+  p.rec_floats = record_floats(rows, head_dim);
+  p.q_len = q_len;
+  p.rows = rows;
   p.head_dim = head_dim;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.init = init;
   p.seq_group = seq_group;
   p.n_groups = n_groups;
 
-  if (st == PKV_OK && i8) {
+  if (st == PKV_OK && mq) {
+    st = dtype == PKV_F16 ? dispatch_mq<kF16>(head_dim, gpad, mk, mv, p, grid, smem, s)
+                          : dispatch_mq<kBF16>(head_dim, gpad, mk, mv, p, grid, smem, s);
+  } else if (st == PKV_OK && i8) {
     st = dtype == PKV_F16 ? dispatch_i8<kF16>(gpad, mk, p, grid, smem, s) : dispatch_i8<kBF16>(gpad, mk, p, grid, smem, s);
   } else if (st == PKV_OK) {
     switch (dtype) {
@@ -532,6 +560,30 @@ pkv_status paged_attention_decode_int8(const void* q, const uint8_t* kv_cache, c
   return decode_impl(q, kv_cache, kv_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
                      n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, workspace, workspace_bytes, stream,
                      nullptr, nullptr, nullptr, 0, &i8);
+}
+
+pkv_status paged_attention_mq_workspace_size(int32_t batch, int32_t q_len, int32_t n_q_heads, int32_t n_kv_heads,
+                                             int32_t head_dim, pkv_dtype dtype, size_t* bytes) {
+  if (!bytes || batch < 0 || q_len < 1 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0)
+    return PKV_ERR_INVALID_ARG;
+  if (q_len > 16 || dtype == PKV_F32 || elem_bytes(dtype) == 0 || (head_dim != 64 && head_dim != 128))
+    return PKV_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
+  const int rows = heads_per_segment_mq(n_q_heads / n_kv_heads, q_len) * q_len;
+  *bytes = workspace_for(di.sm_count * kConsumerWarps, kDefaultSubChunks, rows, head_dim);
+  return PKV_OK;
+}
+
+pkv_status paged_attention_decode_mq(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t batch, int32_t q_len, int32_t num_blocks,
+                                     float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                     int32_t block_size, void* out, pkv_dtype dtype, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  return decode_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
+                     n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, workspace, workspace_bytes, stream,
+                     nullptr, nullptr, nullptr, 0, nullptr, q_len);
 }
 
 // ---------------------------------------------------------------------------

@@ -289,10 +289,20 @@ struct DecodeParams {
   int32_t sub_chunks;      // balancing chunks cut from the end of each unit's range (0..4)
   int32_t static_permille; // share of each unit's range that the unit keeps
   int32_t stages;      // ring slots per consumer warp
-  int32_t rec_floats;  // floats per partial record: gp * (head_dim + 2), rounded up to 4
+  int32_t rec_floats;  // floats per partial record: rows * (head_dim + 2), rounded up to 4
+  int32_t q_len;       // queries per sequence (the last q_len tokens of its context)
+  int32_t rows;        // rows per segment: q_len * gp
   int32_t head_dim;
   float scale_log2;    // scale * log2(e)
 };
+
+// Row `row` of segment (b, hg) -- query row / gp, head hg * gp + row % gp
+// -- as an index into [batch][q_len][n_q] (q, out; [batch][n_q] when q_len
+// is 1).
+__device__ __forceinline__ size_t out_row(const DecodeParams& p, int b, int hg, int row) {
+  const int qi = row / p.gp;
+  return (static_cast<size_t>(b) * p.q_len + qi) * p.n_q_heads + hg * p.gp + (row - qi * p.gp);
+}
 
 // Position of a warp in its unit's tile range.
 struct Walk {
@@ -452,7 +462,10 @@ __device__ __forceinline__ uint32_t tile_offset(int tok, int dim) {
 }
 
 // ---- tensor-core consumer (16-bit data, 2..16 query heads per kv head) ----
-template <int DT, int D, int GPAD>
+// kMQ: several queries per sequence (rows = query x head); query qi sees the
+// context up to its own position, ctx - q_len + qi, so that in the tile that
+// holds the sequence's last tokens each row has its own causal limit.
+template <int DT, int D, int GPAD, bool kMQ = false>
 struct MmaConsumer {
   static constexpr bool kBf16 = (DT == kBF16);
   static constexpr int ES = 2;
@@ -463,6 +476,12 @@ struct MmaConsumer {
   uint32_t qa[KS][4];
   float o[NT][4];
   float m[2], l[2];
+  int mq_gp = 1, mq_len = 1;  // kMQ: heads per query row block, queries per sequence
+
+  __device__ __forceinline__ void set_mq(int gp, int q_len) {
+    mq_gp = gp;
+    mq_len = q_len;
+  }
 
   // Q of the segment's gp heads from the warp's shared buffer ([gp][D]).
   __device__ __forceinline__ void begin(const uint8_t* qbuf, int gp, int lane) {
@@ -535,6 +554,10 @@ struct MmaConsumer {
     float alpha[2] = {1.f, 1.f};
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
+      // Tokens this row sees in the tile (kMQ: `nv` is the count of context
+      // tokens from the tile's start on, unclamped; query qi stops
+      // q_len - 1 - qi tokens before the context's end).
+      const int nvr = kMQ ? min(kBlockTokens, nv - (mq_len - 1 - (lane / 4 + 8 * r) / mq_gp)) : nv;
       float x[2][2];
       float mx = -INFINITY;
 #pragma unroll
@@ -542,7 +565,7 @@ struct MmaConsumer {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int tok = nt * 8 + 2 * t + e;
-          x[nt][e] = (tok < nv) ? s[nt][2 * r + e] * scale_log2 : -INFINITY;
+          x[nt][e] = (tok < nvr) ? s[nt][2 * r + e] * scale_log2 : -INFINITY;
           mx = fmaxf(mx, x[nt][e]);
         }
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -550,14 +573,16 @@ struct MmaConsumer {
       const float mn = fmaxf(m[r], mx);
       if (mn > m[r]) {
         grow = true;
-        alpha[r] = exp2f(m[r] - mn);
+        // kMQ: a row may have seen no token yet (m = -inf; O and l are 0).
+        alpha[r] = (kMQ && m[r] == -INFINITY) ? 0.f : exp2f(m[r] - mn);
       }
       float sum = 0.f;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          pr[r][nt][e] = exp2f(x[nt][e] - mn);
+          // kMQ: a row with no token so far in this piece has mn = -inf.
+          pr[r][nt][e] = (kMQ && x[nt][e] == -INFINITY) ? 0.f : exp2f(x[nt][e] - mn);
           sum += pr[r][nt][e];
         }
       l[r] = l[r] * alpha[r] + sum;
@@ -592,10 +617,11 @@ struct MmaConsumer {
     }
 
     // Rows of V past the context may hold anything (NaN included): zero them.
+    const int nvt = kMQ ? min(nv, kBlockTokens) : nv;
     uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
-    if (nv < kBlockTokens) {
-      vm0 = ((2 * t < nv) ? 0x0000ffffu : 0u) | ((2 * t + 1 < nv) ? 0xffff0000u : 0u);
-      vm1 = ((2 * t + 8 < nv) ? 0x0000ffffu : 0u) | ((2 * t + 9 < nv) ? 0xffff0000u : 0u);
+    if (nvt < kBlockTokens) {
+      vm0 = ((2 * t < nvt) ? 0x0000ffffu : 0u) | ((2 * t + 1 < nvt) ? 0xffff0000u : 0u);
+      vm1 = ((2 * t + 8 < nvt) ? 0x0000ffffu : 0u) | ((2 * t + 9 < nvt) ? 0xffff0000u : 0u);
     }
 #pragma unroll
     for (int nd2 = 0; nd2 < D / 16; ++nd2) {
@@ -627,9 +653,9 @@ struct MmaConsumer {
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
       const int row = g + 8 * r;
-      if (row >= p.gp) continue;
+      if (row >= p.rows) continue;
       if (rec == nullptr) {
-        T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + row) * D;
+        T* ob = static_cast<T*>(p.out) + out_row(p, b, hg, row) * D;
         const float inv = 1.f / lt[r];
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
@@ -645,8 +671,8 @@ struct MmaConsumer {
         }
       } else {
         if (t == 0) {
-          rec[p.gp * D + row] = m[r];
-          rec[p.gp * D + p.gp + row] = lt[r];
+          rec[p.rows * D + row] = m[r];
+          rec[p.rows * D + p.rows + row] = lt[r];
         }
         float* ro = rec + row * D;
 #pragma unroll
@@ -1083,16 +1109,16 @@ struct MmaConsumerI8 : MmaConsumer<DT, 128, GPAD> {
   }
 };
 
-template <int DT, int D, int GPAD, bool kI8 = false>
+template <int DT, int D, int GPAD, bool kI8 = false, bool kMQ = false>
 struct ConsumerFor {
-  using type = MmaConsumer<DT, D, GPAD>;
+  using type = MmaConsumer<DT, D, GPAD, kMQ>;
 };
 template <int DT, int D>
-struct ConsumerFor<DT, D, 0, false> {
+struct ConsumerFor<DT, D, 0, false, false> {
   using type = SimtConsumer<DT, D>;
 };
 template <int DT, int GPAD>
-struct ConsumerFor<DT, 128, GPAD, true> {
+struct ConsumerFor<DT, 128, GPAD, true, false> {
   using type = MmaConsumerI8<DT, GPAD>;
 };
 
@@ -1120,15 +1146,16 @@ __device__ __forceinline__ void prefetch_slice_l2(const void* base, size_t bytes
   }
 }
 
-// Copy the gp x head_dim Q rows of segment (b, hg) into a warp's shared
+// Copy the rows x head_dim Q rows of segment (b, hg) into a warp's shared
 // buffer with 16-byte cp.async (completion: cp_async_wait_all + __syncwarp).
 template <int ES, int D>
-__device__ __forceinline__ void q_fetch(uint8_t* qbuf, const void* q, int n_q_heads, int b, int hg, int gp,
-                                        int lane) {
-  const uint8_t* src =
-      static_cast<const uint8_t*>(q) + (static_cast<size_t>(b) * n_q_heads + static_cast<size_t>(hg) * gp) * D * ES;
-  const int chunks = gp * D * ES / 16;
-  for (int c = lane; c < chunks; c += 32) cp_async_16(qbuf + c * 16, src + c * 16);
+__device__ __forceinline__ void q_fetch(uint8_t* qbuf, const DecodeParams& p, int b, int hg, int lane) {
+  constexpr int kRowChunks = D * ES / 16;
+  const uint8_t* q = static_cast<const uint8_t*>(p.q);
+  for (int c = lane; c < p.rows * kRowChunks; c += 32) {
+    const int row = c / kRowChunks, w = c - row * kRowChunks;
+    cp_async_16(qbuf + c * 16, q + (out_row(p, b, hg, row) * D * ES) + w * 16);
+  }
   cp_async_commit();
 }
 
@@ -1146,11 +1173,11 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
   using T = typename DTypeInfo<DT>::T;
   constexpr int DPL = D / 32;
   const int seg = mt.x, b = seg / p.ng, hg = seg % p.ng, n = mt.y - u + 1;
-  const int mo = p.gp * D + g, lo = p.gp * D + p.gp + g, oo = g * D + lane * DPL;
+  const int mo = p.rows * D + g, lo = p.rows * D + p.rows + g, oo = g * D + lane * DPL;
   auto rec_of = [&](int j) -> const float* {  // record of piece j (chunk u + j)
     return p.records + (static_cast<size_t>(u + j) * 2 + (j == 0 ? mt.z : 0)) * p.rec_floats;
   };
-  T* const ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g) * D + lane * DPL;
+  T* const ob = static_cast<T*>(p.out) + out_row(p, b, hg, g) * D + lane * DPL;
   auto store = [&](const float (&acc)[DPL], float inv) {
     if constexpr (DPL == 4) {
       store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
@@ -1250,8 +1277,9 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
 // producer/consumer pipeline; a grid-wide barrier follows (every wait before
 // it is bounded, so every thread reaches it); phase 2 merges split segments
 // and zero-fills the rows of empty sequences.
-// kI8: the cache holds INT8 codes and per-token scales (MmaConsumerI8).
-template <int DT, int D, int GPAD, bool kI8>
+// kI8: the cache holds INT8 records (MmaConsumerI8).  kMQ: q_len > 1
+// queries per sequence (tensor-core consumer with per-row causal limits).
+template <int DT, int D, int GPAD, bool kI8, bool kMQ>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     pkv_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeParams p) {
@@ -1264,9 +1292,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   constexpr int kRingStride = kI8 ? i8_record_bytes(D) : 2 * kTileBytes;
   constexpr int kStageBytes = kRingStride;  // bytes landing per slot
   constexpr int kQBufBytes = (GPAD == 0 ? 1 : GPAD) * D * ES;
-  using Consumer = typename ConsumerFor<DT, D, GPAD, kI8>::type;
+  using Consumer = typename ConsumerFor<DT, D, GPAD, kI8, kMQ>::type;
   using OutT = typename DTypeInfo<DT>::T;
   static_assert(!kI8 || (D == 128 && GPAD != 0), "INT8 cache: head_dim 128, tensor-core consumer");
+  static_assert(!kMQ || (GPAD != 0 && !kI8), "several queries: 16-bit cache, tensor-core consumer");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -1310,7 +1339,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     int local = 0;
     for (int b = lo; b < hi; ++b) {
       const int c0 = __ldg(p.context_lens + b);
-      const int c = clamp_ctx(c0, max_ctx);
+      int c = clamp_ctx(c0, max_ctx);
+      if (c > 0 && c < p.q_len) c = 0;  // fewer tokens than queries: flagged, no output but zeros
       if (c != c0) flag_error(PKV_DEVERR_CONTEXT);
       ctxs[b] = c;
       local += ((c + kBlockTokens - 1) / kBlockTokens) * p.ng;
@@ -1504,10 +1534,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           cur_hg = wk.hg;
           seg_start = prefix[wk.b] + wk.hg * wk.nb;
           seg_end = seg_start + wk.nb;
-          if (!q_ready) q_fetch<ES, D>(qbuf, p.q, p.n_q_heads, wk.b, wk.hg, p.gp, lane);
+          if (!q_ready) q_fetch<ES, D>(qbuf, p, wk.b, wk.hg, lane);
           cp_async_wait_all();
           __syncwarp();
-          cs.begin(qbuf, p.gp, lane);
+          cs.begin(qbuf, p.rows, lane);
+          if constexpr (kMQ) cs.set_mq(p.gp, p.q_len);
           if (p.init != nullptr && wk.j == 0 && has_init(p, wk.b)) cs.load_init(p, wk.b, wk.hg, lane);
           __syncwarp();
           q_ready = false;
@@ -1519,7 +1550,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (wk.j == wk.nb - 1 && !last) {
           Walk nx = wk;
           walk_next(nx, prefix, ctxs, B, p.ng);
-          q_fetch<ES, D>(qbuf, p.q, p.n_q_heads, nx.b, nx.hg, p.gp, lane);
+          q_fetch<ES, D>(qbuf, p, nx.b, nx.hg, lane);
           q_ready = true;
         }
         const int slot = warp * p.stages + stage;
@@ -1540,13 +1571,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           n1 = info.z;
           Walk nw;
           if (next_chunk >= 0 && walk_begin(nw, prefix, ctxs, B, n0, n1)) {
-            q_fetch<ES, D>(qbuf, p.q, p.n_q_heads, nw.b, nw.hg, p.gp, lane);
+            q_fetch<ES, D>(qbuf, p, nw.b, nw.hg, lane);
             q_ready = true;
           } else {
             next_chunk = -1;
           }
         }
-        const int nv = min(kBlockTokens, wk.ctx - wk.j * kBlockTokens);
+        // Context tokens from this tile's start on (the tile holds at most 16).
+        const int rem = wk.ctx - wk.j * kBlockTokens;
+        const int nv = kMQ ? rem : min(kBlockTokens, rem);
         const uint32_t kaddr = smem_u32(ring + static_cast<size_t>(slot) * kRingStride);
         const uint32_t vaddr = kI8 ? kaddr + D * kBlockTokens : kaddr + kTileBytes;
         cs.tile(kaddr, vaddr, nv, p.scale_log2, lane);
@@ -1585,17 +1618,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   {
     constexpr int kWarps = kConsumerWarps + 1;
     const int gw = blockIdx.x * kWarps + warp, n_warps = gridDim.x * kWarps;
-    const int items = n_chunks * p.gp;
+    const int items = n_chunks * p.rows;
     const int n_segs = B * p.ng;
     // Item metadata is loaded 32 items at a time, lane t for the round's
     // t-th item of this warp.
     for (int base = gw; base < items; base += 32 * n_warps) {
       int4 my_item = make_int4(-1, 0, 0, 0);
       const int i_lane = base + lane * n_warps;
-      if (i_lane < items) my_item = __ldcg(p.meta + i_lane / p.gp);
+      if (i_lane < items) my_item = __ldcg(p.meta + i_lane / p.rows);
       for (int t = 0; t < 32 && base + t * n_warps < items; ++t) {
         const int i = base + t * n_warps;
-        const int c = i / p.gp;
+        const int c = i / p.rows;
         int4 mt;
         mt.x = __shfl_sync(0xffffffffu, my_item.x, t);
         mt.y = __shfl_sync(0xffffffffu, my_item.y, t);
@@ -1603,7 +1636,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         // Entries of chunks that an aborted launch never reached may be
         // stale: only well-formed ones are merged.
         if (mt.x >= 0 && mt.x < n_segs && mt.y > c && mt.y < n_chunks && (mt.z == 0 || mt.z == 1))
-          merge_head<DT, D>(p, c, mt, i % p.gp, lane);
+          merge_head<DT, D>(p, c, mt, i % p.rows, lane);
       }
     }
     // The claim counter must have seen every balancing chunk plus one failed
@@ -1624,9 +1657,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int b = sgi / p.ng, hg = sgi % p.ng;
       if (ctxs[b] != 0) continue;
       const bool with_init = p.init != nullptr && has_init(p, b);
-      for (int e = lane; e < p.gp * (D / 4); e += 32) {
+      for (int e = lane; e < p.rows * (D / 4); e += 32) {
         const int g = e / (D / 4), d4 = (e % (D / 4)) * 4;
-        const size_t rowi = static_cast<size_t>(b) * p.n_q_heads + hg * p.gp + g;
+        const size_t rowi = out_row(p, b, hg, g);  // the initial state is given for q_len 1 only
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         float inv = 0.f;
         if (with_init) {
