@@ -182,7 +182,12 @@ def run_ours(args) -> None:
     torch.cuda.set_device(dev)
 
     make, desc = WORKLOADS[args.workload]
-    w = make(args.seed)
+    mq = args.q_len > 1
+    if mq and (args.workload != "llama3_8b_gqa" or args.cascade or args.kv != "16-bit"):
+        raise SystemExit("--q-len > 1 is measured on llama3_8b_gqa with the 16-bit cache")
+    w = W.uniform_gqa(seed=args.seed, q_len=args.q_len) if mq else make(args.seed)
+    if mq:
+        desc += f"; {args.q_len} queries per sequence (the last {args.q_len} tokens, causal)"
     es = w.k_cache.element_size()
     int8 = args.kv == "int8"
     if int8 and args.cascade:
@@ -211,6 +216,9 @@ def run_ours(args) -> None:
                                                              cv.block_tables, cv.context_lens))
         ws = torch.zeros(pkv.paged_attention_cascade_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
                                                                     w.dtype), dtype=torch.uint8, device=dev)
+    elif mq:
+        ws = torch.zeros(pkv.paged_attention_mq_workspace_size(w.batch, args.q_len, w.n_q_heads, w.n_kv_heads,
+                                                               w.head_dim, w.dtype), dtype=torch.uint8, device=dev)
     else:
         ws = torch.zeros(pkv.paged_attention_workspace_size(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim,
                                                             w.dtype), dtype=torch.uint8, device=dev)
@@ -222,7 +230,9 @@ def run_ours(args) -> None:
             pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream_)
 
     def decode(stream_=None):
-        if int8:
+        if mq:
+            pkv.paged_attention_decode_mq(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream_)
+        elif int8:
             pkv.paged_attention_decode_int8(q, kv8, bt, cl, w.scale, out=out, workspace=ws, stream=stream_)
         elif args.cascade:
             pkv.paged_attention_decode_cascade(q, kc, vc, c_pt, c_pl, c_sg, c_bt, c_cl, w.scale, out=out,
@@ -307,7 +317,7 @@ def run_ours(args) -> None:
     step_s = sum(step_ms) / 1e3
     max_step_s = reduce_max(step_s, world, dev)
     value = aggregate(kv_bytes, max_step_s / args.steps, world) / 1e9
-    tokens_per_s = aggregate(w.batch, max_step_s / args.steps, world)
+    tokens_per_s = aggregate(w.batch * args.q_len, max_step_s / args.steps, world)
     dec_avg_s = sum(decode_ms) / len(decode_ms) / 1e3
     achieved = decode_bytes / dec_avg_s / 1e9
     peak, peak_kind = measured_hbm_peak()
@@ -364,7 +374,7 @@ def run_ours(args) -> None:
     result = None
     if rank == 0:
         cpu = (cpu_baseline(w, kv_bytes, budget_s=args.cpu_budget)
-               if (world == 1 and not args.no_cpu and not int8) else None)
+               if (world == 1 and not args.no_cpu and not int8 and not mq) else None)
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -386,7 +396,8 @@ def run_ours(args) -> None:
             "roofline": {"bound": "hbm",
                          "kernel": ("paged_attention_decode_cascade (pkv_prefix_kernel + pkv_decode_kernel)"
                                     if args.cascade else
-                                    "paged_attention_decode_int8 (pkv_decode_kernel, INT8)" if int8
+                                    "paged_attention_decode_int8 (pkv_decode_kernel, INT8)" if int8 else
+                                    "paged_attention_decode_mq (pkv_decode_kernel, several queries)" if mq
                                     else "paged_attention_decode (pkv_decode_kernel)"),
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -499,6 +510,8 @@ def main(argv=None) -> None:
     ap.add_argument("--cascade", action="store_true",
                     help="decode shared-prefix workloads with paged_attention_decode_cascade")
     ap.add_argument("--ref-seqs", type=int, default=0, help="sequences per reference-arm step (0: all)")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="queries per sequence (multi-query decode of the last q_len tokens)")
     ap.add_argument("--kv", choices=["16-bit", "int8"], default="16-bit",
                     help="cache format: the workload's 16-bit dtype, or INT8 codes with per-token scales")
     args = ap.parse_args(argv)
