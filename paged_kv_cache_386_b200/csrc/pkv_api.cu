@@ -8,6 +8,7 @@
 #include "pagedkv.h"
 #include "pkv_kernels.cuh"
 #include "pkv_prefix.cuh"
+#include "pkv_prefix_tc.cuh"
 
 namespace pkv {
 namespace {
@@ -247,6 +248,32 @@ pkv_status launch_prefix(const CUtensorMap& mk, const CUtensorMap& mv, const Pre
   const int rows = pp.batch * pp.group;
   const dim3 grid((rows + kPrefixRows - 1) / kPrefixRows, n_kv, pp.n_groups);
   kern<<<grid, kPrefixThreads, smem, stream>>>(mk, mv, pp);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+// The tensor-memory prefix kernel (head dim 128): 128-row tiles, 192 KiB of
+// operands plus barriers and the member list.
+size_t prefix_tc_smem(int batch) {
+  return 1024 + kTcSmemBytes + (2 * kTcStages + 7) * sizeof(uint64_t) + 16 + static_cast<size_t>(batch) * 4;
+}
+
+template <int DT>
+pkv_status launch_prefix_tc(const CUtensorMap& mk, const CUtensorMap& mv, const PrefixParams& pp, int n_kv,
+                            cudaStream_t stream) {
+  auto kern = pkv_prefix_tc_kernel<DT>;
+  static bool opted_in[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+  if (!opted_in[dev]) {
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - 256) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    opted_in[dev] = true;
+  }
+  const int rows = pp.batch * pp.group;
+  const dim3 grid((rows + kTcRows - 1) / kTcRows, n_kv, pp.n_groups);
+  kern<<<grid, kTcThreads, prefix_tc_smem(pp.batch), stream>>>(mk, mv, pp);
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -705,8 +732,13 @@ pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, co
   pp.scale_log2 = scale * 1.4426950408889634f;
   const size_t stage_bytes = static_cast<size_t>(2) * kPrefixBlocks * (head_dim * 2 / 128) * kBoxBytes;
   const size_t smem = 1024 + kPrefixStages * (stage_bytes + 2 * sizeof(uint64_t)) + 16 + static_cast<size_t>(batch) * 4;
-  if (smem + 256 > static_cast<size_t>(di.smem_optin)) st = st == PKV_OK ? PKV_ERR_UNSUPPORTED : st;
-  if (st == PKV_OK) {
+  // Head dim 128 runs on the tensor-memory kernel when its operands fit.
+  const bool tc = head_dim == 128 && prefix_tc_smem(batch) + 256 <= static_cast<size_t>(di.smem_optin);
+  if (!tc && smem + 256 > static_cast<size_t>(di.smem_optin)) st = st == PKV_OK ? PKV_ERR_UNSUPPORTED : st;
+  if (st == PKV_OK && tc) {
+    st = dtype == PKV_F16 ? launch_prefix_tc<kF16>(mk, mv, pp, n_kv_heads, s)
+                          : launch_prefix_tc<kBF16>(mk, mv, pp, n_kv_heads, s);
+  } else if (st == PKV_OK) {
     if (dtype == PKV_F16)
       st = head_dim == 64 ? launch_prefix<kF16, 64>(mk, mv, pp, n_kv_heads, smem, s)
                           : launch_prefix<kF16, 128>(mk, mv, pp, n_kv_heads, smem, s);
