@@ -198,6 +198,30 @@ pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, co
                                           int32_t block_size, void* out, pkv_dtype dtype,
                                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Tuning and test hooks for paged_attention_decode_cascade_ex. Zero-initialise. */
+typedef struct pkv_cascade_options {
+  int32_t prefix_splits; /* 0: default; 1..4: CTAs (one thread-block cluster) per 128-row prefix
+                            tile, each taking an equal share of the prefix, merged in the
+                            cluster's rank 0 through distributed shared memory (tensor-memory
+                            prefix kernel only) */
+  int32_t prefix_kernel; /* 0: default (tensor-memory kernel for head_dim 128, else the mma.sync
+                            kernel); 1: tensor-memory kernel (PKV_ERR_UNSUPPORTED where it does
+                            not apply); 2: mma.sync kernel */
+  int32_t reserved[6];   /* must be zero */
+} pkv_cascade_options;
+
+/* paged_attention_decode_cascade with options (NULL options = the default). */
+pkv_status paged_attention_decode_cascade_ex(const void* q, const void* k_cache, const void* v_cache,
+                                             int32_t n_groups, const int32_t* prefix_block_tables,
+                                             int32_t max_prefix_blocks, const int32_t* prefix_lens,
+                                             const int32_t* seq_group, const int32_t* block_tables,
+                                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                             int32_t batch, int32_t num_blocks, float scale,
+                                             int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                             int32_t block_size, void* out, pkv_dtype dtype,
+                                             void* workspace, size_t workspace_bytes, void* stream,
+                                             const pkv_cascade_options* options);
+
 /* Tuning and test hooks for paged_attention_decode_ex. Zero-initialise. */
 struct pkv_decode_options {
   int32_t num_units;   /* 0: default split (one work unit per consumer warp on every SM);

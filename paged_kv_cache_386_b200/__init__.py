@@ -53,6 +53,11 @@ class _Options(ctypes.Structure):
                 ("reserved", ctypes.c_int32 * 4)]
 
 
+class _CascadeOptions(ctypes.Structure):
+    _fields_ = [("prefix_splits", ctypes.c_int32), ("prefix_kernel", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
+
+
 class _BMStats(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int32), ("free_blocks", ctypes.c_int32),
                 ("cached_idle_blocks", ctypes.c_int32), ("used_blocks", ctypes.c_int32),
@@ -93,6 +98,9 @@ def _load() -> ctypes.CDLL:
     lib.paged_attention_decode_cascade.argtypes = [p, p, p, i32, p, i32, p, p, p, i32, p, i32, i32, f32, i32, i32,
                                                    i32, i32, p, ctypes.c_int, p, sz, p]
     lib.paged_attention_decode_cascade.restype = ctypes.c_int
+    lib.paged_attention_decode_cascade_ex.argtypes = lib.paged_attention_decode_cascade.argtypes + [
+        ctypes.POINTER(_CascadeOptions)]
+    lib.paged_attention_decode_cascade_ex.restype = ctypes.c_int
     lib.paged_attention_decode_noalloc.argtypes = dec[:15] + [p]
     lib.paged_attention_decode_noalloc.restype = ctypes.c_int
     lib.pkv_get_device_error.argtypes = [p, ctypes.POINTER(ctypes.c_uint32)]
@@ -229,12 +237,15 @@ def paged_attention_cascade_workspace_size(batch: int, n_q_heads: int, n_kv_head
 
 def paged_attention_decode_cascade(q, k_cache, v_cache, prefix_block_tables, prefix_lens, seq_group,
                                    block_tables, context_lens, scale: float, out=None, workspace=None,
-                                   block_size: int = 16, stream=None):
+                                   block_size: int = 16, stream=None, prefix_splits: int = 0,
+                                   prefix_kernel: int = 0):
     """Decode for sequences that share prefix blocks: group i's prefix
     (``prefix_lens[i]`` tokens in ``prefix_block_tables[i]``) is attended once
     per kv head for all its members (``seq_group[b] == i``), then each
     sequence's private suffix (``block_tables[b]``, ``context_lens[b]``
-    tokens) continues from that state."""
+    tokens) continues from that state.  ``prefix_splits`` (1-4, 0 = default)
+    and ``prefix_kernel`` (0 default, 1 tensor-memory, 2 mma.sync) are the
+    tuning hooks of ``pkv_cascade_options``."""
     lib = _load()
     B, n_q, d = q.shape
     num_blocks, n_kv, bs, d2 = k_cache.shape
@@ -250,14 +261,15 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, prefix_block_tables, pre
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
     n_groups = prefix_lens.shape[0]
-    _check(lib.paged_attention_decode_cascade(
+    opts = _CascadeOptions(prefix_splits=int(prefix_splits), prefix_kernel=int(prefix_kernel))
+    _check(lib.paged_attention_decode_cascade_ex(
         _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), n_groups,
         _dev(prefix_block_tables, "prefix_block_tables") if n_groups else None,
         prefix_block_tables.shape[1] if n_groups else 0,
         _dev(prefix_lens, "prefix_lens") if n_groups else None, _dev(seq_group, "seq_group") if n_groups else None,
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
         B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
-        ws_ptr, ws_bytes, _stream(stream)), "paged_attention_decode_cascade")
+        ws_ptr, ws_bytes, _stream(stream), ctypes.byref(opts)), "paged_attention_decode_cascade")
     return out
 
 

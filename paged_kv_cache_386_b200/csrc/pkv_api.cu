@@ -257,9 +257,56 @@ size_t prefix_tc_smem(int batch) {
   return 1024 + kTcSmemBytes + (2 * kTcStages + 7) * sizeof(uint64_t) + 16 + static_cast<size_t>(batch) * 4;
 }
 
+// Launch configuration of the tensor-memory prefix kernel: one cluster of
+// `splits` CTAs per 128-row tile of every (group, kv head).
+cudaLaunchConfig_t prefix_tc_config(const PrefixParams& pp, int n_kv, int splits, cudaStream_t stream,
+                                    cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  const int rows = pp.batch * pp.group;
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + kTcRows - 1) / kTcRows * splits), n_kv, pp.n_groups);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = prefix_tc_smem(pp.batch);
+  cfg.stream = stream;
+  attr->id = cudaLaunchAttributeClusterDimension;
+  attr->val.clusterDim.x = static_cast<unsigned>(splits);
+  attr->val.clusterDim.y = 1;
+  attr->val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Prefix shares per tile: enough clusters to cover the SMs once, at most
+// kTcMaxSplit, and only sizes the device can co-schedule.  Rows per group are
+// not known on the host; the estimate takes every group's tiles as full but
+// the total as at most the tiles of the batch plus one ragged tile per group.
+template <int DT>
+int prefix_tc_splits(const PrefixParams& pp, int n_kv, int sm_count, cudaStream_t stream) {
+  const long tiles_batch = (static_cast<long>(pp.batch) * pp.group + kTcRows - 1) / kTcRows;
+  const long ctas = static_cast<long>(n_kv) * std::min(tiles_batch * pp.n_groups, tiles_batch + pp.n_groups - 1);
+  int splits = static_cast<int>(std::max(1L, std::min<long>(kTcMaxSplit, sm_count / std::max(1L, ctas))));
+  // Whether clusters of each size can be co-scheduled, per device (0 unknown, 1 yes, -1 no).
+  static int feasible[kMaxDevices][kTcMaxSplit + 1] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+  for (; splits > 1; --splits) {
+    if (feasible[dev][splits] == 0) {
+      cudaLaunchAttribute attr;
+      cudaLaunchConfig_t cfg = prefix_tc_config(pp, n_kv, splits, stream, &attr);
+      int clusters = 0;
+      const bool yes =
+          cudaOccupancyMaxActiveClusters(&clusters, pkv_prefix_tc_kernel<DT>, &cfg) == cudaSuccess && clusters > 0;
+      (void)cudaGetLastError();
+      feasible[dev][splits] = yes ? 1 : -1;
+    }
+    if (feasible[dev][splits] > 0) break;
+  }
+  return splits;
+}
+
 template <int DT>
 pkv_status launch_prefix_tc(const CUtensorMap& mk, const CUtensorMap& mv, const PrefixParams& pp, int n_kv,
-                            cudaStream_t stream) {
+                            int splits, int sm_count, cudaStream_t stream) {
   auto kern = pkv_prefix_tc_kernel<DT>;
   static bool opted_in[kMaxDevices] = {};
   int dev = 0;
@@ -271,10 +318,12 @@ pkv_status launch_prefix_tc(const CUtensorMap& mk, const CUtensorMap& mv, const 
       return PKV_ERR_CUDA;
     opted_in[dev] = true;
   }
-  const int rows = pp.batch * pp.group;
-  const dim3 grid((rows + kTcRows - 1) / kTcRows, n_kv, pp.n_groups);
-  kern<<<grid, kTcThreads, prefix_tc_smem(pp.batch), stream>>>(mk, mv, pp);
-  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  if (splits <= 0) splits = prefix_tc_splits<DT>(pp, n_kv, sm_count, stream);
+  if (splits > kTcMaxSplit) return PKV_ERR_INVALID_ARG;
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t cfg = prefix_tc_config(pp, n_kv, splits, stream, &attr);
+  if (cfg.gridDim.x > 0x7fffffffu / 2) return PKV_ERR_INVALID_ARG;
+  return cudaLaunchKernelEx(&cfg, kern, mk, mv, pp) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 }  // namespace
@@ -679,6 +728,27 @@ pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, co
                                           float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                           int32_t block_size, void* out, pkv_dtype dtype, void* workspace,
                                           size_t workspace_bytes, void* stream) {
+  return paged_attention_decode_cascade_ex(q, k_cache, v_cache, n_groups, prefix_block_tables, max_prefix_blocks,
+                                           prefix_lens, seq_group, block_tables, max_blocks_per_seq, context_lens,
+                                           batch, num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out,
+                                           dtype, workspace, workspace_bytes, stream, nullptr);
+}
+
+pkv_status paged_attention_decode_cascade_ex(const void* q, const void* k_cache, const void* v_cache,
+                                             int32_t n_groups, const int32_t* prefix_block_tables,
+                                             int32_t max_prefix_blocks, const int32_t* prefix_lens,
+                                             const int32_t* seq_group, const int32_t* block_tables,
+                                             int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
+                                             int32_t num_blocks, float scale, int32_t n_q_heads, int32_t n_kv_heads,
+                                             int32_t head_dim, int32_t block_size, void* out, pkv_dtype dtype,
+                                             void* workspace, size_t workspace_bytes, void* stream,
+                                             const pkv_cascade_options* options) {
+  pkv_cascade_options opt = {};
+  if (options) opt = *options;
+  if (opt.prefix_splits < 0 || opt.prefix_splits > kTcMaxSplit || opt.prefix_kernel < 0 || opt.prefix_kernel > 2)
+    return PKV_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (opt.reserved[i] != 0) return PKV_ERR_INVALID_ARG;
   pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                     num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
   if (st != PKV_OK || batch == 0) return st;
@@ -733,11 +803,13 @@ pkv_status paged_attention_decode_cascade(const void* q, const void* k_cache, co
   const size_t stage_bytes = static_cast<size_t>(2) * kPrefixBlocks * (head_dim * 2 / 128) * kBoxBytes;
   const size_t smem = 1024 + kPrefixStages * (stage_bytes + 2 * sizeof(uint64_t)) + 16 + static_cast<size_t>(batch) * 4;
   // Head dim 128 runs on the tensor-memory kernel when its operands fit.
-  const bool tc = head_dim == 128 && prefix_tc_smem(batch) + 256 <= static_cast<size_t>(di.smem_optin);
+  const bool tc_fits = head_dim == 128 && prefix_tc_smem(batch) + 256 <= static_cast<size_t>(di.smem_optin);
+  if (opt.prefix_kernel == 1 && !tc_fits) return PKV_ERR_UNSUPPORTED;
+  const bool tc = tc_fits && opt.prefix_kernel != 2;
   if (!tc && smem + 256 > static_cast<size_t>(di.smem_optin)) st = st == PKV_OK ? PKV_ERR_UNSUPPORTED : st;
   if (st == PKV_OK && tc) {
-    st = dtype == PKV_F16 ? launch_prefix_tc<kF16>(mk, mv, pp, n_kv_heads, s)
-                          : launch_prefix_tc<kBF16>(mk, mv, pp, n_kv_heads, s);
+    st = dtype == PKV_F16 ? launch_prefix_tc<kF16>(mk, mv, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s)
+                          : launch_prefix_tc<kBF16>(mk, mv, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s);
   } else if (st == PKV_OK) {
     if (dtype == PKV_F16)
       st = head_dim == 64 ? launch_prefix<kF16, 64>(mk, mv, pp, n_kv_heads, smem, s)

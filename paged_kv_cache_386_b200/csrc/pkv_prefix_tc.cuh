@@ -9,8 +9,12 @@
 // scaled scores, is the state from which the decode kernel continues over the
 // sequence's private suffix.
 //
-// One CTA per 128-row tile of one (group, kv head), head dim 128, 192
-// threads:
+// A cluster of 1-4 CTAs per 128-row tile of one (group, kv head), head dim
+// 128; CTA k of the cluster takes the k-th share of the prefix stages, so that
+// a few tiles still fill the SMs.  After its last stage each CTA of rank > 0
+// leaves its partial (O, m, l) in its own shared memory; rank 0 reads them
+// through distributed shared memory, merges them with its own (each term
+// scaled by 2^(m_k - max m)) and writes the row's state.  192 threads:
 //   warps 0-3  softmax: thread r owns row r (tensor-memory lane r);
 //   warp 4     producer: TMA loads of 64 prefix tokens (4 blocks) of K and V
 //              per stage into a 4-stage ring;
@@ -54,6 +58,46 @@ constexpr int kTcStages = 4;
 constexpr int kTcSmemBytes = kTcQBytes + 2 * kTcPBytes + kTcStages * kTcStageBytes;  // 192 KiB
 constexpr uint32_t kTcTmemCols = 256;  // S0 [0,64), S1 [64,128), O [128,256)
 constexpr uint32_t kTcOCol = 2 * kTcKeys;
+constexpr int kTcMaxSplit = 4;          // CTAs per cluster (prefix shares per tile)
+constexpr int kTcPartStride = 128 + 4;  // floats per row of a partial O in shared memory (float4 accesses
+                                        // of 8 consecutive rows fall in distinct bank groups)
+static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcStages * kTcStageBytes,
+              "a partial state fits in the drained K/V ring");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster; writes before it are visible to
+// distributed-shared-memory reads after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// The address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
 // stride byte offsets (16-byte units), descriptor version 1, 128-byte swizzle.
@@ -148,7 +192,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ int n_members;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, kvh = blockIdx.y, grp = blockIdx.z;
+  const uint32_t crank = cluster_rank(), csize = cluster_size();
+  const int tile = blockIdx.x / csize, kvh = blockIdx.y, grp = blockIdx.z;
   const int G = p.group;
 
   // Members of this group, in increasing sequence order (block-wide compaction).
@@ -175,14 +220,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   const int R = n_members * G;
   const int row0 = tile * kTcRows;
-  if (row0 >= R) return;  // uniform over the CTA: no barrier or tensor memory is in use yet
+  if (row0 >= R) return;  // uniform over the cluster: no barrier or tensor memory is in use yet
 
   int plen = __ldg(p.prefix_lens + grp);
   if (plen < 0 || plen > p.max_prefix_blocks * kBlockTokens || (plen % kBlockTokens) != 0) {
     flag_error(PKV_DEVERR_CONTEXT);
     plen = plen < 0 ? 0 : min(plen - plen % kBlockTokens, p.max_prefix_blocks * kBlockTokens);
   }
-  const int n_stages = (plen + kTcKeys - 1) / kTcKeys;
+  // This CTA's share of the prefix: stages [s_begin, s_begin + n_stages).
+  const int n_total = (plen + kTcKeys - 1) / kTcKeys;
+  const int s_begin = n_total * static_cast<int>(crank) / static_cast<int>(csize);
+  const int n_stages = n_total * static_cast<int>(crank + 1) / static_cast<int>(csize) - s_begin;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kTcStages; ++i) {
@@ -226,6 +274,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);  // softmax warps' lanes
+  float* part_o = reinterpret_cast<float*>(ring);  // a rank > 0 CTA's partial O: [128 rows][kTcPartStride]
+  float* part_ml = part_o + kTcRows * kTcPartStride;  // its m [128], then l [128]
+  float m_ref = -INFINITY, l_sum = 0.f;  // the softmax thread's row state
+  bool row_ok = true;
 
   if (warp == 4) {
     // ---------------- producer: 16 TMA requests per stage, one per lane ----------------
@@ -240,7 +293,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < n_stages; ++s) {
       const int slot = s % kTcStages;
       if (!mbar_wait_bounded(&kv_empty[slot], ((s / kTcStages) & 1) ^ 1u, abort_flag, kWaitLimitNs)) break;
-      const int j = s * kTcBlocks + blk;
+      const int j = (s_begin + s) * kTcBlocks + blk;
       // Blocks past the prefix reload block 0 of the prefix (finite values;
       // their probabilities are 0).
       int phys = __ldg(tab + (j * kBlockTokens < plen ? j : 0));
@@ -316,8 +369,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // ---------------- softmax: thread r owns row r ----------------
     const int r = threadIdx.x;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m_ref = -INFINITY, l_sum = 0.f;
     // Every tensor-memory access below is warp-converged (.sync.aligned):
     // waits and decisions are made warp-uniform first.
     bool ok = true;
@@ -338,7 +389,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[s & 1]);
 
-      const int live = min(kTcKeys, plen - s * kTcKeys);
+      const int live = min(kTcKeys, plen - (s_begin + s) * kTcKeys);
       float mx8[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) mx8[j] = -INFINITY;
@@ -401,42 +452,107 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // The row's state: O from tensor memory (unnormalised), m, l.
-    const int row = row0 + r;
     if (ok && n_stages > 0)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(n_stages - 1) & 1], ((n_stages - 1) >> 1) & 1,
                                                       abort_flag, kWaitLimitNs));
     tc_fence_after();
-    if (ok) {
-      const bool mine = row < R;
-      size_t rowi = 0;
-      if (mine) rowi = static_cast<size_t>(members[row / G]) * p.n_q_heads + kvh * G + row % G;
-      float* ob = p.init + rowi * D;
+    row_ok = ok;
+    if (crank > 0) {
+      // Partial state into the drained ring (every copy into it has been
+      // consumed by an MMA that has completed); l = NaN marks a failed row.
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
-        if (n_stages > 0) {
-          tmem_ld32(lane_base + kTcOCol + c * 32, v);  // every lane of the warp
+        if (ok && n_stages > 0) {
+          tmem_ld32(lane_base + kTcOCol + c * 32, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0.f;
         }
-        if (mine) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(ob + c * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(part_o + r * kTcPartStride + c * 32 + i) =
+              make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+      part_ml[r] = m_ref;
+      part_ml[kTcRows + r] = ok ? l_sum : __int_as_float(0x7fc00000);
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // partial states written
+  tc_fence_after();
+  if (warp < 4 && crank == 0) {
+    // The row's state: O (unnormalised), m, l, merged over the cluster.
+    const int r = threadIdx.x;
+    const int row = row0 + r;
+    float m_all = m_ref;
+    float mk[kTcMaxSplit], lk[kTcMaxSplit];
+    bool valid = row_ok;
+    const uint32_t ml_addr = smem_u32(part_ml);
+#pragma unroll
+    for (int k = 1; k < kTcMaxSplit; ++k) {
+      mk[k] = -INFINITY;
+      lk[k] = 0.f;
+      if (k < static_cast<int>(csize)) {
+        mk[k] = ld_cluster(cluster_map(ml_addr + r * 4, k));
+        lk[k] = ld_cluster(cluster_map(ml_addr + (kTcRows + r) * 4, k));
+        valid = valid && !isnan(lk[k]);
+        m_all = fmaxf(m_all, mk[k]);
+      }
+    }
+    // Weight of each share: 2^(m_k - max m), 0 for a share with no keys.
+    const float a0 = m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_all);
+    float l_all = a0 * l_sum;
+#pragma unroll
+    for (int k = 1; k < kTcMaxSplit; ++k) {
+      mk[k] = mk[k] == -INFINITY ? 0.f : exp2f(mk[k] - m_all);  // now the weight
+      l_all += mk[k] * lk[k];
+    }
+    const bool mine = row < R && valid;
+    size_t rowi = 0;
+    if (mine) rowi = static_cast<size_t>(members[row / G]) * p.n_q_heads + kvh * G + row % G;
+    float* ob = p.init + rowi * D;
+    const uint32_t po_addr = smem_u32(part_o) + r * kTcPartStride * 4;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float v[32];
+      if (row_ok && n_stages > 0) {
+        tmem_ld32(lane_base + kTcOCol + c * 32, v);  // every lane of the warp
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= a0;
+#pragma unroll
+      for (int k = 1; k < kTcMaxSplit; ++k) {
+        if (k >= static_cast<int>(csize)) break;
+        const uint32_t src = cluster_map(po_addr + c * 128, k);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 t = ld_cluster4(src + i * 4);
+          v[i] += mk[k] * t.x;
+          v[i + 1] += mk[k] * t.y;
+          v[i + 2] += mk[k] * t.z;
+          v[i + 3] += mk[k] * t.w;
         }
       }
       if (mine) {
-        const size_t nqb = static_cast<size_t>(p.batch) * p.n_q_heads;
-        p.init[nqb * D + rowi] = m_ref;
-        p.init[nqb * D + nqb + rowi] = l_sum;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(ob + c * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
       }
     }
-    tc_fence_before();
+    if (mine) {
+      const size_t nqb = static_cast<size_t>(p.batch) * p.n_q_heads;
+      p.init[nqb * D + rowi] = m_all;
+      p.init[nqb * D + nqb + rowi] = l_all;
+    }
   }
-  __syncthreads();
+  tc_fence_before();
+  cluster_sync();  // the other CTAs' shared memory stays in place until rank 0 has read it
   if (warp == 5) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols));

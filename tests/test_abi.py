@@ -127,3 +127,17 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         pkv.paged_attention_decode(t, cache, cache, torch.zeros(1, 1, dtype=torch.int32),
                                    torch.ones(1, dtype=torch.int32), 0.1, out=t.clone())
+
+
+def test_cascade_options_are_checked_on_the_host(lib):
+    ptr = ctypes.c_void_p(16)  # never dereferenced: the options are rejected first
+    for fields in ({"prefix_splits": 5}, {"prefix_splits": -1}, {"prefix_kernel": 3}):
+        opts = pkv._CascadeOptions(**fields)
+        st = lib.paged_attention_decode_cascade_ex(ptr, ptr, ptr, 1, ptr, 4, ptr, ptr, ptr, 4, ptr, 2, 8, 0.125,
+                                                   8, 2, 128, 16, ptr, 2, None, 0, None, ctypes.byref(opts))
+        assert st == INVALID, fields
+    opts = pkv._CascadeOptions()
+    opts.reserved[3] = 1
+    st = lib.paged_attention_decode_cascade_ex(ptr, ptr, ptr, 1, ptr, 4, ptr, ptr, ptr, 4, ptr, 2, 8, 0.125,
+                                               8, 2, 128, 16, ptr, 2, None, 0, None, ctypes.byref(opts))
+    assert st == INVALID

@@ -12,7 +12,7 @@ from tests.gpu_helpers import assert_close, bits, sample_rows
 pytestmark = pytest.mark.gpu
 
 
-def run_cascade(w, cv=None, check_errors=True, workspace=None):
+def run_cascade(w, cv=None, check_errors=True, workspace=None, **opts):
     dev = torch.device("cuda")
     kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
     if w.appended:
@@ -20,7 +20,7 @@ def run_cascade(w, cv=None, check_errors=True, workspace=None):
     cv = cv or W.cascade_view(w)
     out = pkv.paged_attention_decode_cascade(
         w.q.to(dev), kc, vc, cv.prefix_block_tables.to(dev), cv.prefix_lens.to(dev), cv.seq_group.to(dev),
-        cv.block_tables.to(dev), cv.context_lens.to(dev), w.scale, workspace=workspace)
+        cv.block_tables.to(dev), cv.context_lens.to(dev), w.scale, workspace=workspace, **opts)
     torch.cuda.synchronize()
     if check_errors:
         assert pkv.pkv_get_device_error() == 0
@@ -117,3 +117,35 @@ def test_cascade_fp32_is_unsupported():
     with pytest.raises(pkv.PagedKVError) as e:
         run_cascade(w)
     assert e.value.status == 2
+
+
+# Prefix lengths that leave some cluster ranks with no stage (16 tokens: one
+# 64-key stage), end in a partial stage (272, 336) or split unevenly (592:
+# ten stages over 3 or 4 ranks), with a ragged last row tile.
+SPLIT_PREFIXES = [16, 272, 336, 592]
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 4])
+@pytest.mark.parametrize("prefix", SPLIT_PREFIXES)
+def test_cascade_prefix_split_across_cluster(splits, prefix):
+    w = W.shared_prefix(n_seqs=18, prefix=prefix, suffix=(1, 60), seed=50 + prefix)
+    out = run_cascade(w, prefix_splits=splits, prefix_kernel=1)
+    ref, _, _ = oracle.workload_decode(w)
+    assert_close(out, ref, w.dtype, what=f"splits={splits} prefix={prefix}")
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_cascade_both_prefix_kernels(kernel):
+    w = W.best_of_n(prompts=3, n=8, prompt_len=384, gen_len=40, seed=51)
+    out = run_cascade(w, prefix_kernel=kernel)
+    ref, _, _ = oracle.workload_decode(w)
+    assert_close(out, ref, w.dtype, what=f"prefix kernel {kernel}")
+
+
+def test_cascade_split_full_size_sampled():
+    w = W.shared_prefix(seed=1)
+    rows = sample_rows(w, 96)
+    for splits in (2, 4):
+        out = run_cascade(w, prefix_splits=splits)
+        ref, _, _ = oracle.workload_decode(w, rows=rows)
+        assert_close(out, ref, w.dtype, rows=rows, what=f"shared_prefix_70b splits={splits}")
