@@ -139,6 +139,24 @@ pkv_status encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dt, i
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// A block's whole K or V tile of one kv head as one TMA box (head dim 128,
+// 16-bit): dims {64 dims, 16 tokens, 2 halves of the head dim, kv head,
+// block}, box {64, 16, 2, 1, 1}, landing as [half][token][128 B] with the
+// 128-byte swizzle.
+pkv_status encode_cache_map_tile(CUtensorMap* map, const void* cache, pkv_dtype dt, int num_blocks, int n_kv) {
+  const CUtensorMapDataType ty = dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint64_t row = 128 * 2;
+  const cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(kBlockTokens), 2, static_cast<cuuint64_t>(n_kv),
+                              static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t strides[4] = {row, 128, row * kBlockTokens, row * kBlockTokens * n_kv};
+  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(kBlockTokens), 2, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = g_encode(map, ty, 5, const_cast<void*>(cache), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
 // The decode kernel is launched cooperatively: its CTAs (at most one per SM)
 // are guaranteed to be co-resident, which its grid-wide barrier needs.
 template <int DT, int D, int GPAD, bool kI8 = false, bool kMQ = false>
@@ -254,7 +272,7 @@ pkv_status launch_prefix(const CUtensorMap& mk, const CUtensorMap& mv, const Pre
 // The tensor-memory prefix kernel (head dim 128): 128-row tiles, 192 KiB of
 // operands plus barriers and the member list.
 size_t prefix_tc_smem(int batch) {
-  return 1024 + kTcSmemBytes + (2 * kTcStages + 7) * sizeof(uint64_t) + 16 + static_cast<size_t>(batch) * 4;
+  return 1024 + kTcSmemBytes + kTcBarBytes + kTcExchBytes + static_cast<size_t>(batch) * 4;
 }
 
 // Launch configuration of the tensor-memory prefix kernel: one cluster of
@@ -808,8 +826,12 @@ pkv_status paged_attention_decode_cascade_ex(const void* q, const void* k_cache,
   const bool tc = tc_fits && opt.prefix_kernel != 2;
   if (!tc && smem + 256 > static_cast<size_t>(di.smem_optin)) st = st == PKV_OK ? PKV_ERR_UNSUPPORTED : st;
   if (st == PKV_OK && tc) {
-    st = dtype == PKV_F16 ? launch_prefix_tc<kF16>(mk, mv, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s)
-                          : launch_prefix_tc<kBF16>(mk, mv, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s);
+    CUtensorMap mv_tile;
+    st = encode_cache_map_tile(&mv_tile, v_cache, dtype, num_blocks, n_kv_heads);
+    if (st == PKV_OK)
+      st = dtype == PKV_F16
+               ? launch_prefix_tc<kF16>(mk, mv_tile, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s)
+               : launch_prefix_tc<kBF16>(mk, mv_tile, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s);
   } else if (st == PKV_OK) {
     if (dtype == PKV_F16)
       st = head_dim == 64 ? launch_prefix<kF16, 64>(mk, mv, pp, n_kv_heads, smem, s)

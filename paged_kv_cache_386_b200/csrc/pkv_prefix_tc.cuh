@@ -11,33 +11,37 @@
 //
 // A cluster of 1-4 CTAs per 128-row tile of one (group, kv head), head dim
 // 128; CTA k of the cluster takes the k-th share of the prefix stages, so that
-// a few tiles still fill the SMs.  After its last stage each CTA of rank > 0
-// leaves its partial (O, m, l) in its own shared memory; rank 0 reads them
-// through distributed shared memory, merges them with its own (each term
-// scaled by 2^(m_k - max m)) and writes the row's state.  192 threads:
-//   warps 0-3  softmax: thread r owns row r (tensor-memory lane r);
-//   warp 4     producer: TMA loads of 64 prefix tokens (4 blocks) of K and V
-//              per stage into a 4-stage ring;
-//   warp 5     allocates the tensor memory; its lane 0 issues every MMA.
-// Per stage s:  S_s = Q K_s^T (M 128, N 64 keys, K 128) into one of two S
+// a few tiles still fill the SMs.  After its last stage each CTA leaves the
+// partial (O, m, l) of the rows it does not own in its own shared memory; the
+// owner of a row group (rank lg * size / 4) reads the other shares through
+// distributed shared memory, weights each by 2^(m_k - max m), and writes the
+// row's state with coalesced stores.  320 threads:
+//   warps 0-7  softmax: warps lg and lg + 4 share rows 32 lg .. 32 lg + 31
+//              (tensor-memory lanes), each taking 32 of the 64 scores of a
+//              stage; they exchange row maxima through shared memory;
+//   warp 8     producer: TMA loads of 64 prefix tokens (4 blocks) of K and V
+//              per stage into a 4-stage ring, from the kernel's start on;
+//   warp 9     allocates the tensor memory; its lane 0 issues every MMA.
+// Per stage s:  S_s = Q K_s^T (M 128, N 64 keys, K 128) into one of three S
 // buffers in tensor memory; the softmax warps read their S row, turn it into
 // probabilities P_s (16-bit, shared memory) and the MMA thread accumulates
-// O += P_s V_s (M 128, N 128 dims, K 64 keys) in tensor memory.  S of the
-// next stage is issued before O += P V of this one, so that the softmax of a
-// stage overlaps the tensor cores; P is double-buffered, so that the softmax
-// of stage s + 1 does not wait for O += P V of stage s.  The running maximum
-// is only moved (and O,
-// l rescaled) when a row's maximum grows by more than 2^8, so that O rarely
-// makes a round trip through registers; P stays below 2^8.
+// O += P_s V_s (M 128, N 128 dims, K 64 keys) in tensor memory.  S runs up to
+// two stages ahead of the softmax, so that the softmax of a stage never waits
+// for the tensor cores; P is double-buffered, so that the softmax of stage
+// s + 1 does not wait for O += P V of stage s.  The running maximum
+// is only moved (and O, l rescaled) when a row's maximum grows by more than
+// 2^8, so that O rarely makes a round trip through registers; P stays below
+// 2^8.
 //
 // Shared-memory operands use the 128-byte swizzle (16-byte chunk c of a
 // 128-byte row r at chunk c ^ (r % 8)), in 1 KiB atoms of 8 rows:
 //   Q     K-major A operand:  [64-dim block][128 rows][128 B];
 //   P     K-major A operand:  [128 rows][128 B] (64 keys);
 //   K     K-major B operand:  [64-dim block][64 tokens][128 B];
-//   V     MN-major B operand: [64-dim block][64 tokens][128 B].
-// The K and V blocks land there from the decode kernel's tensor maps (one
-// 16-row x 128-byte box per block and 64-dim block).
+//   V     MN-major B operand: [block][64-dim half][16 tokens][128 B].
+// K lands from the decode kernel's tensor map (one 16-row x 128-byte box per
+// block and 64-dim half), V from a 5-D map over the same cache whose box is a
+// block's whole tile.
 #pragma once
 
 #include "pkv_prefix.cuh"
@@ -47,7 +51,10 @@ namespace pkv {
 constexpr int kTcRows = 128;                  // query rows per CTA (M)
 constexpr int kTcKeys = 64;                   // prefix tokens per stage (N of S, K of P V)
 constexpr int kTcBlocks = kTcKeys / kBlockTokens;
-constexpr int kTcThreads = 192;
+constexpr int kTcSoftmaxWarps = 8;           // two per row group of 32: each takes 32 of the 64 scores
+constexpr int kTcProducerWarp = 8;
+constexpr int kTcMmaWarp = 9;
+constexpr int kTcThreads = 320;
 constexpr int kTcQBytes = kTcRows * 128 * 2;        // Q: 128 rows x 128 dims, 32 KiB
 constexpr int kTcQHalf = kTcQBytes / 2;             // one 64-dim block of Q: 16 KiB
 constexpr int kTcPBytes = kTcRows * kTcKeys * 2;    // P: 128 rows x 64 keys, 16 KiB
@@ -56,13 +63,67 @@ constexpr int kTcKVHalf = kTcKVBytes / 2;           // one 64-dim block: 8 KiB
 constexpr int kTcStageBytes = 2 * kTcKVBytes;       // K and V of one stage
 constexpr int kTcStages = 4;
 constexpr int kTcSmemBytes = kTcQBytes + 2 * kTcPBytes + kTcStages * kTcStageBytes;  // 192 KiB
-constexpr uint32_t kTcTmemCols = 256;  // S0 [0,64), S1 [64,128), O [128,256)
-constexpr uint32_t kTcOCol = 2 * kTcKeys;
+constexpr int kTcSBufs = 3;             // S buffers in tensor memory: S is issued two stages ahead
+constexpr uint32_t kTcTmemCols = 512;   // S0 [0,64), S1 [64,128), S2 [128,192), O [256,384)
+constexpr uint32_t kTcOCol = 256;
 constexpr int kTcMaxSplit = 4;          // CTAs per cluster (prefix shares per tile)
 constexpr int kTcPartStride = 128 + 4;  // floats per row of a partial O in shared memory (float4 accesses
                                         // of 8 consecutive rows fall in distinct bank groups)
 static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcStages * kTcStageBytes,
               "a partial state fits in the drained K/V ring");
+static_assert(kTcRows * 128 * 4 <= kTcQBytes + 2 * kTcPBytes, "the output rows fit where Q and P were");
+// Barriers, tensor-memory slot and abort flag, then the softmax exchange
+// arrays (pair maxima [2][2][128], pair sums [2][128], destination rows [128]).
+constexpr int kTcBarBytes = (2 * kTcStages + 2 * kTcSBufs + 4) * 8 + 16;
+constexpr int kTcExchBytes = (4 * kTcRows + 2 * kTcRows + kTcRows) * 4;
+
+// 5-D tiled TMA load global -> this CTA's shared memory (no multicast): the
+// V tile of one block and kv head in one request, box {64 dims, 16 tokens,
+// 2 halves of the head dim} landing as [half][token][128 B].
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+
+// Softmax arithmetic with fewer issue slots: two fp32 lanes per packed FMA /
+// add (sm_100), two new values per three-input max, and the hardware base-2
+// exponential with flush to zero (the probabilities become 16-bit anyway).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -90,12 +151,13 @@ __device__ __forceinline__ float ld_cluster(uint32_t addr) {
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
+// Ordered after the cluster barrier by that barrier's memory clobber; no
+// clobber here, so that a batch of them is in flight at once.
 __device__ __forceinline__ float4 ld_cluster4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
+               : "r"(addr));
   return v;
 }
 
@@ -181,13 +243,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kTcStages * kTcStageBytes);
   uint64_t* kv_full = bars;                // [kTcStages]
   uint64_t* kv_empty = bars + kTcStages;   // [kTcStages]
-  uint64_t* s_full = bars + 2 * kTcStages; // [2]
-  uint64_t* s_free = s_full + 2;           // [2]
-  uint64_t* p_full = s_full + 4;
-  uint64_t* o_done = s_full + 5;           // [2]: P V of stages with that parity (P buffer free, O updated)
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(s_full + 7);
+  uint64_t* s_full = bars + 2 * kTcStages; // [kTcSBufs]
+  uint64_t* s_free = s_full + kTcSBufs;    // [kTcSBufs]
+  uint64_t* p_full = s_free + kTcSBufs;    // [2]: P of stages with that parity written
+  uint64_t* o_done = p_full + 2;           // [2]: P V of stages with that parity (P buffer free, O updated)
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(o_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* members = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 2));  // [batch]
+  float* red_max = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kTcBarBytes);  // [2][2][128]
+  float* red_l = red_max + 4 * kTcRows;                                                     // [2][128]
+  int* row_dst = reinterpret_cast<int*>(red_l + 2 * kTcRows);                               // [128]
+  int* members = row_dst + kTcRows;                                                         // [batch]
   __shared__ int warp_counts[kTcThreads / 32];
   __shared__ int n_members;
 
@@ -195,6 +260,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t crank = cluster_rank(), csize = cluster_size();
   const int tile = blockIdx.x / csize, kvh = blockIdx.y, grp = blockIdx.z;
   const int G = p.group;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < kTcSBufs; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kTcSoftmaxWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], kTcSoftmaxWarps);
+      mbar_init(&o_done[i], 1);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  int plen = __ldg(p.prefix_lens + grp);
+  const bool plen_bad = plen < 0 || plen > p.max_prefix_blocks * kBlockTokens || (plen % kBlockTokens) != 0;
+  if (plen_bad) plen = plen < 0 ? 0 : min(plen - plen % kBlockTokens, p.max_prefix_blocks * kBlockTokens);
+  // This CTA's share of the prefix: stages [s_begin, s_begin + n_stages).
+  const int n_total = (plen + kTcKeys - 1) / kTcKeys;
+  const int s_begin = n_total * static_cast<int>(crank) / static_cast<int>(csize);
+  const int n_stages = n_total * static_cast<int>(crank + 1) / static_cast<int>(csize) - s_begin;
+  // The producer reads the block table a window of 32 entries (8 stages) at
+  // a time, one window ahead, lane l holding entry l of the window; the first
+  // two windows are in flight during the member scan.  Entries past the
+  // prefix read as entry 0 (finite values whose probabilities are 0).
+  const int32_t* tab = p.prefix_tables + static_cast<size_t>(grp) * p.max_prefix_blocks;
+  const int n_prefix_blocks = plen / kBlockTokens;
+  auto tab_entry = [&](int j) { return __ldg(tab + (j < n_prefix_blocks ? j : 0)); };
+  int tab_cur = 0, tab_next = 0;
+  if (warp == kTcProducerWarp) {
+    tab_cur = tab_entry(s_begin * kTcBlocks + lane);
+    tab_next = tab_entry(s_begin * kTcBlocks + 32 + lane);
+  }
 
   // Members of this group, in increasing sequence order (block-wide compaction).
   {
@@ -220,91 +321,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   const int R = n_members * G;
   const int row0 = tile * kTcRows;
-  if (row0 >= R) return;  // uniform over the cluster: no barrier or tensor memory is in use yet
+  if (row0 >= R) return;  // uniform over the cluster: no copy, MMA or tensor memory is in use yet
 
-  int plen = __ldg(p.prefix_lens + grp);
-  if (plen < 0 || plen > p.max_prefix_blocks * kBlockTokens || (plen % kBlockTokens) != 0) {
-    flag_error(PKV_DEVERR_CONTEXT);
-    plen = plen < 0 ? 0 : min(plen - plen % kBlockTokens, p.max_prefix_blocks * kBlockTokens);
-  }
-  // This CTA's share of the prefix: stages [s_begin, s_begin + n_stages).
-  const int n_total = (plen + kTcKeys - 1) / kTcKeys;
-  const int s_begin = n_total * static_cast<int>(crank) / static_cast<int>(csize);
-  const int n_stages = n_total * static_cast<int>(crank + 1) / static_cast<int>(csize) - s_begin;
+  if (plen_bad && threadIdx.x == 0) flag_error(PKV_DEVERR_CONTEXT);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kTcStages; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-    }
-    mbar_init(p_full, 4);
-    mbar_init(&o_done[0], 1);
-    mbar_init(&o_done[1], 1);
-    *abort_flag = 0;
-    mbar_fence_init();
-  }
-  if (warp == 5) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(const_cast<uint32_t*>(tmem_slot))),
-                 "r"(kTcTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  // Q rows into the swizzled A operand (zero rows past R).
-  if (warp < 4) {
-    const int r = threadIdx.x;
-    const int row = row0 + r;
-    const uint4* src = nullptr;
-    if (row < R) {
-      const int b = members[row / G], h = kvh * G + row % G;
-      src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
-                                           (static_cast<size_t>(b) * p.n_q_heads + h) * D * 2);
-    }
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint4 v = src ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(q_s + tc_chunk(r, c)) = v;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);  // softmax warps' lanes
-  float* part_o = reinterpret_cast<float*>(ring);  // a rank > 0 CTA's partial O: [128 rows][kTcPartStride]
-  float* part_ml = part_o + kTcRows * kTcPartStride;  // its m [128], then l [128]
-  float m_ref = -INFINITY, l_sum = 0.f;  // the softmax thread's row state
-  bool row_ok = true;
+  // Softmax-warp geometry: row group lg (tensor-memory lanes 32 lg ..), half hf of the scores.
+  const int lg = warp & 3, hf = (warp >> 2) & 1;
+  const int r = lg * 32 + lane;
+  const uint32_t owner = static_cast<uint32_t>(lg) * csize / 4;  // cluster rank that writes these rows
+  float m_ref = -INFINITY, l_row = 0.f;                           // the softmax thread's row state
+  bool ok = true;
+  uint32_t tmem = 0;
 
-  if (warp == 4) {
-    // ---------------- producer: 16 TMA requests per stage, one per lane ----------------
-    const int32_t* tab = p.prefix_tables + static_cast<size_t>(grp) * p.max_prefix_blocks;
+  if (warp == kTcProducerWarp) {
+    // ---------------- producer: 12 TMA requests per stage ----------------
+    // Lanes 0-7: K, block lane / 2, dim half lane % 2 (one 16-token x 64-dim
+    // box each); lanes 8-11: V of block lane - 8 (one 16-token x 128-dim box).
+    // Starts at once: the copies of the first stages overlap the Q load.
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
-    const int blk = (lane >> 2) & 3, isv = (lane >> 1) & 1, y = lane & 1;
-    const bool active = lane < 4 * kTcBlocks;
+    const bool is_k = lane < 2 * kTcBlocks, is_v = !is_k && lane < 3 * kTcBlocks;
+    const int blk = is_k ? lane >> 1 : is_v ? lane - 2 * kTcBlocks : 0, y = lane & 1;
     int issued = 0;
     for (int s = 0; s < n_stages; ++s) {
       const int slot = s % kTcStages;
-      if (!mbar_wait_bounded(&kv_empty[slot], ((s / kTcStages) & 1) ^ 1u, abort_flag, kWaitLimitNs)) break;
-      const int j = (s_begin + s) * kTcBlocks + blk;
-      // Blocks past the prefix reload block 0 of the prefix (finite values;
-      // their probabilities are 0).
-      int phys = __ldg(tab + (j * kBlockTokens < plen ? j : 0));
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait_bounded(&kv_empty[slot], ((s / kTcStages) & 1) ^ 1u, abort_flag, kWaitLimitNs)))
+        break;  // warp-uniform, so that the shuffles below stay converged
+      if (s > 0 && (s & 7) == 0) {
+        tab_cur = tab_next;
+        tab_next = tab_entry((s_begin + s + 8) * kTcBlocks + lane);
+      }
+      int phys = __shfl_sync(0xffffffffu, tab_cur, (s & 7) * kTcBlocks + blk);
       if (phys < 0 || phys >= p.num_blocks) {
         flag_error(PKV_DEVERR_BLOCK_ID);
         phys = 0;
       }
       if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], kTcStageBytes);
       __syncwarp();
-      uint8_t* dst = ring + slot * kTcStageBytes + isv * kTcKVBytes + y * kTcKVHalf + blk * (kBlockTokens * 128);
-      if (active) tma_load_4d(dst, isv ? &tm_v : &tm_k, &kv_full[slot], y * X, 0, kvh, phys);
+      uint8_t* stage = ring + slot * kTcStageBytes;
+      if (is_k) tma_load_4d(stage + y * kTcKVHalf + blk * (kBlockTokens * 128), &tm_k, &kv_full[slot], y * X, 0, kvh,
+                            phys);
+      if (is_v) tma_load_5d(stage + kTcKVBytes + blk * (2 * kBlockTokens * 128), &tm_v, &kv_full[slot], 0, 0, 0, kvh,
+                            phys);
       ++issued;
     }
     // Do not leave while copies may still be landing.
@@ -319,241 +380,343 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
-    // ---------------- MMA issue (one thread) ----------------
-    if (lane == 0 && n_stages > 0) {
-      constexpr uint32_t kIdS = tc_idesc<kBf16>(false, kTcKeys), kIdPV = tc_idesc<kBf16>(true, D);
-      const uint32_t qa = smem_u32(q_s), pa = smem_u32(p_s), ra = smem_u32(ring);
-      auto issue_s = [&](int s) {
-        const uint32_t ka = ra + (s % kTcStages) * kTcStageBytes;
-        const uint32_t d = tmem + (s & 1) * kTcKeys;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          tc_mma(d, smem_desc_sw128(qa + (kk >> 2) * kTcQHalf + (kk & 3) * 32, 16, 1024),
-                 smem_desc_sw128(ka + (kk >> 2) * kTcKVHalf + (kk & 3) * 32, 16, 1024), kIdS, kk > 0);
-        }
-        tc_commit(&s_full[s & 1]);
-      };
-      bool ok = mbar_wait_bounded(&kv_full[0], 0, abort_flag, kWaitLimitNs);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-      }
-      for (int s = 0; ok && s < n_stages; ++s) {
-        if (s + 1 < n_stages) {
-          ok = mbar_wait_bounded(&kv_full[(s + 1) % kTcStages], ((s + 1) / kTcStages) & 1, abort_flag, kWaitLimitNs);
-          // The S buffer of stage s + 1 was last read by the softmax of stage s - 1.
-          if (ok && s >= 1) ok = mbar_wait_bounded(&s_free[(s + 1) & 1], ((s - 1) >> 1) & 1, abort_flag, kWaitLimitNs);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(s + 1);
-        }
-        if (!mbar_wait_bounded(p_full, s & 1, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t va = ra + (s % kTcStages) * kTcStageBytes + kTcKVBytes;
-        const uint32_t pb = pa + (s & 1) * kTcPBytes;
-#pragma unroll
-        for (int kt = 0; kt < kTcKeys / 16; ++kt) {
-          tc_mma(tmem + kTcOCol, smem_desc_sw128(pb + kt * 32, 16, 1024),
-                 smem_desc_sw128(va + kt * 16 * 128, kTcKVHalf, 1024), kIdPV, s > 0 || kt > 0);
-        }
-        tc_commit(&o_done[s & 1]);
-        tc_commit(&kv_empty[s % kTcStages]);
-      }
-      // Before the tensor memory is freed, every MMA issued must have completed.
-      if (!ok) mbar_wait_bounded(&o_done[(n_stages - 1) & 1], ((n_stages - 1) >> 1) & 1, abort_flag, kWaitLimitNs);
-    }
   } else {
-    // ---------------- softmax: thread r owns row r ----------------
-    const int r = threadIdx.x;
-    // Every tensor-memory access below is warp-converged (.sync.aligned):
-    // waits and decisions are made warp-uniform first.
-    bool ok = true;
-    for (int s = 0; s < n_stages; ++s) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[s & 1], (s >> 1) & 1, abort_flag, kWaitLimitNs));
-      if (!ok) break;
-      tc_fence_after();
-      float x[kTcKeys];
-#pragma unroll
-      for (int c = 0; c < kTcKeys / 32; ++c) {
-        float v[32];
-        tmem_ld32(lane_base + (s & 1) * kTcKeys + c * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = v[i];
+    if (warp == kTcMmaWarp) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(const_cast<uint32_t*>(tmem_slot))),
+                   "r"(kTcTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    } else {
+      // Q rows into the swizzled A operand (zero rows past R): thread t copies
+      // eight 16-byte chunks of row t % 128.
+      // A negative scale is taken as |scale| on -Q (exact), so that the
+      // softmax can take its maximum over the raw scores.
+      const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
+      const int qr = threadIdx.x & (kTcRows - 1), c0 = (threadIdx.x >> 7) * 8;
+      const int row = row0 + qr;
+      const uint4* src = nullptr;
+      if (row < R) {
+        const int b = members[row / G], h = kvh * G + row % G;
+        src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
+                                             (static_cast<size_t>(b) * p.n_q_heads + h) * D * 2);
       }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[s & 1]);
-
-      const int live = min(kTcKeys, plen - (s_begin + s) * kTcKeys);
-      float mx8[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) mx8[j] = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < kTcKeys; ++i) {
-        x[i] = i < live ? x[i] * p.scale_log2 : -INFINITY;
-        mx8[i & 7] = fmaxf(mx8[i & 7], x[i]);  // eight independent chains
+      for (int c = c0; c < c0 + 8; ++c) {
+        uint4 v = src ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        v.x ^= flip;
+        v.y ^= flip;
+        v.z ^= flip;
+        v.w ^= flip;
+        *reinterpret_cast<uint4*>(q_s + tc_chunk(qr, c)) = v;
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // P buffer s % 2 is free once P V of stage s - 2 is done.
-      if (s >= 2) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait_bounded(&o_done[s & 1], ((s - 2) >> 1) & 1, abort_flag, kWaitLimitNs));
-        if (!ok) break;
-        tc_fence_after();
-      }
-      // Move the reference maximum only when it grows by more than 2^8 (so
-      // that O rarely makes the round trip); when any row of the warp moves,
-      // the whole warp takes the round trip, with factor 1 for the others.
-      // O is stable once P V of stage s - 1 is done.
-      const bool move = mx > m_ref + 8.f;
-      if (s > 0 && __any_sync(0xffffffffu, move)) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(s - 1) & 1], ((s - 1) >> 1) & 1, abort_flag,
-                                                       kWaitLimitNs));
-        if (!ok) break;
-        tc_fence_after();
-        const float alpha = move ? exp2f(m_ref - mx) : 1.f;
-        l_sum *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(lane_base + kTcOCol + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st32(lane_base + kTcOCol + c * 32, v);
-        }
-        tmem_wait_st();
-      }
-      if (move) m_ref = mx;
-      float sum8[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
-#pragma unroll
-      for (int c = 0; c < kTcKeys / 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float a = exp2f(x[8 * c + 2 * k] - m_ref), b = exp2f(x[8 * c + 2 * k + 1] - m_ref);
-          sum8[2 * k] += a;
-          sum8[2 * k + 1] += b;
-          w[k] = pack2<kBf16>(a, b);
-        }
-        *reinterpret_cast<uint4*>(p_s + (s & 1) * kTcPBytes + tc_chunk(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      l_sum += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && n_stages > 0)
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(n_stages - 1) & 1], ((n_stages - 1) >> 1) & 1,
-                                                      abort_flag, kWaitLimitNs));
+    tc_fence_before();
+    named_bar_sync(1, (kTcSoftmaxWarps + 1) * 32);  // softmax warps and the MMA warp
     tc_fence_after();
-    row_ok = ok;
-    if (crank > 0) {
-      // Partial state into the drained ring (every copy into it has been
-      // consumed by an MMA that has completed); l = NaN marks a failed row.
+    tmem = *tmem_slot;
+
+    if (warp == kTcMmaWarp) {
+      // ---------------- MMA issue (one thread) ----------------
+      // S of a stage is issued as soon as its K has landed and its S buffer
+      // is free (up to two stages ahead of the softmax), O += P V as soon as
+      // its P is written; the thread polls both and issues in stage order
+      // within each kind.
+      if (lane == 0 && n_stages > 0) {
+        constexpr uint32_t kIdS = tc_idesc<kBf16>(false, kTcKeys), kIdPV = tc_idesc<kBf16>(true, D);
+        const uint32_t qa = smem_u32(q_s), pa = smem_u32(p_s), ra = smem_u32(ring);
+        int ns = 0, np = 0;  // next stage whose S, whose P V is to be issued
+        uint64_t t0 = global_timer_ns();
+        bool mok = true;
+        while (np < n_stages) {
+          bool progress = false;
+          if (ns < n_stages && mbar_test_wait(&kv_full[ns % kTcStages], (ns / kTcStages) & 1) &&
+              (ns < kTcSBufs || mbar_test_wait(&s_free[ns % kTcSBufs], ((ns - kTcSBufs) / kTcSBufs) & 1))) {
+            tc_fence_after();
+            const uint32_t ka = ra + (ns % kTcStages) * kTcStageBytes;
+            const uint32_t d = tmem + (ns % kTcSBufs) * kTcKeys;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float v[32];
-        if (ok && n_stages > 0) {
-          tmem_ld32(lane_base + kTcOCol + c * 32, v);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              tc_mma(d, smem_desc_sw128(qa + (kk >> 2) * kTcQHalf + (kk & 3) * 32, 16, 1024),
+                     smem_desc_sw128(ka + (kk >> 2) * kTcKVHalf + (kk & 3) * 32, 16, 1024), kIdS, kk > 0);
+            }
+            tc_commit(&s_full[ns % kTcSBufs]);
+            ++ns;
+            progress = true;
+          }
+          if (np < ns && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
+            tc_fence_after();
+            const uint32_t va = ra + (np % kTcStages) * kTcStageBytes + kTcKVBytes;
+            const uint32_t pb = pa + (np & 1) * kTcPBytes;
+#pragma unroll
+            for (int kt = 0; kt < kTcKeys / 16; ++kt) {
+              // V of block kt: [half][16 tokens][128 B], halves 2 KiB apart.
+              tc_mma(tmem + kTcOCol, smem_desc_sw128(pb + kt * 32, 16, 1024),
+                     smem_desc_sw128(va + kt * 2 * kBlockTokens * 128, kBlockTokens * 128, 1024), kIdPV,
+                     np > 0 || kt > 0);
+            }
+            tc_commit(&o_done[np & 1]);
+            tc_commit(&kv_empty[np % kTcStages]);
+            ++np;
+            progress = true;
+          }
+          if (progress) {
+            t0 = global_timer_ns();
+          } else if (*abort_flag) {
+            mok = false;
+            break;
+          } else if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            flag_error(kDevErrTimeout);
+            mok = false;
+            break;
+          }
+        }
+        // Before the tensor memory is freed, every MMA issued must have completed.
+        if (!mok && np > 0)
+          mbar_wait_bounded(&o_done[(np - 1) & 1], ((np - 1) >> 1) & 1, abort_flag, kWaitLimitNs);
+      }
+    } else {
+      // ---------------- softmax: warps (lg, hf) share rows 32 lg .. 32 lg + 31 ----------------
+      // Every tensor-memory access is warp-converged (.sync.aligned): waits
+      // and decisions are made warp-uniform first.  The pair barrier is
+      // reached on every stage, also after a failed wait, so that the two
+      // warps of a pair never wait for each other in vain.
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(lg * 32) << 16);
+      const float sc = fabsf(p.scale_log2);
+      float l_half = 0.f;
+      for (int s = 0; s < n_stages; ++s) {
+        const int sb = s % kTcSBufs;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[sb], (s / kTcSBufs) & 1, abort_flag,
+                                                                kWaitLimitNs));
+        float x[32];
+        if (ok) {
+          tc_fence_after();
+          tmem_ld32(lane_base + sb * kTcKeys + hf * 32, x);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          for (int i = 0; i < 32; ++i) x[i] = 0.f;
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[sb]);
+
+        // Scores past the prefix (only in the last stage) are masked.
+        const int live = min(kTcKeys, plen - (s_begin + s) * kTcKeys) - hf * 32;
+        if (live < 32) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(part_o + r * kTcPartStride + c * 32 + i) =
-              make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          for (int i = 0; i < 32; ++i) x[i] = i < live ? x[i] : -INFINITY;
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], x[i], x[i + 1]);
+        float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        mx = live > 0 ? mx * sc : -INFINITY;  // the maximum of the scaled scores (sc >= 0)
+        red_max[((s & 1) * 2 + hf) * kTcRows + r] = mx;
+        named_bar_sync(2 + lg, 64);
+        mx = fmaxf(mx, red_max[((s & 1) * 2 + (hf ^ 1)) * kTcRows + r]);  // the row's maximum, same in both
+        // P buffer s % 2 is free once P V of stage s - 2 is done.
+        if (ok && s >= 2) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_bounded(&o_done[s & 1], ((s - 2) >> 1) & 1, abort_flag, kWaitLimitNs));
+          if (ok) tc_fence_after();
+        }
+        // Move the reference maximum only when it grows by more than 2^8 (so
+        // that O rarely makes the round trip); when any row of the warp
+        // moves, the warp takes the round trip for its 64 columns of O, with
+        // factor 1 for the rows that stay.  O is stable once P V of stage
+        // s - 1 is done.  Both warps of a pair decide alike.
+        const bool move = mx > m_ref + 8.f;
+        if (ok && s > 0 && __any_sync(0xffffffffu, move)) {
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(s - 1) & 1], ((s - 1) >> 1) & 1, abort_flag,
+                                                         kWaitLimitNs));
+          if (ok) {
+            tc_fence_after();
+            const float alpha = move ? exp2f(m_ref - mx) : 1.f;
+            l_half *= alpha;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              float v[32];
+              tmem_ld32(lane_base + kTcOCol + hf * 64 + c * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] *= alpha;
+              tmem_st32(lane_base + kTcOCol + hf * 64 + c * 32, v);
+            }
+            tmem_wait_st();
+          }
+        }
+        if (move) m_ref = mx;
+        {
+          const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m_ref, -m_ref);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) f2_unpack(f2_fma(f2_pack(x[i], x[i + 1]), sc2, nm2), x[i], x[i + 1]);
+        }
+        if (live < 32) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = i < live ? x[i] : -INFINITY;
+        }
+        uint64_t sum2[2] = {0ull, 0ull};
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float a = ex2_ftz(x[8 * cc + 2 * k]), b = ex2_ftz(x[8 * cc + 2 * k + 1]);
+            sum2[k & 1] = f2_add(sum2[k & 1], f2_pack(a, b));
+            w[k] = pack2<kBf16>(a, b);
+          }
+          *reinterpret_cast<uint4*>(p_s + (s & 1) * kTcPBytes + tc_chunk(r, hf * 4 + cc)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(sum2[0], a0, a1);
+          f2_unpack(sum2[1], b0, b1);
+          l_half += (a0 + a1) + (b0 + b1);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[s & 1]);
       }
-      part_ml[r] = m_ref;
-      part_ml[kTcRows + r] = ok ? l_sum : __int_as_float(0x7fc00000);
+      if (ok && n_stages > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(n_stages - 1) & 1], ((n_stages - 1) >> 1) & 1,
+                                                        abort_flag, kWaitLimitNs));
+      tc_fence_after();
+      // The row's sum over both halves; NaN marks a row whose pipeline failed.
+      red_l[hf * kTcRows + r] = ok ? l_half : __int_as_float(0x7fc00000);
+      named_bar_sync(2 + lg, 64);
+      l_row = red_l[hf * kTcRows + r] + red_l[(hf ^ 1) * kTcRows + r];
+      if (owner != crank) {
+        // Partial state for the owner of these rows, in the drained ring
+        // (every copy into it has been consumed by an MMA that has completed).
+        float* part_o = reinterpret_cast<float*>(ring);  // [128 rows][kTcPartStride]
+        float* part_ml = part_o + kTcRows * kTcPartStride;  // m [128], l [128]
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          if (ok && n_stages > 0) {
+            tmem_ld32(lane_base + kTcOCol + hf * 64 + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(part_o + r * kTcPartStride + hf * 64 + c * 32 + i) =
+                make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+        if (hf == 0) {
+          part_ml[r] = m_ref;
+          part_ml[kTcRows + r] = l_row;
+        }
+      }
     }
   }
   tc_fence_before();
   cluster_sync();  // partial states written
   tc_fence_after();
-  if (warp < 4 && crank == 0) {
-    // The row's state: O (unnormalised), m, l, merged over the cluster.
-    const int r = threadIdx.x;
-    const int row = row0 + r;
+  if (warp < kTcSoftmaxWarps && owner == crank) {
+    // The row's state, merged over the cluster: O (unnormalised), m, l.
+    const uint32_t part_o_addr = smem_u32(ring);
+    const uint32_t part_ml_addr = part_o_addr + kTcRows * kTcPartStride * 4;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(lg * 32) << 16);
     float m_all = m_ref;
-    float mk[kTcMaxSplit], lk[kTcMaxSplit];
-    bool valid = row_ok;
-    const uint32_t ml_addr = smem_u32(part_ml);
+    float wk[kTcMaxSplit], lk[kTcMaxSplit];
+    bool valid = !isnan(l_row);
 #pragma unroll
-    for (int k = 1; k < kTcMaxSplit; ++k) {
-      mk[k] = -INFINITY;
+    for (int k = 0; k < kTcMaxSplit; ++k) {
+      wk[k] = -INFINITY;
       lk[k] = 0.f;
-      if (k < static_cast<int>(csize)) {
-        mk[k] = ld_cluster(cluster_map(ml_addr + r * 4, k));
-        lk[k] = ld_cluster(cluster_map(ml_addr + (kTcRows + r) * 4, k));
+      if (k < static_cast<int>(csize) && k != static_cast<int>(crank)) {
+        wk[k] = ld_cluster(cluster_map(part_ml_addr + r * 4, k));
+        lk[k] = ld_cluster(cluster_map(part_ml_addr + (kTcRows + r) * 4, k));
         valid = valid && !isnan(lk[k]);
-        m_all = fmaxf(m_all, mk[k]);
+        m_all = fmaxf(m_all, wk[k]);
       }
     }
     // Weight of each share: 2^(m_k - max m), 0 for a share with no keys.
-    const float a0 = m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_all);
-    float l_all = a0 * l_sum;
+    const float a_self = m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_all);
+    float l_all = a_self * l_row;
 #pragma unroll
-    for (int k = 1; k < kTcMaxSplit; ++k) {
-      mk[k] = mk[k] == -INFINITY ? 0.f : exp2f(mk[k] - m_all);  // now the weight
-      l_all += mk[k] * lk[k];
+    for (int k = 0; k < kTcMaxSplit; ++k) {
+      wk[k] = wk[k] == -INFINITY ? 0.f : exp2f(wk[k] - m_all);
+      l_all += wk[k] * lk[k];
     }
-    const bool mine = row < R && valid;
-    size_t rowi = 0;
-    if (mine) rowi = static_cast<size_t>(members[row / G]) * p.n_q_heads + kvh * G + row % G;
-    float* ob = p.init + rowi * D;
-    const uint32_t po_addr = smem_u32(part_o) + r * kTcPartStride * 4;
+    const int row = row0 + r;
+    if (hf == 0) {
+      int dst = -1;
+      if (row < R && valid) {
+        dst = members[row / G] * p.n_q_heads + kvh * G + row % G;
+        const size_t nqb = static_cast<size_t>(p.batch) * p.n_q_heads;
+        p.init[nqb * D + dst] = m_all;
+        p.init[nqb * D + nqb + dst] = l_all;
+      }
+      row_dst[r] = dst;
+    }
+    // This warp's 64 columns of its own share of O, weighted, into
+    // [128 rows][512 B] where Q and P were (16-byte chunk c of row r at
+    // c ^ (r % 8)).
+    uint8_t* out_s = q_s;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      float v[32];
-      if (row_ok && n_stages > 0) {
-        tmem_ld32(lane_base + kTcOCol + c * 32, v);  // every lane of the warp
+    for (int c = 0; c < 2; ++c) {
+      float t[32];
+      if (ok && n_stages > 0) {
+        tmem_ld32(lane_base + kTcOCol + hf * 64 + c * 32, t);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        for (int i = 0; i < 32; ++i) t[i] = 0.f;
       }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= a0;
-#pragma unroll
-      for (int k = 1; k < kTcMaxSplit; ++k) {
-        if (k >= static_cast<int>(csize)) break;
-        const uint32_t src = cluster_map(po_addr + c * 128, k);
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float4 t = ld_cluster4(src + i * 4);
-          v[i] += mk[k] * t.x;
-          v[i + 1] += mk[k] * t.y;
-          v[i + 2] += mk[k] * t.z;
-          v[i + 3] += mk[k] * t.w;
-        }
-      }
-      if (mine) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(ob + c * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      for (int i = 0; i < 8; ++i) {
+        const int chunk = (hf * 16 + c * 8 + i) ^ (r & 7);
+        *reinterpret_cast<float4*>(out_s + r * 512 + chunk * 16) =
+            make_float4(t[4 * i] * a_self, t[4 * i + 1] * a_self, t[4 * i + 2] * a_self, t[4 * i + 3] * a_self);
       }
     }
-    if (mine) {
-      const size_t nqb = static_cast<size_t>(p.batch) * p.n_q_heads;
-      p.init[nqb * D + rowi] = m_all;
-      p.init[nqb * D + nqb + rowi] = l_all;
+    named_bar_sync(2 + lg, 64);
+    // Rows out, coalesced: warp (lg, hf) takes rows 32 lg + 16 hf .. + 15,
+    // lane l the 16-byte chunk l of each.  The other shares of the same
+    // chunk are added from their CTAs' shared memory, one 512-byte row per
+    // warp-wide load, with the row's weight from the lane that owns the row.
+    const int rbase = lg * 32 + hf * 16;
+    const int dst_l = row_dst[rbase + (lane & 15)];
+    float4 o[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int rr = rbase + j;
+      o[j] = *reinterpret_cast<const float4*>(out_s + rr * 512 + ((lane ^ (rr & 7)) * 16));
+    }
+#pragma unroll
+    for (int k = 0; k < kTcMaxSplit; ++k) {
+      if (k < static_cast<int>(csize) && k != static_cast<int>(crank)) {
+        const uint32_t src = cluster_map(part_o_addr + (rbase * kTcPartStride + lane * 4) * 4, k);
+        float4 t[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) t[j] = ld_cluster4(src + j * kTcPartStride * 4);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float w = __shfl_sync(0xffffffffu, wk[k], hf * 16 + j);
+          o[j].x += w * t[j].x;
+          o[j].y += w * t[j].y;
+          o[j].z += w * t[j].z;
+          o[j].w += w * t[j].w;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int dst = __shfl_sync(0xffffffffu, dst_l, j);
+      if (dst >= 0) *reinterpret_cast<float4*>(p.init + static_cast<size_t>(dst) * D + lane * 4) = o[j];
     }
   }
   tc_fence_before();
-  cluster_sync();  // the other CTAs' shared memory stays in place until rank 0 has read it
-  if (warp == 5) {
+  cluster_sync();  // the other CTAs' shared memory stays in place until every owner has read it
+  if (warp == kTcMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols));
   }
