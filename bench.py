@@ -394,7 +394,7 @@ def run_ours(args) -> None:
             "tokens_per_s_per_layer": round(tokens_per_s, 1),
             "kv_bytes_per_step": kv_bytes,
             "roofline": {"bound": "hbm",
-                         "kernel": ("paged_attention_decode_cascade (pkv_prefix_kernel + pkv_decode_kernel)"
+                         "kernel": ("paged_attention_decode_cascade (pkv_prefix_tc_kernel + pkv_decode_kernel)"
                                     if args.cascade else
                                     "paged_attention_decode_int8 (pkv_decode_kernel, INT8)" if int8 else
                                     "paged_attention_decode_mq (pkv_decode_kernel, several queries)" if mq

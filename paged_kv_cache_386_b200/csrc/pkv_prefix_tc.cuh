@@ -20,11 +20,11 @@
 //              (tensor-memory lanes), each taking 32 of the 64 scores of a
 //              stage; they exchange row maxima through shared memory;
 //   warp 8     producer: TMA loads of 64 prefix tokens (4 blocks) of K and V
-//              per stage into a 4-stage ring, from the kernel's start on;
+//              per stage into a 6-stage ring, from the kernel's start on;
 //   warp 9     allocates the tensor memory; its lane 0 issues every MMA.
 // Per stage s:  S_s = Q K_s^T (M 128, N 64 keys, K 128) into one of three S
 // buffers in tensor memory; the softmax warps read their S row, turn it into
-// probabilities P_s (16-bit, shared memory) and the MMA thread accumulates
+// probabilities P_s (16-bit, tensor memory) and the MMA thread accumulates
 // O += P_s V_s (M 128, N 128 dims, K 64 keys) in tensor memory.  S runs up to
 // two stages ahead of the softmax, so that the softmax of a stage never waits
 // for the tensor cores; P is double-buffered, so that the softmax of stage
@@ -33,10 +33,9 @@
 // 2^8, so that O rarely makes a round trip through registers; P stays below
 // 2^8.
 //
-// Shared-memory operands use the 128-byte swizzle (16-byte chunk c of a
-// 128-byte row r at chunk c ^ (r % 8)), in 1 KiB atoms of 8 rows:
-//   Q     K-major A operand:  [64-dim block][128 rows][128 B];
-//   P     K-major A operand:  [128 rows][128 B] (64 keys);
+// Q and P, the A operands, live in tensor memory (lane = row).  The B
+// operands are in shared memory with the 128-byte swizzle (16-byte chunk c
+// of a 128-byte row r at chunk c ^ (r % 8)), in 1 KiB atoms of 8 rows:
 //   K     K-major B operand:  [64-dim block][64 tokens][128 B];
 //   V     MN-major B operand: [block][64-dim half][16 tokens][128 B].
 // K lands from the decode kernel's tensor map (one 16-row x 128-byte box per
@@ -55,23 +54,32 @@ constexpr int kTcSoftmaxWarps = 8;           // two per row group of 32: each ta
 constexpr int kTcProducerWarp = 8;
 constexpr int kTcMmaWarp = 9;
 constexpr int kTcThreads = 320;
-constexpr int kTcQBytes = kTcRows * 128 * 2;        // Q: 128 rows x 128 dims, 32 KiB
-constexpr int kTcQHalf = kTcQBytes / 2;             // one 64-dim block of Q: 16 KiB
-constexpr int kTcPBytes = kTcRows * kTcKeys * 2;    // P: 128 rows x 64 keys, 16 KiB
 constexpr int kTcKVBytes = kTcKeys * 128 * 2;       // K (or V) of one stage: 64 tokens x 128 dims, 16 KiB
 constexpr int kTcKVHalf = kTcKVBytes / 2;           // one 64-dim block: 8 KiB
 constexpr int kTcStageBytes = 2 * kTcKVBytes;       // K and V of one stage
-constexpr int kTcStages = 4;
-constexpr int kTcSmemBytes = kTcQBytes + 2 * kTcPBytes + kTcStages * kTcStageBytes;  // 192 KiB
+constexpr int kTcStages = 6;
+constexpr int kTcSmemBytes = kTcStages * kTcStageBytes;  // the K/V ring, 192 KiB
 constexpr int kTcSBufs = 3;             // S buffers in tensor memory: S is issued two stages ahead
-constexpr uint32_t kTcTmemCols = 512;   // S0 [0,64), S1 [64,128), S2 [128,192), O [256,384)
+// Tensor-memory columns (one fp32 or one pair of 16-bit values each):
+// S0 [0,64), S1 [64,128), S2 [128,192), O [256,384), Q [384,448) and two P
+// buffers [448,480), [480,512).  Q and P are the A operands of the two MMAs,
+// read from tensor memory, so that the tensor cores fetch only K and V from
+// shared memory.
+constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTcOCol = 256;
+constexpr uint32_t kTcQCol = 384;
+constexpr uint32_t kTcPCol = 448;
 constexpr int kTcMaxSplit = 4;          // CTAs per cluster (prefix shares per tile)
 constexpr int kTcPartStride = 128 + 4;  // floats per row of a partial O in shared memory (float4 accesses
                                         // of 8 consecutive rows fall in distinct bank groups)
 static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcStages * kTcStageBytes,
               "a partial state fits in the drained K/V ring");
-static_assert(kTcRows * 128 * 4 <= kTcQBytes + 2 * kTcPBytes, "the output rows fit where Q and P were");
+// After the last stage the drained ring holds a CTA's partial state for the
+// rows it does not own (from byte 0) and the output rows it owns (from
+// kTcOutOffset).
+constexpr int kTcOutOffset = 68 * 1024;
+static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcOutOffset, "partial state before the output rows");
+static_assert(kTcOutOffset + kTcRows * 512 <= kTcSmemBytes, "output rows fit in the drained ring");
 // Barriers, tensor-memory slot and abort flag, then the softmax exchange
 // arrays (pair maxima [2][2][128], pair sums [2][128], destination rows [128]).
 constexpr int kTcBarBytes = (2 * kTcStages + 2 * kTcSBufs + 4) * 8 + 16;
@@ -176,11 +184,16 @@ __host__ __device__ constexpr uint32_t tc_idesc(bool b_mn_major, uint32_t n) {
          ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate) {
+// D (+)= A B on the tensor cores (kind::f16, fp32 accumulate in tensor
+// memory), A (M x 16, 16-bit) in tensor memory (lane = row, each 32-bit
+// column a pair of consecutive K elements), B from a shared-memory
+// descriptor.
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                          bool accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -217,14 +230,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31]));
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Byte offset of the 16-byte chunk c of row r in a swizzled 128-row operand
-// ([64-column block][128 rows][128 B]).
-__device__ __forceinline__ uint32_t tc_chunk(int r, int c) {
-  return static_cast<uint32_t>((c >> 3) * kTcQHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
 
 template <int DT>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -237,9 +252,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* q_s = base;                               // [2][128 rows][128 B]
-  uint8_t* p_s = base + kTcQBytes;                   // two P buffers, each [128 rows][128 B]
-  uint8_t* ring = p_s + 2 * kTcPBytes;               // [stage]{K, V}, each [2][64 tokens][128 B]
+  uint8_t* ring = base;                     // [stage]{K, V}: K [2][64 tokens][128 B], V [4 blocks][2][16][128 B]
+  uint8_t* out_s = ring + kTcOutOffset;     // after the last stage: the merged output rows, [128 rows][512 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kTcStages * kTcStageBytes);
   uint64_t* kv_full = bars;                // [kTcStages]
   uint64_t* kv_empty = bars + kTcStages;   // [kTcStages]
@@ -381,18 +395,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   } else {
+    float qv[32];  // a softmax thread's 64 dims of its Q row, as 32 pairs
     if (warp == kTcMmaWarp) {
       asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                        smem_u32(const_cast<uint32_t*>(tmem_slot))),
                    "r"(kTcTmemCols));
       asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     } else {
-      // Q rows into the swizzled A operand (zero rows past R): thread t copies
-      // eight 16-byte chunks of row t % 128.
+      // Q rows into tensor memory (zero rows past R): softmax warp (lg, hf)
+      // writes dims [64 hf, 64 hf + 64) of its 32 rows (lanes).
       // A negative scale is taken as |scale| on -Q (exact), so that the
       // softmax can take its maximum over the raw scores.
       const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
-      const int qr = threadIdx.x & (kTcRows - 1), c0 = (threadIdx.x >> 7) * 8;
+      const int qr = lg * 32 + lane, c0 = hf * 8;
       const int row = row0 + qr;
       const uint4* src = nullptr;
       if (row < R) {
@@ -401,20 +416,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                              (static_cast<size_t>(b) * p.n_q_heads + h) * D * 2);
       }
 #pragma unroll
-      for (int c = c0; c < c0 + 8; ++c) {
-        uint4 v = src ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-        v.x ^= flip;
-        v.y ^= flip;
-        v.z ^= flip;
-        v.w ^= flip;
-        *reinterpret_cast<uint4*>(q_s + tc_chunk(qr, c)) = v;
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = src ? __ldg(src + c0 + c) : make_uint4(0u, 0u, 0u, 0u);
+        qv[4 * c] = __uint_as_float(v.x ^ flip);
+        qv[4 * c + 1] = __uint_as_float(v.y ^ flip);
+        qv[4 * c + 2] = __uint_as_float(v.z ^ flip);
+        qv[4 * c + 3] = __uint_as_float(v.w ^ flip);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     tc_fence_before();
-    named_bar_sync(1, (kTcSoftmaxWarps + 1) * 32);  // softmax warps and the MMA warp
+    named_bar_sync(1, (kTcSoftmaxWarps + 1) * 32);  // softmax warps and the MMA warp: tensor memory allocated
     tc_fence_after();
     tmem = *tmem_slot;
+    if (warp != kTcMmaWarp) {
+      tmem_st32(tmem + (static_cast<uint32_t>(lg * 32) << 16) + kTcQCol + hf * 32, qv);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    named_bar_sync(1, (kTcSoftmaxWarps + 1) * 32);  // Q is in tensor memory
+    tc_fence_after();
 
     if (warp == kTcMmaWarp) {
       // ---------------- MMA issue (one thread) ----------------
@@ -424,7 +444,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // within each kind.
       if (lane == 0 && n_stages > 0) {
         constexpr uint32_t kIdS = tc_idesc<kBf16>(false, kTcKeys), kIdPV = tc_idesc<kBf16>(true, D);
-        const uint32_t qa = smem_u32(q_s), pa = smem_u32(p_s), ra = smem_u32(ring);
+        const uint32_t ra = smem_u32(ring);
         int ns = 0, np = 0;  // next stage whose S, whose P V is to be issued
         uint64_t t0 = global_timer_ns();
         bool mok = true;
@@ -437,8 +457,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t d = tmem + (ns % kTcSBufs) * kTcKeys;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              tc_mma(d, smem_desc_sw128(qa + (kk >> 2) * kTcQHalf + (kk & 3) * 32, 16, 1024),
-                     smem_desc_sw128(ka + (kk >> 2) * kTcKVHalf + (kk & 3) * 32, 16, 1024), kIdS, kk > 0);
+              tc_mma_ts(d, tmem + kTcQCol + kk * 8, smem_desc_sw128(ka + (kk >> 2) * kTcKVHalf + (kk & 3) * 32, 16, 1024),
+                        kIdS, kk > 0);
             }
             tc_commit(&s_full[ns % kTcSBufs]);
             ++ns;
@@ -447,13 +467,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (np < ns && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
             tc_fence_after();
             const uint32_t va = ra + (np % kTcStages) * kTcStageBytes + kTcKVBytes;
-            const uint32_t pb = pa + (np & 1) * kTcPBytes;
 #pragma unroll
             for (int kt = 0; kt < kTcKeys / 16; ++kt) {
               // V of block kt: [half][16 tokens][128 B], halves 2 KiB apart.
-              tc_mma(tmem + kTcOCol, smem_desc_sw128(pb + kt * 32, 16, 1024),
-                     smem_desc_sw128(va + kt * 2 * kBlockTokens * 128, kBlockTokens * 128, 1024), kIdPV,
-                     np > 0 || kt > 0);
+              tc_mma_ts(tmem + kTcOCol, tmem + kTcPCol + (np & 1) * (kTcKeys / 2) + kt * 8,
+                        smem_desc_sw128(va + kt * 2 * kBlockTokens * 128, kBlockTokens * 128, 1024), kIdPV,
+                        np > 0 || kt > 0);
             }
             tc_commit(&o_done[np & 1]);
             tc_commit(&kv_empty[np % kTcStages]);
@@ -558,17 +577,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 32; ++i) x[i] = i < live ? x[i] : -INFINITY;
         }
         uint64_t sum2[2] = {0ull, 0ull};
+        uint32_t pw[16];  // this half's 32 probabilities as 16-bit pairs
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t w[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float a = ex2_ftz(x[8 * cc + 2 * k]), b = ex2_ftz(x[8 * cc + 2 * k + 1]);
-            sum2[k & 1] = f2_add(sum2[k & 1], f2_pack(a, b));
-            w[k] = pack2<kBf16>(a, b);
-          }
-          *reinterpret_cast<uint4*>(p_s + (s & 1) * kTcPBytes + tc_chunk(r, hf * 4 + cc)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+        for (int k = 0; k < 16; ++k) {
+          const float a = ex2_ftz(x[2 * k]), b = ex2_ftz(x[2 * k + 1]);
+          sum2[k & 1] = f2_add(sum2[k & 1], f2_pack(a, b));
+          pw[k] = pack2<kBf16>(a, b);
+        }
+        if (ok) {
+          tmem_st16(lane_base + kTcPCol + (s & 1) * (kTcKeys / 2) + hf * 16, pw);
+          tmem_wait_st();
         }
         {
           float a0, a1, b0, b1;
@@ -576,7 +594,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           f2_unpack(sum2[1], b0, b1);
           l_half += (a0 + a1) + (b0 + b1);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[s & 1]);
@@ -658,9 +675,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       row_dst[r] = dst;
     }
     // This warp's 64 columns of its own share of O, weighted, into
-    // [128 rows][512 B] where Q and P were (16-byte chunk c of row r at
-    // c ^ (r % 8)).
-    uint8_t* out_s = q_s;
+    // [128 rows][512 B] (16-byte chunk c of row r at c ^ (r % 8)).
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       float t[32];

@@ -149,3 +149,22 @@ def test_cascade_split_full_size_sampled():
         out = run_cascade(w, prefix_splits=splits)
         ref, _, _ = oracle.workload_decode(w, rows=rows)
         assert_close(out, ref, w.dtype, rows=rows, what=f"shared_prefix_70b splits={splits}")
+
+
+@pytest.mark.parametrize("scale", [-0.0884, 0.0, 0.5])
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_cascade_scale_sign_and_size(scale, kernel):
+    # A negative scale runs on -Q in the tensor-memory kernel; zero gives
+    # uniform weights; a large one stresses the lazy rescale of O.
+    w = W.shared_prefix(n_seqs=10, prefix=208, suffix=(1, 40), seed=53, scale=scale)
+    out = run_cascade(w, prefix_kernel=kernel, prefix_splits=2 if kernel == 1 else 0)
+    ref, _, _ = oracle.workload_decode(w)
+    assert_close(out, ref, w.dtype, what=f"scale={scale} kernel={kernel}")
+
+
+@pytest.mark.parametrize("splits", [1, 2])
+def test_cascade_fp16_tensor_memory_kernel(splits):
+    w = W.shared_prefix(n_seqs=9, prefix=400, suffix=(1, 70), dtype=torch.float16, seed=54)
+    out = run_cascade(w, prefix_kernel=1, prefix_splits=splits)
+    ref, _, _ = oracle.workload_decode(w)
+    assert_close(out, ref, w.dtype, what=f"fp16 splits={splits}")
