@@ -46,19 +46,19 @@ KERNEL_SOURCES = ["paged_kv_cache_386_b200/csrc/pkv_kernels.cuh", "paged_kv_cach
                   "paged_kv_cache_386_b200/csrc/pkv_api.cu"]
 
 WORKLOADS = {
-    "llama3_8b_gqa": (lambda seed: W.uniform_gqa(seed=seed),
+    "llama3_8b_gqa": (lambda seed, **kw: W.uniform_gqa(seed=seed, **kw),
                       "llama3_8b_gqa: batch 64, 32 q / 8 kv heads, head_dim 128, bf16, block 16, "
                       "context U[128,4096], shuffled pool +10%"),
-    "llama2_7b_mha": (lambda seed: W.lognormal_mha(seed=seed),
+    "llama2_7b_mha": (lambda seed, **kw: W.lognormal_mha(seed=seed, **kw),
                       "llama2_7b_mha: batch 256, 32 q = 32 kv heads, head_dim 128, fp16, block 16, "
                       "context round(clip(lognormal(ln 300, 1), 1, 2048)), shuffled pool +10%"),
-    "shared_prefix_70b": (lambda seed: W.shared_prefix(seed=seed),
+    "shared_prefix_70b": (lambda seed, **kw: W.shared_prefix(seed=seed, **kw),
                           "shared_prefix_70b: 128 seqs, 64 q / 8 kv heads, head_dim 128, bf16, one shared "
                           "2048-token prefix + private suffix U[16,512]"),
-    "best_of_8": (lambda seed: W.best_of_n(seed=seed),
+    "best_of_8": (lambda seed, **kw: W.best_of_n(seed=seed, **kw),
                   "best_of_8: 16 prompts x 8 samples, 2000-token shared prompt + 100 private tokens, "
                   "64 q / 8 kv heads, head_dim 128, bf16"),
-    "long_ctx_128k": (lambda seed: W.long_context(seed=seed),
+    "long_ctx_128k": (lambda seed, **kw: W.long_context(seed=seed, **kw),
                       "long_ctx_128k: batch 4 x 131072 tokens, 64 q / 8 kv heads, head_dim 128, bf16, "
                       "4 sink keys x4"),
 }
@@ -185,7 +185,8 @@ def run_ours(args) -> None:
     mq = args.q_len > 1
     if mq and (args.workload != "llama3_8b_gqa" or args.cascade or args.kv != "16-bit"):
         raise SystemExit("--q-len > 1 is measured on llama3_8b_gqa with the 16-bit cache")
-    w = W.uniform_gqa(seed=args.seed, q_len=args.q_len) if mq else make(args.seed)
+    w = (W.uniform_gqa(seed=args.seed, q_len=args.q_len, placement=args.placement) if mq
+         else make(args.seed, placement=args.placement))
     if mq:
         desc += f"; {args.q_len} queries per sequence (the last {args.q_len} tokens, causal)"
     es = w.k_cache.element_size()
@@ -365,8 +366,11 @@ def run_ours(args) -> None:
     try:
         entries = json.loads(PROFILE_TRAFFIC.read_text())
         for prof in (entries if isinstance(entries, list) else [entries]):
+            # The capture is of one exact workload: kernel sources, shape,
+            # cache format, seed and placement must all match.
             if (prof.get("kernel_hash") == kernel_hash() and prof.get("workload") == args.workload
-                    and prof.get("kv", "16-bit") == ("int8" if int8 else "16-bit") and not args.cascade):
+                    and prof.get("kv", "16-bit") == ("int8" if int8 else "16-bit") and not args.cascade and not mq
+                    and prof.get("seed", 0) == args.seed and prof.get("placement", "shuffle") == args.placement):
                 traffic = prof.get("dram_bytes_per_launch")
     except Exception:
         traffic = None
@@ -381,8 +385,10 @@ def run_ours(args) -> None:
             "ms_per_step": round(max_step_s / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": ("int8 KV / " if int8 else "") + W.DTYPE_NAMES[w.dtype],
-            "data": "synthetic (seeded N(0,1) q/K/V, random block placement)",
+            "data": ("synthetic (seeded N(0,1) q/K/V, random block placement)" if args.placement == "shuffle" else
+                     "synthetic (seeded N(0,1) q/K/V, blocks of each sequence consecutive in the pool)"),
             "config": {"workload": desc, "global_batch": w.batch * world, "seq_len": "ragged",
+                       "placement": args.placement,
                        "mean_context": round(tr["tokens"] / w.batch, 1), "parallelism": f"replicas x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed)", "seed": args.seed,
                        "warmup_steps_run": warm_steps,
@@ -443,9 +449,22 @@ def cpu_baseline(w, kv_bytes: int, budget_s: float = 20.0) -> dict:
         done_bytes += sum(layout.blocks_for(lens[b]) for b in seqs) * n_kv * 16 * d * es * 2
         if t_total > budget_s:
             break
+    # The same oracle on one core, on the first sequences, for a few seconds.
+    one_bytes, one_seqs, t_one = 0, 0, 0.0
+    for b in order:
+        rows = [(b, h) for h in range(w.n_q_heads)]
+        t0 = time.perf_counter()
+        oracle.paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=rows, n_threads=1)
+        t_one += time.perf_counter() - t0
+        one_seqs += 1
+        one_bytes += layout.blocks_for(lens[b]) * n_kv * 16 * d * es * 2
+        if t_one > min(5.0, budget_s / 3):
+            break
     return {"value": round(done_bytes / t_total / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"append + fp64 decode of {done_seqs} of {w.batch} sequences (all q heads), "
-                      f"{t_total:.1f} s on {cores} threads"}
+                      f"{t_total:.1f} s on {cores} threads",
+            "one_core": {"value": round(one_bytes / t_one / 1e9, 4), "unit": UNIT,
+                         "sample": f"fp64 decode of {one_seqs} sequences (all q heads), {t_one:.1f} s on 1 thread"}}
 
 
 # ---------------------------------------------------------------------------
@@ -459,7 +478,7 @@ def run_reference(args) -> None:
     import oracle
 
     make, desc = WORKLOADS[args.workload]
-    w = make(args.seed)
+    w = make(args.seed, placement=args.placement)
     cores = oracle.cpu_cores()
     es = w.k_cache.element_size()
     # Each step: append of every new token + decode of a fixed sample of
@@ -503,6 +522,9 @@ def main(argv=None) -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="llama3_8b_gqa")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--placement", choices=["shuffle", "identity"], default="shuffle",
+                    help="physical block placement: a random permutation of the pool, or each sequence's blocks "
+                         "consecutive (paged vs contiguous reads with the same kernel)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of a CUDA graph replay")
