@@ -141,3 +141,24 @@ def test_cascade_options_are_checked_on_the_host(lib):
     st = lib.paged_attention_decode_cascade_ex(ptr, ptr, ptr, 1, ptr, 4, ptr, ptr, ptr, 4, ptr, 2, 8, 0.125,
                                                8, 2, 128, 16, ptr, 2, None, 0, None, ctypes.byref(opts))
     assert st == INVALID
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    # The boundary is a C ABI: the header must stand alone in strict C99.
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    src = tmp_path / "uses_header.c"
+    src.write_text('#include "pagedkv.h"\n'
+                   "int main(void) {\n"
+                   "  pkv_decode_options d = {0};\n"
+                   "  pkv_cascade_options c = {0};\n"
+                   "  pkv_bm_stats_t s;\n"
+                   "  (void)d; (void)c; (void)s;\n"
+                   "  return PKV_OK;\n"
+                   "}\n")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                        "-I", str(HEADER.parent), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
