@@ -1,6 +1,6 @@
 // pkv_device.cuh -- inline-PTX helpers for sm_100a used by the paged KV kernels:
-// mbarriers with bounded waits, TMA tensor loads (no multicast), ldmatrix,
-// mma.sync, packing and the per-device error word.
+// mbarriers with bounded waits, TMA tensor loads into the issuing CTA's own
+// shared memory, ldmatrix, mma.sync, packing and the per-device error word.
 #pragma once
 
 #include <cuda.h>
@@ -94,8 +94,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // ---------------------------------------------------------------------------
-// TMA: 4-D tiled load global -> shared, completion on an mbarrier.  CTA-local
-// destination, no multicast.
+// TMA: 4-D tiled load global -> shared, completion on an mbarrier.  The
+// destination is the issuing CTA's own shared memory.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -111,8 +111,7 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
 }
 
 // Contiguous bulk copy global -> this CTA's shared memory, completing on an
-// mbarrier (both addresses 16-byte aligned, bytes a multiple of 16).  No
-// multicast.
+// mbarrier (both addresses 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),

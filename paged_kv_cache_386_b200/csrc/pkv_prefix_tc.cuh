@@ -85,7 +85,7 @@ static_assert(kTcOutOffset + kTcRows * 512 <= kTcSmemBytes, "output rows fit in 
 constexpr int kTcBarBytes = (2 * kTcStages + 2 * kTcSBufs + 4) * 8 + 16;
 constexpr int kTcExchBytes = (4 * kTcRows + 2 * kTcRows + kTcRows) * 4;
 
-// 5-D tiled TMA load global -> this CTA's shared memory (no multicast): the
+// 5-D tiled TMA load global -> this CTA's own shared memory: the
 // V tile of one block and kv head in one request, box {64 dims, 16 tokens,
 // 2 halves of the head dim} landing as [half][token][128 B].
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
