@@ -90,3 +90,21 @@ def test_generation_is_deterministic():
     for x, y in [(a.q, b.q), (a.block_tables, b.block_tables), (a.slot_mapping, b.slot_mapping)]:
         assert torch.equal(x, y)
     assert torch.equal(a.k_cache.view(torch.int16), b.k_cache.view(torch.int16))
+
+
+def test_identity_placement_is_consecutive_with_the_same_traffic():
+    # bench.py --placement identity: the same sequences with each one's blocks
+    # consecutive in the pool, sequences back to back; the bytes a decode must
+    # read do not change.
+    a = W.uniform_gqa(batch=6, seed=3)
+    b = W.uniform_gqa(batch=6, seed=3, placement="identity")
+    assert a.lens() == b.lens()
+    assert torch.equal(a.q, b.q) and torch.equal(a.k_new, b.k_new)
+    nxt = 0
+    for s in range(b.batch):
+        nb = layout.blocks_for(b.lens()[s])
+        assert b.block_tables[s, :nb].tolist() == list(range(nxt, nxt + nb))
+        nxt += nb
+    args = (a.n_q_heads, a.n_kv_heads, a.head_dim, a.k_cache.element_size())
+    assert (layout.decode_traffic(a.block_tables, a.context_lens, *args)
+            == layout.decode_traffic(b.block_tables, b.context_lens, *args))
