@@ -11,11 +11,15 @@ Prints one JSON line (rank 0).  ``value`` is the KV-read throughput of the
 step in GB/s: the K and V bytes of every (block, kv head) tile the step reads
 (the algorithmic bytes; tail blocks count whole) divided by the device time
 of the step, measured with CUDA events on the launching stream.  Between
-timed steps a 256 MiB buffer is written (untimed) so that every step starts
-with a cold L2.  With N GPUs each rank runs its own replica (the path needs
-no exchange between GPUs) and ``value`` sums the replicas over the slowest
-rank's time.  ``--impl reference`` times the CPU oracle instead, on a bounded
-sample of the same workload.
+timed steps a 256 MiB buffer is written and a second one read (untimed), so
+that every step starts with a cold L2 holding no dirty lines.  ``e2e`` is the
+same metric through the public API with host buffers: each step's inputs
+copied in from pinned memory and its output copied back, pipelined over three
+streams as a serving loop runs them (the serial figure is reported beside
+it).  With N GPUs each rank runs its own replica (the path needs no exchange
+between GPUs) and ``value`` sums the replicas over the slowest rank's time.
+``--impl reference`` times the CPU oracle instead, on a bounded sample of the
+same workload.
 """
 
 from __future__ import annotations
