@@ -28,6 +28,8 @@ MUTANTS = [
      "size_t dst = (((size_t)blk * block_size + off) * n_kv_heads + h) * row;"),
     ("f16_exponent_bias", "expo - 25", "expo - 24"),
     ("f16_subnormal_scale", "ldexp((double)frac, -24)", "ldexp((double)frac, -25)"),
+    ("bf16_low_half", "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+    ("f16_sign_dropped", "return sign ? -mag : mag;", "return mag;"),
 ]
 
 
