@@ -1,9 +1,12 @@
 """Benchmark of one paged decode step: paged_kv_append of one new token per
 sequence, then paged_attention_decode over the whole batch.
 
-Default workload: the Llama-3-8B-shaped layer (batch 64, 32 q / 8 kv heads,
-head_dim 128, bf16, 16-token blocks, context lengths uniform in [128, 4096],
-blocks shuffled in a pool 10% larger than needed), seeded synthetic data.
+Default workload: the long-context split-KV layer, the largest single-GPU
+shape (batch 4 x 131,072 tokens, 64 q / 8 kv heads, head_dim 128, bf16,
+16-token blocks placed at random in a pool of exactly 4 x 8192 blocks, the
+first 4 keys of every sequence scaled x4 as attention sinks; 2.15 GB of K and
+V per step), seeded synthetic data.  ``--workload`` selects the other shapes
+(Llama-3-8B GQA, Llama-2-7B MHA, the shared-prefix ones).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -188,7 +191,7 @@ def run_ours(args) -> None:
     make, desc = WORKLOADS[args.workload]
     mq = args.q_len > 1
     if mq and (args.workload != "llama3_8b_gqa" or args.cascade or args.kv != "16-bit"):
-        raise SystemExit("--q-len > 1 is measured on llama3_8b_gqa with the 16-bit cache")
+        raise SystemExit("--q-len > 1 is measured on llama3_8b_gqa with the 16-bit cache (--workload llama3_8b_gqa)")
     w = (W.uniform_gqa(seed=args.seed, q_len=args.q_len, placement=args.placement) if mq
          else make(args.seed, placement=args.placement))
     if mq:
@@ -531,47 +534,87 @@ def run_ours(args) -> None:
         print(json.dumps(result), flush=True)
 
 
-def cpu_baseline(w, kv_bytes: int, budget_s: float = 20.0) -> dict:
-    """The oracle (append + fp64 decode) on the host cores, on whole sequences
-    of the same workload, for about ``budget_s`` seconds or one full pass."""
+def oracle_units(w) -> list[tuple[int, int]]:
+    """The (sequence, kv head) units of a workload, interleaved over the
+    sequences: one unit is every query head of one kv head of one sequence,
+    the work that reads that sequence's K and V of that kv head once."""
+    return [(b, h) for h in range(w.n_kv_heads) for b in range(w.batch)]
+
+
+def unit_rows(w, units) -> list[tuple[int, int]]:
+    g = w.n_q_heads // w.n_kv_heads
+    return [(b, h * g + i) for b, h in units for i in range(g)]
+
+
+def unit_bytes(w, units) -> int:
+    """K and V bytes the units read (whole blocks, as the GPU path counts them)."""
+    lens = w.lens()
+    es = w.k_cache.element_size()
+    return sum(layout.blocks_for(lens[b]) * 16 * w.head_dim * es * 2 for b, _ in units)
+
+
+def oracle_batches(w, cores: int, token_heads: int) -> list[list[tuple[int, int]]]:
+    """Consecutive batches of units, each about ``token_heads`` (context tokens
+    x query heads) of oracle work and at least one unit."""
+    lens = w.lens()
+    g = w.n_q_heads // w.n_kv_heads
+    out, cur, acc = [], [], 0
+    for u in oracle_units(w):
+        cur.append(u)
+        acc += lens[u[0]] * g
+        if acc >= token_heads:
+            out.append(cur)
+            cur, acc = [], 0
+    if cur:
+        out.append(cur)
+    return out
+
+
+# fp64 oracle work one host thread does in about a second (context tokens x
+# query heads), used to size the samples.
+ORACLE_TOKEN_HEADS_PER_S = 250_000
+
+
+def cpu_baseline(w, kv_bytes: int, budget_s: float = 15.0) -> dict:
+    """The oracle (append + fp64 decode) on the host cores, on a bounded
+    sample of the same workload: batches of (sequence, kv head) units, each
+    about a second of work on all threads, until ``budget_s`` has passed or
+    the whole workload is done."""
     import oracle
 
     cores = oracle.cpu_cores()
-    lens = w.lens()
-    n_kv, d, es = w.n_kv_heads, w.head_dim, w.k_cache.element_size()
-    order = list(range(w.batch))
-    done_bytes, done_seqs, t_total = 0, 0, 0.0
     kc, vc = w.k_cache.clone(), w.v_cache.clone()
     t0 = time.perf_counter()
     oracle.kv_append(w.k_new, w.v_new, w.slot_mapping, kc, vc, w.block_size)
-    t_total += time.perf_counter() - t0
-    chunk = 8
-    for s in range(0, len(order), chunk):
-        seqs = order[s:s + chunk]
-        rows = [(b, h) for b in seqs for h in range(w.n_q_heads)]
+    t_total = time.perf_counter() - t0
+    done_units, done_bytes = 0, 0
+    for units in oracle_batches(w, cores, cores * ORACLE_TOKEN_HEADS_PER_S):
         t0 = time.perf_counter()
-        oracle.paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=rows, n_threads=cores)
+        oracle.paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=unit_rows(w, units),
+                            n_threads=cores)
         t_total += time.perf_counter() - t0
-        done_seqs += len(seqs)
-        done_bytes += sum(layout.blocks_for(lens[b]) for b in seqs) * n_kv * 16 * d * es * 2
+        done_units += len(units)
+        done_bytes += unit_bytes(w, units)
         if t_total > budget_s:
             break
-    # The same oracle on one core, on the first sequences, for a few seconds.
-    one_bytes, one_seqs, t_one = 0, 0, 0.0
-    for b in order:
-        rows = [(b, h) for h in range(w.n_q_heads)]
+    # The same oracle on one thread, a few seconds of it.
+    one_units, one_bytes, t_one = 0, 0, 0.0
+    for units in oracle_batches(w, 1, ORACLE_TOKEN_HEADS_PER_S):
         t0 = time.perf_counter()
-        oracle.paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=rows, n_threads=1)
+        oracle.paged_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, rows=unit_rows(w, units),
+                            n_threads=1)
         t_one += time.perf_counter() - t0
-        one_seqs += 1
-        one_bytes += layout.blocks_for(lens[b]) * n_kv * 16 * d * es * 2
+        one_units += len(units)
+        one_bytes += unit_bytes(w, units)
         if t_one > min(5.0, budget_s / 3):
             break
+    n_all = w.batch * w.n_kv_heads
     return {"value": round(done_bytes / t_total / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"append + fp64 decode of {done_seqs} of {w.batch} sequences (all q heads), "
-                      f"{t_total:.1f} s on {cores} threads",
+            "sample": f"append of all {w.batch} new tokens + fp64 decode of {done_units} of {n_all} "
+                      f"(sequence, kv head) units (all their q heads), {t_total:.1f} s on {cores} threads",
             "one_core": {"value": round(one_bytes / t_one / 1e9, 4), "unit": UNIT,
-                         "sample": f"fp64 decode of {one_seqs} sequences (all q heads), {t_one:.1f} s on 1 thread"}}
+                         "sample": f"fp64 decode of {one_units} (sequence, kv head) units, {t_one:.1f} s "
+                                   f"on 1 thread"}}
 
 
 # ---------------------------------------------------------------------------
@@ -587,13 +630,14 @@ def run_reference(args) -> None:
     make, desc = WORKLOADS[args.workload]
     w = make(args.seed, placement=args.placement)
     cores = oracle.cpu_cores()
-    es = w.k_cache.element_size()
     # Each step: append of every new token + decode of a fixed sample of
-    # sequences (all q heads), sized to keep the whole run within minutes.
-    n_seq = w.batch if args.ref_seqs <= 0 else min(args.ref_seqs, w.batch)
-    sample = list(range(0, w.batch, max(1, w.batch // n_seq)))[:n_seq]
-    rows = [(b, h) for b in sample for h in range(w.n_q_heads)]
-    kv_bytes = sum(layout.blocks_for(w.lens()[b]) for b in sample) * w.n_kv_heads * 16 * w.head_dim * es * 2
+    # (sequence, kv head) units (every q head of each), about a second of
+    # work on all threads unless --ref-units asks for more, so that the whole
+    # run stays within minutes.
+    batches = oracle_batches(w, cores, cores * ORACLE_TOKEN_HEADS_PER_S)
+    sample = batches[0] if args.ref_units <= 0 else oracle_units(w)[: args.ref_units]
+    rows = unit_rows(w, sample)
+    kv_bytes = unit_bytes(w, sample)
 
     def step():
         kc, vc = w.k_cache, w.v_cache
@@ -607,8 +651,8 @@ def run_reference(args) -> None:
         step()
     dt = time.perf_counter() - t0
     value = kv_bytes * args.steps / dt / 1e9
-    sample_desc = (f"append of all {w.batch} new tokens + fp64 decode of {len(sample)} of {w.batch} "
-                   f"sequences (all q heads) per step")
+    sample_desc = (f"append of all {w.batch} new tokens + fp64 decode of {len(sample)} of "
+                   f"{w.batch * w.n_kv_heads} (sequence, kv head) units (all their q heads) per step")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
@@ -627,7 +671,7 @@ def main(argv=None) -> None:
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="llama3_8b_gqa")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="long_ctx_128k")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--placement", choices=["shuffle", "identity"], default="shuffle",
                     help="physical block placement: a random permutation of the pool, or each sequence's blocks "
@@ -638,7 +682,8 @@ def main(argv=None) -> None:
     ap.add_argument("--no-clocks", action="store_true", help="do not sample SM clocks during the timed region")
     ap.add_argument("--cascade", action="store_true",
                     help="decode shared-prefix workloads with paged_attention_decode_cascade")
-    ap.add_argument("--ref-seqs", type=int, default=0, help="sequences per reference-arm step (0: all)")
+    ap.add_argument("--ref-units", type=int, default=0,
+                    help="(sequence, kv head) units per reference-arm step (0: about a second of work)")
     ap.add_argument("--q-len", type=int, default=1,
                     help="queries per sequence (multi-query decode of the last q_len tokens)")
     ap.add_argument("--kv", choices=["16-bit", "int8"], default="16-bit",

@@ -43,8 +43,10 @@
  * failed check returns a status and enqueues nothing.  Values that only the
  * device sees (block ids, context lengths, slots) are range-checked by the
  * kernels: a bad value sets a bit in a per-device error word (read and cleared
- * by pkv_get_device_error), the offending access is skipped or reads zeros,
- * and the kernel never traps.  No entry point aborts the process.
+ * by pkv_get_device_error), the offending access is skipped (a block whose
+ * id is out of range contributes no token to any softmax; a row that is left
+ * with no token is a zero row), and the kernel never traps.  No entry point
+ * aborts the process.
  */
 #ifndef PAGEDKV_H_
 #define PAGEDKV_H_
@@ -76,10 +78,12 @@ typedef enum pkv_status {
 } pkv_status;
 
 /* Bits of the device error word (pkv_get_device_error). */
-#define PKV_DEVERR_BLOCK_ID 0x1u   /* block table entry outside [0, num_blocks): zeros were read */
+#define PKV_DEVERR_BLOCK_ID 0x1u   /* block table entry outside [0, num_blocks): nothing was read from
+                                      it and its tokens were left out of the softmax */
 #define PKV_DEVERR_CONTEXT 0x2u    /* context length < 0 or > max_blocks_per_seq * block_size: clamped */
 #define PKV_DEVERR_SLOT 0x4u       /* slot >= num_blocks * block_size: the token was not written */
-#define PKV_DEVERR_TIMEOUT 0x8u    /* a bounded in-kernel wait (2 s) gave up: that launch wrote no result */
+#define PKV_DEVERR_TIMEOUT 0x8u    /* a bounded in-kernel wait (2 s by default) gave up: that launch's
+                                      output is undefined (the kernel drained its own copies and ended) */
 #define PKV_DEVERR_SCHEDULE 0x10u  /* the decode workspace was not zero-filled before its first use: that
                                       launch's result is wrong (the workspace is zeroed again) */
 
@@ -235,7 +239,14 @@ struct pkv_decode_options {
                               paged_attention_workspace_size_ex, zero-filled before first use.
                               Measured on B200 it costs more than the imbalance it removes */
   int32_t static_permille; /* 0: default (800); 500..999: share of its range a unit keeps */
-  int32_t reserved[4]; /* must be zero */
+  int32_t wait_limit_us;   /* 0: default (2 s); n > 0: every bounded wait of this launch gives up
+                              after n microseconds (with PKV_DEVERR_TIMEOUT) */
+  int32_t test_withhold_unit; /* test hook for the failure path. 0: off; u + 1: the producer never
+                                 issues the copies of work unit u (u < the unit count), so that
+                                 its consumer's bounded wait runs out: the launch returns with
+                                 PKV_DEVERR_TIMEOUT set and writes no defined result, and the
+                                 next call is unaffected.  Nothing faults or hangs */
+  int32_t reserved[2]; /* must be zero */
 };
 
 /* paged_attention_decode with options (NULL options = paged_attention_decode). */

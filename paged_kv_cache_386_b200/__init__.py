@@ -50,7 +50,8 @@ class PagedKVError(RuntimeError):
 class _Options(ctypes.Structure):
     _fields_ = [("num_units", ctypes.c_int32), ("force_simt", ctypes.c_int32),
                 ("balance_chunks", ctypes.c_int32), ("static_permille", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 4)]
+                ("wait_limit_us", ctypes.c_int32), ("test_withhold_unit", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 class _CascadeOptions(ctypes.Structure):
@@ -140,10 +141,30 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-def _stream(stream) -> int | None:
+def _stream(stream, device=None) -> int | None:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _same_device(device, *tensors) -> None:
+    for t in tensors:
+        if t is not None and t.device != device:
+            raise ValueError(f"every tensor must be on {device} (found {t.device})")
+
+
+def _check_decode_io(q, k_cache, v_cache, out, *others) -> None:
+    """The C layer sees raw pointers and q's dtype only: check here that the
+    caches and out have q's dtype, that out has q's shape, and that every
+    tensor is on q's device (the call runs with that device current)."""
+    if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError(f"k_cache/v_cache dtype ({k_cache.dtype}, {v_cache.dtype}) must equal q's ({q.dtype})")
+    if out.dtype != q.dtype or tuple(out.shape) != tuple(q.shape):
+        raise ValueError(f"out must have q's dtype and shape ({q.dtype}, {tuple(q.shape)}), "
+                         f"got ({out.dtype}, {tuple(out.shape)})")
+    if not out.is_contiguous():
+        raise ValueError("out must be contiguous")
+    _same_device(q.device, k_cache, v_cache, out, *others)
 
 
 def _dev(t: torch.Tensor, name: str) -> int:
@@ -173,12 +194,17 @@ def paged_kv_append(k, v, slot_mapping, k_cache, v_cache, block_size: int = 16, 
     num_blocks, n_kv, bs, d = k_cache.shape
     if bs != block_size or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("cache shapes disagree")
-    if k.dtype != k_cache.dtype or v.dtype != k_cache.dtype or slot_mapping.dtype != torch.int64:
+    if (k.dtype != k_cache.dtype or v.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype
+            or slot_mapping.dtype != torch.int64):
         raise ValueError("dtype mismatch (slot_mapping must be int64)")
-    _check(lib.paged_kv_append(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping"),
-                               k.shape[0], _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-                               num_blocks, bs, n_kv, d, _DTYPE[k_cache.dtype], _stream(stream)),
-           "paged_kv_append")
+    if tuple(k.shape[1:]) != (n_kv, d) or tuple(v.shape) != tuple(k.shape) or slot_mapping.shape[0] != k.shape[0]:
+        raise ValueError("k, v must be [num_tokens, n_kv_heads, head_dim] and slot_mapping [num_tokens]")
+    _same_device(k_cache.device, k, v, slot_mapping, v_cache)
+    with torch.cuda.device(k_cache.device):
+        _check(lib.paged_kv_append(_dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping"),
+                                   k.shape[0], _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                   num_blocks, bs, n_kv, d, _DTYPE[k_cache.dtype], _stream(stream, k_cache.device)),
+               "paged_kv_append")
 
 
 def paged_attention_workspace_size(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
@@ -200,10 +226,14 @@ def new_workspace(nbytes: int, device=None) -> torch.Tensor:
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out=None,
                            workspace=None, num_units: int = 0, force_simt: bool = False,
                            balance_chunks: int = 0, static_permille: int = 0,
-                           block_size: int = 16, stream=None):
+                           block_size: int = 16, stream=None, wait_limit_us: int = 0,
+                           test_withhold_unit: int = -1):
     """Single-query attention through the block table; returns ``out``.
     With ``balance_chunks`` > 0 the workspace (see new_workspace) must be
-    zero-filled before its first use."""
+    zero-filled before its first use.  ``wait_limit_us`` and
+    ``test_withhold_unit`` are the failure-path test hooks of
+    ``pkv_decode_options`` (a unit whose copies are never issued, so that its
+    bounded wait runs out)."""
     lib = _load()
     B, n_q, d = q.shape
     num_blocks, n_kv, bs, d2 = k_cache.shape
@@ -213,16 +243,19 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         raise ValueError("block_tables and context_lens must be int32")
     if out is None:
         out = torch.empty_like(q)
+    _check_decode_io(q, k_cache, v_cache, out, block_tables, context_lens, workspace)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
     opts = _Options(num_units=int(num_units), force_simt=int(bool(force_simt)),
-                    balance_chunks=int(balance_chunks), static_permille=int(static_permille))
-    _check(lib.paged_attention_decode_ex(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
-        B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
-        ws_ptr, ws_bytes, _stream(stream), ctypes.byref(opts)), "paged_attention_decode")
+                    balance_chunks=int(balance_chunks), static_permille=int(static_permille),
+                    wait_limit_us=int(wait_limit_us), test_withhold_unit=int(test_withhold_unit) + 1)
+    with torch.cuda.device(q.device):
+        _check(lib.paged_attention_decode_ex(
+            _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+            _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+            B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
+            ws_ptr, ws_bytes, _stream(stream, q.device), ctypes.byref(opts)), "paged_attention_decode")
     return out
 
 
@@ -257,19 +290,23 @@ def paged_attention_decode_cascade(q, k_cache, v_cache, prefix_block_tables, pre
             raise ValueError(f"{name} must be int32")
     if out is None:
         out = torch.empty_like(q)
+    _check_decode_io(q, k_cache, v_cache, out, prefix_block_tables, prefix_lens, seq_group, block_tables,
+                     context_lens, workspace)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
     n_groups = prefix_lens.shape[0]
     opts = _CascadeOptions(prefix_splits=int(prefix_splits), prefix_kernel=int(prefix_kernel))
-    _check(lib.paged_attention_decode_cascade_ex(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), n_groups,
-        _dev(prefix_block_tables, "prefix_block_tables") if n_groups else None,
-        prefix_block_tables.shape[1] if n_groups else 0,
-        _dev(prefix_lens, "prefix_lens") if n_groups else None, _dev(seq_group, "seq_group") if n_groups else None,
-        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
-        B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
-        ws_ptr, ws_bytes, _stream(stream), ctypes.byref(opts)), "paged_attention_decode_cascade")
+    with torch.cuda.device(q.device):
+        _check(lib.paged_attention_decode_cascade_ex(
+            _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), n_groups,
+            _dev(prefix_block_tables, "prefix_block_tables") if n_groups else None,
+            prefix_block_tables.shape[1] if n_groups else 0,
+            _dev(prefix_lens, "prefix_lens") if n_groups else None,
+            _dev(seq_group, "seq_group") if n_groups else None,
+            _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+            B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
+            ws_ptr, ws_bytes, _stream(stream, q.device), ctypes.byref(opts)), "paged_attention_decode_cascade")
     return out
 
 
@@ -287,11 +324,13 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
         raise ValueError("block_tables and context_lens must be int32")
     if out is None:
         out = torch.empty_like(q)
-    _check(lib.paged_attention_decode_noalloc(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
-        B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
-        _stream(stream)), "paged_attention_decode_noalloc")
+    _check_decode_io(q, k_cache, v_cache, out, block_tables, context_lens)
+    with torch.cuda.device(q.device):
+        _check(lib.paged_attention_decode_noalloc(
+            _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+            _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+            B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
+            _stream(stream, q.device)), "paged_attention_decode_noalloc")
     return out
 
 
@@ -316,10 +355,12 @@ def paged_kv_copy_blocks(k_cache, v_cache, src_blocks, dst_blocks, block_size: i
     n = src_blocks.numel()
     if n == 0:
         return
-    _check(lib.paged_kv_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-                                    _dev(src_blocks, "src_blocks"), _dev(dst_blocks, "dst_blocks"), n,
-                                    num_blocks, bs, n_kv, d, _DTYPE[k_cache.dtype], _stream(stream)),
-           "paged_kv_copy_blocks")
+    _same_device(k_cache.device, v_cache, src_blocks, dst_blocks)
+    with torch.cuda.device(k_cache.device):
+        _check(lib.paged_kv_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                        _dev(src_blocks, "src_blocks"), _dev(dst_blocks, "dst_blocks"), n,
+                                        num_blocks, bs, n_kv, d, _DTYPE[k_cache.dtype],
+                                        _stream(stream, k_cache.device)), "paged_kv_copy_blocks")
 
 
 def _host(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
@@ -435,9 +476,14 @@ def paged_kv_append_int8(k, v, slot_mapping, kv_cache, block_size: int = 16, str
         raise ValueError("INT8 cache shape disagrees with k")
     if v.dtype != k.dtype or slot_mapping.dtype != torch.int64:
         raise ValueError("dtype mismatch (slot_mapping must be int64)")
-    _check(lib.paged_kv_append_int8(_dev(k, "k"), _dev(v, "v"), _DTYPE[k.dtype], _dev(slot_mapping, "slot_mapping"),
-                                    k.shape[0], _dev(kv_cache, "kv_cache"), num_blocks, block_size, n_kv, d,
-                                    _stream(stream)), "paged_kv_append_int8")
+    if tuple(v.shape) != tuple(k.shape) or slot_mapping.shape[0] != k.shape[0]:
+        raise ValueError("k, v must be [num_tokens, n_kv_heads, head_dim] and slot_mapping [num_tokens]")
+    _same_device(kv_cache.device, k, v, slot_mapping)
+    with torch.cuda.device(kv_cache.device):
+        _check(lib.paged_kv_append_int8(_dev(k, "k"), _dev(v, "v"), _DTYPE[k.dtype],
+                                        _dev(slot_mapping, "slot_mapping"), k.shape[0], _dev(kv_cache, "kv_cache"),
+                                        num_blocks, block_size, n_kv, d, _stream(stream, kv_cache.device)),
+               "paged_kv_append_int8")
 
 
 def paged_attention_decode_int8(q, kv_cache, block_tables, context_lens, scale: float, out=None, workspace=None,
@@ -452,13 +498,18 @@ def paged_attention_decode_int8(q, kv_cache, block_tables, context_lens, scale: 
         raise ValueError("block_tables and context_lens must be int32")
     if out is None:
         out = torch.empty_like(q)
+    if out.dtype != q.dtype or tuple(out.shape) != tuple(q.shape) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor of q's dtype and shape")
+    _same_device(q.device, kv_cache, out, block_tables, context_lens, workspace)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
-    _check(lib.paged_attention_decode_int8(
-        _dev(q, "q"), _dev(kv_cache, "kv_cache"), _dev(block_tables, "block_tables"), block_tables.shape[1],
-        _dev(context_lens, "context_lens"), B, num_blocks, float(scale), n_q, n_kv, d, block_size, _dev(out, "out"),
-        _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream)), "paged_attention_decode_int8")
+    with torch.cuda.device(q.device):
+        _check(lib.paged_attention_decode_int8(
+            _dev(q, "q"), _dev(kv_cache, "kv_cache"), _dev(block_tables, "block_tables"), block_tables.shape[1],
+            _dev(context_lens, "context_lens"), B, num_blocks, float(scale), n_q, n_kv, d, block_size,
+            _dev(out, "out"), _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream, q.device)),
+            "paged_attention_decode_int8")
     return out
 
 
@@ -484,11 +535,14 @@ def paged_attention_decode_mq(q, k_cache, v_cache, block_tables, context_lens, s
         raise ValueError("block_tables and context_lens must be int32")
     if out is None:
         out = torch.empty_like(q)
+    _check_decode_io(q, k_cache, v_cache, out, block_tables, context_lens, workspace)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
-    _check(lib.paged_attention_decode_mq(
-        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables"),
-        block_tables.shape[1], _dev(context_lens, "context_lens"), B, q_len, num_blocks, float(scale), n_q, n_kv, d,
-        bs, _dev(out, "out"), _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream)), "paged_attention_decode_mq")
+    with torch.cuda.device(q.device):
+        _check(lib.paged_attention_decode_mq(
+            _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables"),
+            block_tables.shape[1], _dev(context_lens, "context_lens"), B, q_len, num_blocks, float(scale), n_q,
+            n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream, q.device)),
+            "paged_attention_decode_mq")
     return out

@@ -509,8 +509,9 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   pkv_decode_options opt = {};
   if (options) {
     opt = *options;
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 2; ++i)
       if (opt.reserved[i] != 0) return PKV_ERR_INVALID_ARG;
+    if (opt.wait_limit_us < 0 || opt.test_withhold_unit < 0) return PKV_ERR_INVALID_ARG;
     if (opt.num_units < 0 || (opt.force_simt != 0 && opt.force_simt != 1)) return PKV_ERR_INVALID_ARG;
     if (opt.balance_chunks < 0 || opt.balance_chunks > 4) return PKV_ERR_INVALID_ARG;
     if (opt.static_permille != 0 && (opt.static_permille < 500 || opt.static_permille > 999))
@@ -602,6 +603,8 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   p.init = init;
   p.seq_group = seq_group;
   p.n_groups = n_groups;
+  p.wait_limit_ns = opt.wait_limit_us > 0 ? static_cast<uint64_t>(opt.wait_limit_us) * 1000u : kWaitLimitNs;
+  p.withhold_unit = opt.test_withhold_unit - 1;
 
   if (st == PKV_OK && mq) {
     st = dtype == PKV_F16 ? dispatch_mq<kF16>(head_dim, gpad, mk, mv, p, grid, smem, s)

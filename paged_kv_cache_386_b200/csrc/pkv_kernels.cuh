@@ -294,6 +294,8 @@ struct DecodeParams {
   int32_t rows;        // rows per segment: q_len * gp
   int32_t head_dim;
   float scale_log2;    // scale * log2(e)
+  uint64_t wait_limit_ns;  // bound of every in-kernel wait
+  int32_t withhold_unit;   // test hook: this unit's producer lane issues nothing (-1: none)
 };
 
 // Row `row` of segment (b, hg) -- query row / gp, head hg * gp + row % gp
@@ -656,7 +658,8 @@ struct MmaConsumer {
       if (row >= p.rows) continue;
       if (rec == nullptr) {
         T* ob = static_cast<T*>(p.out) + out_row(p, b, hg, row) * D;
-        const float inv = 1.f / lt[r];
+        // lt is 0 only when every tile of the row was skipped (bad block ids): a zero row.
+        const float inv = lt[r] > 0.f ? 1.f / lt[r] : 0.f;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           float a0, a1;
@@ -839,7 +842,7 @@ struct SimtConsumer {
     const int d0 = sub * DL + tp * DO;
     if (rec == nullptr) {
       T* ob = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.n_q_heads + hg) * D + d0;
-      const float inv = 1.f / lt;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;  // 0: every tile skipped
       if constexpr (DT == kF32) {
 #pragma unroll
         for (int i = 0; i < DO; ++i) ob[i] = o[i] * inv;
@@ -1212,12 +1215,13 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
     for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float w = j < n ? exp2f(mj[j] - M) : 0.f;
+      // M is -inf only when every piece skipped all its tiles (bad block ids).
+      const float w = (j < n && M != -INFINITY) ? exp2f(mj[j] - M) : 0.f;
       L = fmaf(w, lj[j], L);
 #pragma unroll
       for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, o[j][i], acc[i]);
     }
-    store(acc, 1.f / L);
+    store(acc, L > 0.f ? 1.f / L : 0.f);
     return;
   }
   // Scalars of pieces lane and lane + 32; pieces beyond 64 (rare) are folded
@@ -1235,6 +1239,7 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
   for (int j = 64 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(rec_of(j) + mo));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (M == -INFINITY) M = 0.f;  // every piece empty (bad block ids): all weights 0, a zero row
   const float w0 = exp2f(m0 - M), w1 = exp2f(m1 - M);
   float L = w0 * l0 + w1 * l1;
   for (int j = 64 + lane; j < n; j += 32) L = fmaf(exp2f(__ldcg(rec_of(j) + mo) - M), __ldcg(rec_of(j) + lo), L);
@@ -1268,7 +1273,7 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
       for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wj, o[jj][i], acc[i]);
     }
   }
-  store(acc, 1.f / L);
+  store(acc, L > 0.f ? 1.f / L : 0.f);
 }
 
 // GPAD: 0 = CUDA-core consumer (gp == 1); 8 or 16 = tensor-core consumer.
@@ -1381,6 +1386,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // before the current chunk's end and read at its last tile, so the warp
     // (whose lanes run in step) never waits on an L2 round trip.
     const int u = blockIdx.x * kConsumerWarps + lane;
+    // Test hook: the lane of the withheld unit never issues, so that its
+    // consumer's bounded wait runs out (no copy is then in flight for it).
+    const bool withheld = u == p.withhold_unit;
     Walk wn;
     bool walking = false;
     if (lane < kConsumerWarps && u < U) {
@@ -1429,24 +1437,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     uint64_t idle_since = 0;
     while (__any_sync(0xffffffffu, t0.valid)) {
       bool progressed = false;
-      if (t0.valid) {
+      if (t0.valid && !withheld) {
         const int slot = lane * p.stages + stage;
         if (mbar_test_wait(&empty_bar[slot], phase ^ 1u)) {
-          int ph = t0.phys;
-          if (ph < 0 || ph >= p.num_blocks) {
-            flag_error(PKV_DEVERR_BLOCK_ID);
-            ph = 0;
-          }
+          const int ph = t0.phys;
+          // A block id outside the pool: nothing is copied, the slot is
+          // marked (info.w) and its consumer leaves the tile's tokens out.
+          const int bad = (ph < 0 || ph >= p.num_blocks) ? 1 : 0;
+          if (bad) flag_error(PKV_DEVERR_BLOCK_ID);
           asm volatile("st.shared.v4.s32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(&slot_info[slot])), "r"(t0.info.x),
-                       "r"(t0.info.y), "r"(t0.info.z), "r"(t0.info.w)
+                       "r"(t0.info.y), "r"(t0.info.z), "r"(bad)
                        : "memory");  // published to the consumer by the arrive below
-          mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
           uint8_t* sk = ring + static_cast<size_t>(slot) * kRingStride;
-          if constexpr (kI8) {
+          if (bad) {
+            mbar_arrive(&full_bar[slot]);  // completes the phase with no bytes in flight
+          } else if constexpr (kI8) {
+            mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
             // The whole record in one contiguous request.
             const size_t bh = static_cast<size_t>(ph) * p.n_kv_heads + t0.kvh;
             bulk_load(sk, p.kv_i8 + bh * kRingStride, kRingStride, &full_bar[slot]);
           } else {
+            mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
 #pragma unroll
             for (int y = 0; y < Y; ++y)
               tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, t0.kvh, ph);
@@ -1464,13 +1475,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           progressed = true;
         }
       }
-      // Bounded: give up (warp-uniformly) after kWaitLimitNs without progress.
+      // Bounded: give up (warp-uniformly) after the wait limit without progress.
       if (__any_sync(0xffffffffu, progressed)) {
         idle_since = 0;
       } else {
         const uint64_t now = global_timer_ns();
         if (idle_since == 0) idle_since = now;
-        const bool give_up = __shfl_sync(0xffffffffu, (*abort_flag != 0) || (now - idle_since > kWaitLimitNs), 0);
+        const bool give_up = __shfl_sync(0xffffffffu, (*abort_flag != 0) || (now - idle_since > p.wait_limit_ns), 0);
         if (give_up) {
           if (lane == 0 && *abort_flag == 0) {
             *abort_flag = 1;
@@ -1487,7 +1498,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const uint32_t par = static_cast<uint32_t>((cnt - 1) & 1);
         const uint64_t t0s = global_timer_ns();
         while (!mbar_try_wait(&full_bar[lane * p.stages + s], par)) {
-          if (global_timer_ns() - t0s > kWaitLimitNs) {
+          if (global_timer_ns() - t0s > p.wait_limit_ns) {
             flag_error(kDevErrTimeout);
             break;
           }
@@ -1554,18 +1565,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           q_ready = true;
         }
         const int slot = warp * p.stages + stage;
-        if (!mbar_wait_bounded(&full_bar[slot], phase, abort_flag, kWaitLimitNs)) {
+        if (!mbar_wait_bounded(&full_bar[slot], phase, abort_flag, p.wait_limit_ns)) {
           aborted = true;
           break;
         }
+        // From the producer: the next chunk (on a chunk's last tile) and
+        // whether the tile's block id was out of range (info.w).
+        int4 info;
+        asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(info.x), "=r"(info.y), "=r"(info.z), "=r"(info.w)
+                     : "r"(smem_u32(&slot_info[slot])));
         int next_chunk = -1, n0 = 0, n1 = 0;
         if (last) {
           // The chunk this warp runs next, as claimed by its producer lane:
           // start copying the Q of its first segment.
-          int4 info;
-          asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];"
-                       : "=r"(info.x), "=r"(info.y), "=r"(info.z), "=r"(info.w)
-                       : "r"(smem_u32(&slot_info[slot])));
           next_chunk = info.x;
           n0 = info.y;
           n1 = info.z;
@@ -1582,7 +1595,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int nv = kMQ ? rem : min(kBlockTokens, rem);
         const uint32_t kaddr = smem_u32(ring + static_cast<size_t>(slot) * kRingStride);
         const uint32_t vaddr = kI8 ? kaddr + D * kBlockTokens : kaddr + kTileBytes;
-        cs.tile(kaddr, vaddr, nv, p.scale_log2, lane);
+        if (info.w == 0) cs.tile(kaddr, vaddr, nv, p.scale_log2, lane);  // a bad block's tokens are left out
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[slot]);
         if (++stage == p.stages) {

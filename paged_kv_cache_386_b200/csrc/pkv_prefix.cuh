@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kPrefixThreads, 1)
           int phys = 0;
           if (j * kBlockTokens < plen) {
             phys = __ldg(tab + j);
-            if (phys < 0 || phys >= p.num_blocks) {
+            if (phys < 0 || phys >= p.num_blocks) {  // copied from block 0; the consumers mask its keys
               flag_error(PKV_DEVERR_BLOCK_ID);
               phys = 0;
             }
@@ -196,9 +196,21 @@ __global__ void __launch_bounds__(kPrefixThreads, 1)
   for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
+  // Block ids of the stage's blocks, read one stage ahead by lanes 0..3: a
+  // block whose id is outside the pool contributes no key (bit i of `bad`).
+  const int32_t* ctab = p.prefix_tables + static_cast<size_t>(grp) * p.max_prefix_blocks;
+  const int n_prefix_blocks = plen / kBlockTokens;
+  auto stage_id = [&](int s) {
+    const int j = s * kPrefixBlocks + lane;
+    return (lane < kPrefixBlocks && j < n_prefix_blocks) ? __ldg(ctab + j) : 0;
+  };
+  int id_next = n_stages > 0 ? stage_id(0) : 0;
   int slot = 0;
   uint32_t phase = 0;
   for (int s = 0; s < n_stages; ++s) {
+    const int id = id_next;
+    if (s + 1 < n_stages) id_next = stage_id(s + 1);
+    const uint32_t bad = __ballot_sync(0xffffffffu, id < 0 || id >= p.num_blocks) & ((1u << kPrefixBlocks) - 1u);
     if (!mbar_wait_bounded(&full_bar[slot], phase, abort_flag, kWaitLimitNs)) break;
     const uint32_t kb = smem_u32(ring + static_cast<size_t>(slot) * kStageBytes);
     const uint32_t vb = kb + kHalf;
@@ -233,20 +245,23 @@ __global__ void __launch_bounds__(kPrefixThreads, 1)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int tok = nt * 8 + 2 * t + e;
-          const float x = tok < nv ? sc[nt][2 * r + e] * p.scale_log2 : -INFINITY;
+          const float x = (tok < nv && !((bad >> (nt >> 1)) & 1u)) ? sc[nt][2 * r + e] * p.scale_log2 : -INFINITY;
           sc[nt][2 * r + e] = x;
           mx = fmaxf(mx, x);
         }
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float mn = fmaxf(m_run[r], mx);
-      alpha[r] = exp2f(m_run[r] - mn);
+      // -inf only while every key so far was masked (bad block ids): then
+      // every weight is 0 and the state stays empty.
+      const float mb = mn == -INFINITY ? 0.f : mn;
+      alpha[r] = exp2f(m_run[r] - mb);
       float sum = 0.f;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          sc[nt][2 * r + e] = exp2f(sc[nt][2 * r + e] - mn);
+          sc[nt][2 * r + e] = exp2f(sc[nt][2 * r + e] - mb);
           sum += sc[nt][2 * r + e];
         }
       l_run[r] = l_run[r] * alpha[r] + sum;
@@ -267,7 +282,8 @@ __global__ void __launch_bounds__(kPrefixThreads, 1)
       const uint32_t pa2 = pack2<kBf16>(sc[2 * blk + 1][0], sc[2 * blk + 1][1]);
       const uint32_t pa3 = pack2<kBf16>(sc[2 * blk + 1][2], sc[2 * blk + 1][3]);
       const uint32_t tv = vb + blk * kTileBytes;
-      const bool live = blk * kBlockTokens < nv;  // whole blocks only (plen % 16 == 0)
+      // Whole blocks only (plen % 16 == 0); a bad block holds no token either.
+      const bool live = blk * kBlockTokens < nv && !((bad >> blk) & 1u);
 #pragma unroll
       for (int nd2 = 0; nd2 < D / 16; ++nd2) {
         const int tok = (mi & 1) * 8 + rr;

@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tab_next = tab_entry((s_begin + s + 8) * kTcBlocks + lane);
       }
       int phys = __shfl_sync(0xffffffffu, tab_cur, (s & 7) * kTcBlocks + blk);
-      if (phys < 0 || phys >= p.num_blocks) {
+      if (phys < 0 || phys >= p.num_blocks) {  // copied from block 0; the softmax masks its keys
         flag_error(PKV_DEVERR_BLOCK_ID);
         phys = 0;
       }
@@ -504,7 +504,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(lg * 32) << 16);
       const float sc = fabsf(p.scale_log2);
       float l_half = 0.f;
+      // Block ids of this half's two blocks, read one stage ahead: a block
+      // whose id is outside the pool contributes no key (its copy read block
+      // 0, whose scores are masked here).
+      auto half_ids = [&](int s, int& a, int& b) {
+        const int j = (s_begin + s) * kTcBlocks + 2 * hf;
+        a = j < n_prefix_blocks ? __ldg(tab + j) : 0;
+        b = j + 1 < n_prefix_blocks ? __ldg(tab + j + 1) : 0;
+      };
+      int id_next0 = 0, id_next1 = 0;
+      if (n_stages > 0) half_ids(0, id_next0, id_next1);
       for (int s = 0; s < n_stages; ++s) {
+        const int id0 = id_next0, id1 = id_next1;
+        if (s + 1 < n_stages) half_ids(s + 1, id_next0, id_next1);
         const int sb = s % kTcSBufs;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[sb], (s / kTcSBufs) & 1, abort_flag,
                                                                 kWaitLimitNs));
@@ -521,17 +533,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
 
-        // Scores past the prefix (only in the last stage) are masked.
+        // Scores past the prefix (only in the last stage) and those of a bad
+        // block are masked: bit i of `keep` is this half's score i.
         const int live = min(kTcKeys, plen - (s_begin + s) * kTcKeys) - hf * 32;
-        if (live < 32) {
+        uint32_t keep = live >= 32 ? 0xffffffffu : live <= 0 ? 0u : (1u << live) - 1u;
+        if (id0 < 0 || id0 >= p.num_blocks) keep &= 0xffff0000u;
+        if (id1 < 0 || id1 >= p.num_blocks) keep &= 0x0000ffffu;
+        if (keep != 0xffffffffu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = i < live ? x[i] : -INFINITY;
+          for (int i = 0; i < 32; ++i) x[i] = ((keep >> i) & 1u) ? x[i] : -INFINITY;
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 32; i += 2) mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], x[i], x[i + 1]);
         float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        mx = live > 0 ? mx * sc : -INFINITY;  // the maximum of the scaled scores (sc >= 0)
+        mx = keep != 0u ? mx * sc : -INFINITY;  // the maximum of the scaled scores (sc >= 0)
         red_max[((s & 1) * 2 + hf) * kTcRows + r] = mx;
         named_bar_sync(2 + lg, 64);
         mx = fmaxf(mx, red_max[((s & 1) * 2 + (hf ^ 1)) * kTcRows + r]);  // the row's maximum, same in both
@@ -572,9 +588,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; i += 2) f2_unpack(f2_fma(f2_pack(x[i], x[i + 1]), sc2, nm2), x[i], x[i + 1]);
         }
-        if (live < 32) {
+        if (keep != 0xffffffffu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = i < live ? x[i] : -INFINITY;
+          for (int i = 0; i < 32; ++i) x[i] = ((keep >> i) & 1u) ? x[i] : -INFINITY;
         }
         uint64_t sum2[2] = {0ull, 0ull};
         uint32_t pw[16];  // this half's 32 probabilities as 16-bit pairs

@@ -25,7 +25,8 @@ def bits(t: torch.Tensor) -> torch.Tensor:
 
 
 def run_gpu(w, num_units: int = 0, force_simt: bool = False, check_errors: bool = True,
-            return_cache: bool = False, workspace=None, balance_chunks: int = 0, static_permille: int = 0):
+            return_cache: bool = False, workspace=None, balance_chunks: int = 0, static_permille: int = 0,
+            **hooks):
     dev = torch.device("cuda")
     kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
     if w.appended:
@@ -33,7 +34,7 @@ def run_gpu(w, num_units: int = 0, force_simt: bool = False, check_errors: bool 
     out = pkv.paged_attention_decode(w.q.to(dev), kc, vc, w.block_tables.to(dev), w.context_lens.to(dev),
                                      w.scale, num_units=num_units, force_simt=force_simt,
                                      workspace=workspace, balance_chunks=balance_chunks,
-                                     static_permille=static_permille)
+                                     static_permille=static_permille, **hooks)
     torch.cuda.synchronize()
     if check_errors:
         assert pkv.pkv_get_device_error() == 0
@@ -80,3 +81,26 @@ def check_workload(w, rows=None, **kw):
     ref, okc, ovc = oracle.workload_decode(w, rows=rows)
     assert torch.equal(bits(kc), bits(okc)) and torch.equal(bits(vc), bits(ovc)), "append not bit-exact"
     return assert_close(out, ref, w.dtype, rows=rows, what=w.name)
+
+
+def drop_blocks(w, drop: dict, **overrides):
+    """The same workload with logical blocks ``drop[b]`` (a list of block
+    indices) removed from sequence b's table and context: attention over the
+    remaining keys.  The expected result of a decode whose table names those
+    blocks with out-of-range ids (their tokens are left out)."""
+    import copy
+    m = copy.copy(w)
+    bt = w.block_tables.clone()
+    cl = w.context_lens.clone()
+    for b, js in drop.items():
+        n = int(cl[b])
+        keep = [j for j in range((n + 15) // 16) if j not in set(js)]
+        removed = sum(min(16, n - 16 * j) for j in js)
+        row = torch.full((bt.shape[1],), -1, dtype=torch.int32)
+        row[: len(keep)] = w.block_tables[b, keep]
+        bt[b] = row
+        cl[b] = n - removed
+    m.block_tables, m.context_lens = bt, cl
+    for k, v in overrides.items():
+        setattr(m, k, v)
+    return m

@@ -81,8 +81,9 @@ def test_decode_ex_rejects_bad_options(lib):
     st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
                                        None, 0, None, ctypes.byref(opts))
     assert st == INVALID
-    for bad in (dict(reserved=(ctypes.c_int32 * 4)(0, 0, 1, 0)), dict(balance_chunks=5), dict(balance_chunks=-1),
-                dict(static_permille=100), dict(static_permille=1000)):
+    for bad in (dict(reserved=(ctypes.c_int32 * 2)(0, 1)), dict(balance_chunks=5), dict(balance_chunks=-1),
+                dict(static_permille=100), dict(static_permille=1000), dict(wait_limit_us=-5),
+                dict(test_withhold_unit=-2)):
         opts = pkv._Options(**bad)
         st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
                                            None, 0, None, ctypes.byref(opts))

@@ -18,7 +18,8 @@ def run_bench(*args, env_extra=None):
 
 
 def test_reference_arm_prints_one_contract_line():
-    r = run_bench("--impl", "reference", "--steps", "3", "--warmup", "3", "--ref-seqs", "2")
+    r = run_bench("--impl", "reference", "--steps", "3", "--warmup", "3", "--workload", "llama3_8b_gqa",
+                  "--ref-units", "4")
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
     assert len(lines) == 1
@@ -38,7 +39,7 @@ def test_reference_arm_prints_one_contract_line():
 
 
 def test_reference_arm_other_ranks_exit_without_work():
-    r = run_bench("--impl", "reference", "--steps", "3", "--warmup", "3", "--ref-seqs", "2",
+    r = run_bench("--impl", "reference", "--steps", "3", "--warmup", "3", "--ref-units", "1",
                   env_extra={"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
@@ -48,3 +49,12 @@ def test_warmup_below_three_is_rejected():
     r = run_bench("--impl", "reference", "--steps", "3", "--warmup", "2")
     assert r.returncode != 0
     assert "warmup" in r.stderr
+
+
+def test_default_workload_is_the_long_context_shape():
+    # The headline: the largest single-GPU shape, 4 x 131,072 tokens.
+    r = run_bench("--impl", "reference", "--steps", "3", "--warmup", "3", "--ref-units", "1")
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["config"]["workload"].startswith("long_ctx_128k") and "131072" in d["config"]["workload"]
+    assert d["dtype"] == "f64" and d["value"] > 0

@@ -7,7 +7,7 @@ import torch
 import oracle
 import paged_kv_cache_386_b200 as pkv
 import workloads as W
-from tests.gpu_helpers import assert_close, bits, sample_rows
+from tests.gpu_helpers import assert_close, bits, drop_blocks, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -168,3 +168,20 @@ def test_cascade_fp16_tensor_memory_kernel(splits):
     out = run_cascade(w, prefix_kernel=1, prefix_splits=splits)
     ref, _, _ = oracle.workload_decode(w)
     assert_close(out, ref, w.dtype, what=f"fp16 splits={splits}")
+
+
+# Out-of-range ids in a shared prefix table: both prefix kernels copy nothing
+# useful for those blocks, mask their keys and set the flag; the result is
+# attention over the remaining tokens (the oracle without those blocks).
+@pytest.mark.parametrize("kernel,splits", [(1, 1), (1, 2), (2, 0)])
+def test_cascade_bad_prefix_block_is_left_out(kernel, splits):
+    w = W.shared_prefix(n_seqs=6, prefix=256, suffix=(10, 80), seed=55)
+    cv = W.cascade_view(w)
+    drop = [2, 9, 15]   # inside the first stage, inside a later one, the prefix's last block
+    ref, _, _ = oracle.workload_decode(drop_blocks(w, {b: drop for b in range(w.batch)}))
+    cv.prefix_block_tables[0, 2] = w.num_blocks
+    cv.prefix_block_tables[0, 9] = -1
+    cv.prefix_block_tables[0, 15] = 1 << 30
+    out = run_cascade(w, cv, check_errors=False, prefix_kernel=kernel, prefix_splits=splits)
+    assert pkv.pkv_get_device_error() & pkv.DEVERR_BLOCK_ID
+    assert_close(out, ref, w.dtype, what=f"bad prefix blocks, kernel {kernel}")

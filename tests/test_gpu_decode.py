@@ -8,7 +8,7 @@ import torch
 import oracle
 import paged_kv_cache_386_b200 as pkv
 import workloads as W
-from tests.gpu_helpers import assert_close, bits, check_workload, run_gpu, sample_rows
+from tests.gpu_helpers import assert_close, bits, check_workload, drop_blocks, run_gpu, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -41,10 +41,18 @@ FULL = {
 }
 
 
+# Rows compared with the oracle: every row of the long-context shape (4 x 64;
+# each of its 46-piece split contexts is then checked in full), 512 of the
+# Llama-3-8B and Llama-2-7B shapes, 128 of the shared-prefix ones.
+FULL_ROWS = {"long_ctx_128k": None, "llama3_8b_gqa": 512, "llama2_7b_mha": 512,
+             "shared_prefix_70b": 128, "best_of_8": 128}
+
+
 @pytest.mark.parametrize("name", list(FULL))
 def test_full_size_configs_sampled(name):
     w = FULL[name]()
-    check_workload(w, rows=sample_rows(w, 24 if name == "long_ctx_128k" else 96))
+    n = FULL_ROWS[name]
+    check_workload(w, rows=None if n is None else sample_rows(w, n))
 
 
 # --- head shapes, dtypes, paths ---
@@ -273,12 +281,44 @@ def test_explicit_workspace_and_too_small_workspace():
 
 # --- device-side range checks (no trap; a flag and a defined result) ---
 
-def test_bad_block_id_sets_flag():
-    w = W.build_workload("badblk", [40, 40], 4, 4, 64, torch.bfloat16, seed=25, append=False)
-    w.block_tables[1, 1] = w.num_blocks + 5
-    run_gpu(w, check_errors=False)
+# A block table entry outside the pool: nothing is read from it, its tokens
+# are left out of the softmax (a row left with no token is a zero row), and
+# the flag is set.  The oracle of the same workload without those blocks
+# gives the expected result.
+@pytest.mark.parametrize("simt,units", [(False, 0), (False, 7), (True, 0), (True, 7)])
+def test_bad_block_id_is_left_out_and_flagged(simt, units):
+    w = W.build_workload("badblk", [40, 300, 200, 20, 129], 8, 2, 128, torch.bfloat16, seed=25, append=False)
+    bad = {0: [1], 1: [3, 7, 18], 2: [0], 3: [0, 1], 4: [8]}   # middle, first, every and last (partial) blocks
+    ref, _, _ = oracle.workload_decode(drop_blocks(w, bad))
+    for b, js in bad.items():
+        for i, j in enumerate(js):
+            w.block_tables[b, j] = w.num_blocks + 5 if i % 2 == 0 else -3
+    out = run_gpu(w, check_errors=False, force_simt=simt, num_units=units)
     assert pkv.pkv_get_device_error() & pkv.DEVERR_BLOCK_ID
     assert pkv.pkv_get_device_error() == 0   # read clears
+    assert torch.equal(out[3], torch.zeros_like(out[3]))   # every block bad: a zero row
+    assert_close(out, ref, w.dtype, what=f"bad block ids simt={simt} units={units}")
+
+
+# The failure path of the bounded waits: unit 3's copies are never issued, so
+# its consumer's wait (10 ms here) runs out.  The launch must return with the
+# timeout bit set (every thread reaches the grid barrier), and the next call
+# with default settings must be clean and right.
+@pytest.mark.parametrize("simt", [False, True])
+def test_bounded_wait_runs_out_and_the_next_call_is_clean(simt):
+    w = W.uniform_gqa(batch=8, len_lo=200, len_hi=2000, seed=27)
+    ref, _, _ = oracle.workload_decode(w)
+    run_gpu(w, check_errors=False, force_simt=simt, wait_limit_us=10000, test_withhold_unit=3)
+    assert pkv.pkv_get_device_error() & pkv.DEVERR_TIMEOUT
+    out = run_gpu(w, force_simt=simt)
+    assert_close(out, ref, w.dtype, what=f"after a timed-out launch, simt={simt}")
+
+
+def test_withhold_hook_rejects_negative_values():
+    w = W.build_workload("neg", [20], 4, 4, 64, torch.bfloat16, seed=28, append=False)
+    with pytest.raises(pkv.PagedKVError) as e:
+        run_gpu(w, wait_limit_us=-1)
+    assert e.value.status == 1
 
 
 def test_context_beyond_table_sets_flag():
