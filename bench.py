@@ -203,7 +203,12 @@ def run_ours(args) -> None:
     tr = layout.decode_traffic(w.block_tables, w.context_lens, w.n_q_heads, w.n_kv_heads, w.head_dim, es,
                                kv_int8=int8)
     kv_bytes = tr["kv_unique"]
-    decode_bytes = tr["total_unique"]
+    # The plain 16-bit decode step runs as one launch, the append fused into
+    # the decode (paged_kv_append_and_decode); --separate-append times the
+    # two calls instead.
+    fused = not (int8 or mq or args.cascade or args.separate_append)
+    decode_bytes = tr["total_unique"] + (layout.append_traffic(w.k_new.shape[0], w.n_kv_heads, w.head_dim, es)
+                                         if fused else 0)
 
     # Device copies of the whole problem.
     kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
@@ -232,13 +237,18 @@ def run_ours(args) -> None:
                                                             w.dtype), dtype=torch.uint8, device=dev)
 
     def append(stream_=None):
+        if fused:
+            return  # inside the decode launch
         if int8:
             pkv.paged_kv_append_int8(k_new, v_new, slots, kv8, stream=stream_)
         else:
             pkv.paged_kv_append(k_new, v_new, slots, kc, vc, stream=stream_)
 
     def decode(stream_=None):
-        if mq:
+        if fused:
+            pkv.paged_kv_append_and_decode(q, k_new, v_new, slots, kc, vc, bt, cl, w.scale, out=out, workspace=ws,
+                                           stream=stream_)
+        elif mq:
             pkv.paged_attention_decode_mq(q, kc, vc, bt, cl, w.scale, out=out, workspace=ws, stream=stream_)
         elif int8:
             pkv.paged_attention_decode_int8(q, kv8, bt, cl, w.scale, out=out, workspace=ws, stream=stream_)
@@ -298,7 +308,8 @@ def run_ours(args) -> None:
                 flush_l2(1)
                 g.replay()
             torch.cuda.synchronize(dev)
-            launch_note = "CUDA graph of the step (append + decode)"
+            launch_note = ("CUDA graph of the step (one launch: the append fused into the decode)" if fused
+                           else "CUDA graph of the step (append + decode)")
         except Exception as e:  # capture unsupported: time direct calls
             torch.cuda.synchronize(dev)
             g, launch_note = None, f"direct C-ABI calls (graph capture failed: {type(e).__name__})"
@@ -408,6 +419,8 @@ def run_ours(args) -> None:
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
     def append_set(ins, cache, s_):
+        if fused:
+            return
         if int8:
             pkv.paged_kv_append_int8(ins[1], ins[2], ins[3], cache[0], stream=s_)
         else:
@@ -415,7 +428,10 @@ def run_ours(args) -> None:
 
     def decode_set(ins, cache, o, s_):
         q_ = ins[0]
-        if args.cascade:
+        if fused:
+            pkv.paged_kv_append_and_decode(q_, ins[1], ins[2], ins[3], cache[0], cache[1], ins[4], ins[5], w.scale,
+                                           out=o, workspace=ws, stream=s_)
+        elif args.cascade:
             pkv.paged_attention_decode_cascade(q_, cache[0], cache[1], *ins[4:9], w.scale, out=o, workspace=ws,
                                                stream=s_)
         elif mq:
@@ -474,6 +490,7 @@ def run_ours(args) -> None:
             # cache format, seed and placement must all match.
             if (prof.get("kernel_hash") == kernel_hash() and prof.get("workload") == args.workload
                     and prof.get("kv", "16-bit") == ("int8" if int8 else "16-bit") and not args.cascade and not mq
+                    and bool(prof.get("fused", False)) == fused
                     and prof.get("seed", 0) == args.seed and prof.get("placement", "shuffle") == args.placement):
                 traffic = prof.get("dram_bytes_per_launch")
     except Exception:
@@ -506,6 +523,7 @@ def run_ours(args) -> None:
             "roofline": {"bound": "hbm",
                          "kernel": ("paged_attention_decode_cascade (pkv_prefix_tc_kernel + pkv_decode_kernel)"
                                     if args.cascade else
+                                    "paged_kv_append_and_decode (pkv_decode_kernel, append fused)" if fused else
                                     "paged_attention_decode_int8 (pkv_decode_kernel, INT8)" if int8 else
                                     "paged_attention_decode_mq (pkv_decode_kernel, several queries)" if mq
                                     else "paged_attention_decode (pkv_decode_kernel)"),
@@ -523,7 +541,7 @@ def run_ours(args) -> None:
                     "serial_h2d_bytes_per_step": h2d,
                     "serial_value": round(e2e_serial_value, 2),
                     "serial_ms_per_step": round(e2e_serial_s / args.steps * 1e3, 4)},
-            "gpu_launches": (3 if args.cascade else 2) * args.steps,
+            "gpu_launches": (3 if args.cascade else 1 if fused else 2) * args.steps,
             "clocks": clocks.summary(),
             "wall_s_timed_loop": round(wall, 4),
         }
@@ -679,6 +697,9 @@ def main(argv=None) -> None:
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of a CUDA graph replay")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="run the step as paged_kv_append + paged_attention_decode (two launches) instead of "
+                         "the fused paged_kv_append_and_decode")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample SM clocks during the timed region")
     ap.add_argument("--cascade", action="store_true",
                     help="decode shared-prefix workloads with paged_attention_decode_cascade")

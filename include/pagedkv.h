@@ -164,6 +164,33 @@ pkv_status paged_attention_decode(const void* q, const void* k_cache, const void
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * paged_kv_append_and_decode -- one decode step in one launch: the result of
+ * paged_kv_append(k, v, slot_mapping, num_tokens, k_cache, v_cache, ...)
+ * followed by paged_attention_decode(q, k_cache, v_cache, ...) on the same
+ * stream, bit for bit, in the cache and in `out` ("Transformer anatomy"
+ * ch. 15 §15.1: the new token's K and V join the cache, then its query
+ * attends over all of it; §15.5: the new token goes into its slot of the
+ * current block).
+ *
+ * Every CTA of the decode kernel first writes its share of the new rows into
+ * their slots (a negative slot is skipped; one >= num_blocks * block_size is
+ * skipped and sets PKV_DEVERR_SLOT); a grid-wide barrier then orders those
+ * writes before the first K/V tile is read.  This saves the separate append
+ * launch and the gap between the two kernels.  Arguments are those of the
+ * two calls (k, v: [num_tokens][n_kv_heads][head_dim] of `dtype`); the
+ * workspace rules are paged_attention_decode's.  batch == 0 runs the append
+ * alone.
+ */
+pkv_status paged_kv_append_and_decode(const void* q, const void* k, const void* v,
+                                      const int64_t* slot_mapping, int32_t num_tokens, void* k_cache,
+                                      void* v_cache, const int32_t* block_tables,
+                                      int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                      int32_t batch, int32_t num_blocks, float scale, int32_t n_q_heads,
+                                      int32_t n_kv_heads, int32_t head_dim, int32_t block_size, void* out,
+                                      pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
+/*
  * paged_attention_decode_cascade -- paged_attention_decode for batches whose
  * sequences share prefix blocks (prefix caching: sequences that start with the
  * same block-aligned tokens point their tables at the same physical blocks,

@@ -22,7 +22,7 @@ from pathlib import Path
 import torch
 
 __all__ = [
-    "paged_kv_append", "paged_attention_decode", "paged_attention_decode_noalloc",
+    "paged_kv_append", "paged_attention_decode", "paged_kv_append_and_decode", "paged_attention_decode_noalloc",
     "paged_attention_decode_cascade", "paged_attention_cascade_workspace_size",
     "paged_attention_workspace_size", "paged_kv_copy_blocks", "BlockManager", "pkv_bm_hash_blocks",
     "paged_kv_append_int8", "paged_attention_decode_int8", "int8_cache",
@@ -94,6 +94,9 @@ def _load() -> ctypes.CDLL:
     lib.paged_attention_decode.restype = ctypes.c_int
     lib.paged_attention_decode_ex.argtypes = dec + [ctypes.POINTER(_Options)]
     lib.paged_attention_decode_ex.restype = ctypes.c_int
+    lib.paged_kv_append_and_decode.argtypes = [p, p, p, p, i32, p, p, p, i32, p, i32, i32, f32, i32, i32, i32, i32,
+                                               p, ctypes.c_int, p, sz, p]
+    lib.paged_kv_append_and_decode.restype = ctypes.c_int
     lib.paged_attention_cascade_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(sz)]
     lib.paged_attention_cascade_workspace_size.restype = ctypes.c_int
     lib.paged_attention_decode_cascade.argtypes = [p, p, p, i32, p, i32, p, p, p, i32, p, i32, i32, f32, i32, i32,
@@ -256,6 +259,37 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
             _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
             B, num_blocks, float(scale), n_q, n_kv, d, bs, _dev(out, "out"), _DTYPE[q.dtype],
             ws_ptr, ws_bytes, _stream(stream, q.device), ctypes.byref(opts)), "paged_attention_decode")
+    return out
+
+
+def paged_kv_append_and_decode(q, k, v, slot_mapping, k_cache, v_cache, block_tables, context_lens, scale: float,
+                               out=None, workspace=None, block_size: int = 16, stream=None):
+    """paged_kv_append(k, v, slot_mapping, ...) then paged_attention_decode(q,
+    ...) in one launch (the caches are written in place); returns ``out``."""
+    lib = _load()
+    B, n_q, d = q.shape
+    num_blocks, n_kv, bs, d2 = k_cache.shape
+    if d2 != d or bs != block_size or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if k.dtype != q.dtype or v.dtype != q.dtype or slot_mapping.dtype != torch.int64:
+        raise ValueError("k and v must have q's dtype, slot_mapping int64")
+    if tuple(k.shape[1:]) != (n_kv, d) or tuple(v.shape) != tuple(k.shape) or slot_mapping.shape[0] != k.shape[0]:
+        raise ValueError("k, v must be [num_tokens, n_kv_heads, head_dim] and slot_mapping [num_tokens]")
+    if out is None:
+        out = torch.empty_like(q)
+    _check_decode_io(q, k_cache, v_cache, out, k, v, slot_mapping, block_tables, context_lens, workspace)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _check(lib.paged_kv_append_and_decode(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping"), k.shape[0],
+            _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables"),
+            block_tables.shape[1], _dev(context_lens, "context_lens"), B, num_blocks, float(scale), n_q, n_kv, d,
+            bs, _dev(out, "out"), _DTYPE[q.dtype], ws_ptr, ws_bytes, _stream(stream, q.device)),
+            "paged_kv_append_and_decode")
     return out
 
 

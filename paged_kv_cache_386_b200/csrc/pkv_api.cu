@@ -159,10 +159,10 @@ pkv_status encode_cache_map_tile(CUtensorMap* map, const void* cache, pkv_dtype 
 
 // The decode kernel is launched cooperatively: its CTAs (at most one per SM)
 // are guaranteed to be co-resident, which its grid-wide barrier needs.
-template <int DT, int D, int GPAD, bool kI8 = false, bool kMQ = false>
+template <int DT, int D, int GPAD, bool kI8 = false, bool kMQ = false, bool kFused = false>
 pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid, size_t smem,
                          cudaStream_t stream) {
-  auto kern = pkv_decode_kernel<DT, D, GPAD, kI8, kMQ>;
+  auto kern = pkv_decode_kernel<DT, D, GPAD, kI8, kMQ, kFused>;
   // Opt in to the largest dynamic shared memory once per device (the launch
   // itself passes the size it needs).
   static bool opted_in[kMaxDevices] = {};
@@ -189,18 +189,26 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const Dec
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+template <int DT, int D, bool kFused>
+pkv_status dispatch_gpad_f(int gpad, const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid,
+                           size_t smem, cudaStream_t stream) {
+  if constexpr (DT == kF32) {
+    return launch_decode<DT, D, 0, false, false, kFused>(mk, mv, p, grid, smem, stream);
+  } else {
+    switch (gpad) {
+      case 0: return launch_decode<DT, D, 0, false, false, kFused>(mk, mv, p, grid, smem, stream);
+      case 8: return launch_decode<DT, D, 8, false, false, kFused>(mk, mv, p, grid, smem, stream);
+      default: return launch_decode<DT, D, 16, false, false, kFused>(mk, mv, p, grid, smem, stream);
+    }
+  }
+}
+
+// The plain decode, or with the new tokens' append fused in front of it.
 template <int DT, int D>
 pkv_status dispatch_gpad(int gpad, const CUtensorMap& mk, const CUtensorMap& mv, const DecodeParams& p, int grid,
                          size_t smem, cudaStream_t stream) {
-  if constexpr (DT == kF32) {
-    return launch_decode<DT, D, 0>(mk, mv, p, grid, smem, stream);
-  } else {
-    switch (gpad) {
-      case 0: return launch_decode<DT, D, 0>(mk, mv, p, grid, smem, stream);
-      case 8: return launch_decode<DT, D, 8>(mk, mv, p, grid, smem, stream);
-      default: return launch_decode<DT, D, 16>(mk, mv, p, grid, smem, stream);
-    }
-  }
+  return p.app.total > 0 ? dispatch_gpad_f<DT, D, true>(gpad, mk, mv, p, grid, smem, stream)
+                         : dispatch_gpad_f<DT, D, false>(gpad, mk, mv, p, grid, smem, stream);
 }
 
 template <int DT>
@@ -347,6 +355,36 @@ pkv_status launch_prefix_tc(const CUtensorMap& mk, const CUtensorMap& mv, const 
 }  // namespace
 }  // namespace pkv
 
+namespace pkv {
+namespace {
+// Checks of paged_kv_append's arguments and its kernel parameters.
+pkv_status append_params(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                         void* k_cache, void* v_cache, int32_t num_blocks, int32_t block_size, int32_t n_kv_heads,
+                         int32_t head_dim, pkv_dtype dtype, AppendParams* p) {
+  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || n_kv_heads <= 0 || head_dim <= 0)
+    return PKV_ERR_INVALID_ARG;
+  const int es = elem_bytes(dtype);
+  if (es == 0 || block_size != kBlockTokens || (head_dim * es) % 16 != 0) return PKV_ERR_UNSUPPORTED;
+  *p = {};
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PKV_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return PKV_ERR_INVALID_ARG;
+  p->k = static_cast<const uint8_t*>(k);
+  p->v = static_cast<const uint8_t*>(v);
+  p->slot_mapping = slot_mapping;
+  p->k_cache = static_cast<uint8_t*>(k_cache);
+  p->v_cache = static_cast<uint8_t*>(v_cache);
+  p->num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  p->n_kv_heads = n_kv_heads;
+  p->row_chunks = head_dim * es / 16;
+  p->total = static_cast<int64_t>(num_tokens) * n_kv_heads * p->row_chunks;
+  return PKV_OK;
+}
+}  // namespace
+}  // namespace pkv
+
 using namespace pkv;
 
 extern "C" {
@@ -370,27 +408,12 @@ const char* pkv_status_string(pkv_status s) {
 pkv_status paged_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
                            void* k_cache, void* v_cache, int32_t num_blocks, int32_t block_size,
                            int32_t n_kv_heads, int32_t head_dim, pkv_dtype dtype, void* stream) {
-  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || n_kv_heads <= 0 || head_dim <= 0)
-    return PKV_ERR_INVALID_ARG;
-  const int es = elem_bytes(dtype);
-  if (es == 0 || block_size != kBlockTokens || (head_dim * es) % 16 != 0) return PKV_ERR_UNSUPPORTED;
-  if (num_tokens == 0) return PKV_OK;
-  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PKV_ERR_INVALID_ARG;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
-      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
-    return PKV_ERR_INVALID_ARG;
+  AppendParams p;
+  const pkv_status st = append_params(k, v, slot_mapping, num_tokens, k_cache, v_cache, num_blocks, block_size,
+                                      n_kv_heads, head_dim, dtype, &p);
+  if (st != PKV_OK || num_tokens == 0) return st;
   DeviceInfo di;
   if (device_info(&di) != PKV_OK) return PKV_ERR_CUDA;
-  AppendParams p;
-  p.k = static_cast<const uint8_t*>(k);
-  p.v = static_cast<const uint8_t*>(v);
-  p.slot_mapping = slot_mapping;
-  p.k_cache = static_cast<uint8_t*>(k_cache);
-  p.v_cache = static_cast<uint8_t*>(v_cache);
-  p.num_slots = static_cast<int64_t>(num_blocks) * block_size;
-  p.n_kv_heads = n_kv_heads;
-  p.row_chunks = head_dim * es / 16;
-  p.total = static_cast<int64_t>(num_tokens) * n_kv_heads * p.row_chunks;
   const int64_t want = (p.total + 255) / 256;
   const int grid = static_cast<int>(want < int64_t(di.sm_count) * 8 ? want : int64_t(di.sm_count) * 8);
   pkv_append_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
@@ -498,7 +521,8 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
                        float scale, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
                        void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes, void* stream,
                        const pkv_decode_options* options, const float* init, const int32_t* seq_group,
-                       int32_t n_groups, const KvI8* i8 = nullptr, int32_t q_len = 1) {
+                       int32_t n_groups, const KvI8* i8 = nullptr, int32_t q_len = 1,
+                       const AppendParams* app = nullptr) {
   pkv_status st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                     num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
   if (st != PKV_OK) return st;
@@ -605,6 +629,8 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
   p.n_groups = n_groups;
   p.wait_limit_ns = opt.wait_limit_us > 0 ? static_cast<uint64_t>(opt.wait_limit_us) * 1000u : kWaitLimitNs;
   p.withhold_unit = opt.test_withhold_unit - 1;
+  p.app = {};
+  if (app) p.app = *app;
 
   if (st == PKV_OK && mq) {
     st = dtype == PKV_F16 ? dispatch_mq<kF16>(head_dim, gpad, mk, mv, p, grid, smem, s)
@@ -646,6 +672,28 @@ pkv_status paged_attention_decode(const void* q, const void* k_cache, const void
   return paged_attention_decode_ex(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch,
                                    num_blocks, scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype,
                                    workspace, workspace_bytes, stream, nullptr);
+}
+
+pkv_status paged_kv_append_and_decode(const void* q, const void* k, const void* v, const int64_t* slot_mapping,
+                                      int32_t num_tokens, void* k_cache, void* v_cache,
+                                      const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* context_lens, int32_t batch, int32_t num_blocks, float scale,
+                                      int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, int32_t block_size,
+                                      void* out, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  AppendParams app;
+  pkv_status st = append_params(k, v, slot_mapping, num_tokens, k_cache, v_cache, num_blocks, block_size,
+                                n_kv_heads, head_dim, dtype, &app);
+  if (st != PKV_OK) return st;
+  st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks,
+                         scale, n_q_heads, n_kv_heads, head_dim, block_size, out, dtype);
+  if (st != PKV_OK) return st;
+  if (batch == 0)  // no decode: the append alone
+    return paged_kv_append(k, v, slot_mapping, num_tokens, k_cache, v_cache, num_blocks, block_size, n_kv_heads,
+                           head_dim, dtype, stream);
+  return decode_impl(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, batch, num_blocks, scale,
+                     n_q_heads, n_kv_heads, head_dim, block_size, out, dtype, workspace, workspace_bytes, stream,
+                     nullptr, nullptr, nullptr, 0, nullptr, 1, &app);
 }
 
 pkv_status paged_attention_decode_int8(const void* q, const uint8_t* kv_cache, const int32_t* block_tables,

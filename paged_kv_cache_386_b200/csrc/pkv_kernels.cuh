@@ -90,9 +90,10 @@ struct AppendParams {
   int32_t row_chunks;  // 16-byte chunks per head row
 };
 
-__global__ void __launch_bounds__(256) pkv_append_kernel(const AppendParams p) {
-  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < p.total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
+// Chunks idx = start, start + stride, ... of the append: one 16-byte chunk
+// of one head row of one token per index.
+__device__ __forceinline__ void append_range(const AppendParams& p, int64_t start, int64_t stride) {
+  for (int64_t idx = start; idx < p.total; idx += stride) {
     const int c = static_cast<int>(idx % p.row_chunks);
     const int64_t th = idx / p.row_chunks;  // token * n_kv + head
     const int h = static_cast<int>(th % p.n_kv_heads);
@@ -111,6 +112,10 @@ __global__ void __launch_bounds__(256) pkv_append_kernel(const AppendParams p) {
     *reinterpret_cast<int4*>(p.k_cache + dst) = kv;
     *reinterpret_cast<int4*>(p.v_cache + dst) = vv;
   }
+}
+
+__global__ void __launch_bounds__(256) pkv_append_kernel(const AppendParams p) {
+  append_range(p, blockIdx.x * (int64_t)blockDim.x + threadIdx.x, (int64_t)gridDim.x * blockDim.x);
 }
 
 // ---------------------------------------------------------------------------
@@ -296,6 +301,10 @@ struct DecodeParams {
   float scale_log2;    // scale * log2(e)
   uint64_t wait_limit_ns;  // bound of every in-kernel wait
   int32_t withhold_unit;   // test hook: this unit's producer lane issues nothing (-1: none)
+  // Fused append (paged_kv_append_and_decode): the new tokens' K and V are
+  // written into their slots by every CTA before any tile is read (app.total
+  // = 0: none).
+  AppendParams app;
 };
 
 // Row `row` of segment (b, hg) -- query row / gp, head hg * gp + row % gp
@@ -1162,35 +1171,52 @@ __device__ __forceinline__ void q_fetch(uint8_t* qbuf, const DecodeParams& p, in
   cp_async_commit();
 }
 
-// Phase 2 of the decode kernel: one warp merges query head g of the split
-// segment whose first piece chunk u holds (mt = meta[u]); the pieces are held
-// by chunks u..u_hi (chunks are never empty) and are combined in chunk (tile)
-// order as
+// Phase 2 of the decode kernel: one warp merges dims [d0, d0 + 32 DPL) of
+// query head g of the split segment whose first piece chunk u holds (mt =
+// meta[u]); the pieces are held by chunks u..u_hi (chunks are never empty)
+// and are combined in chunk (tile) order as
 //   M = max_i m_i,  w_i = 2^(m_i - M),  out = sum_i w_i O_i / sum_i w_i l_i.
-// Lane j holds the scalars of pieces j and j + 32; each lane owns D/32 dims
-// of the numerator and walks the pieces eight loads at a time, the weights
-// broadcast by shuffles.  Reads go to L2 (ld.global.cg): the records were
-// written by other SMs before the grid barrier.
-template <int DT, int D>
-__device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt, int g, int lane) {
+// Lane j holds the scalars of pieces j and j + 32 (pieces beyond 64 are
+// folded in by a plain loop); each lane owns DPL dims of the numerator.  The
+// records are read in batches of PB pieces, the first batch together with
+// the scalars, so that a merge of up to PB pieces costs one round trip to L2
+// (ld.global.cg: the records were written by other SMs before the grid
+// barrier).  With at most 8 pieces and DPL = D / 32 every load of every piece
+// goes out in one round without shuffles.
+template <int DT, int D, int DPL>
+__device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt, int g, int d0, int lane) {
   using T = typename DTypeInfo<DT>::T;
-  constexpr int DPL = D / 32;
+  constexpr int PB = DPL >= 4 ? 8 : (DPL == 2 ? 12 : 24);  // pieces per batch: PB * DPL registers
   const int seg = mt.x, b = seg / p.ng, hg = seg % p.ng, n = mt.y - u + 1;
-  const int mo = p.rows * D + g, lo = p.rows * D + p.rows + g, oo = g * D + lane * DPL;
+  const int mo = p.rows * D + g, lo = p.rows * D + p.rows + g, oo = g * D + d0 + lane * DPL;
   auto rec_of = [&](int j) -> const float* {  // record of piece j (chunk u + j)
     return p.records + (static_cast<size_t>(u + j) * 2 + (j == 0 ? mt.z : 0)) * p.rec_floats;
   };
-  T* const ob = static_cast<T*>(p.out) + out_row(p, b, hg, g) * D + lane * DPL;
+  auto load_o = [&](const float* r, float (&x)[DPL]) {
+    if constexpr (DPL == 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(r + oo));
+      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else if constexpr (DPL == 2) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(r + oo));
+      x[0] = v.x; x[1] = v.y;
+    } else {
+      x[0] = __ldcg(r + oo);
+    }
+  };
+  T* const ob = static_cast<T*>(p.out) + out_row(p, b, hg, g) * D + d0 + lane * DPL;
   auto store = [&](const float (&acc)[DPL], float inv) {
     if constexpr (DPL == 4) {
       store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
     } else if constexpr (DT == kF32) {
-      *reinterpret_cast<float2*>(ob) = make_float2(acc[0] * inv, acc[1] * inv);
-    } else {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) ob[i] = acc[i] * inv;
+    } else if constexpr (DPL == 2) {
       *reinterpret_cast<uint32_t*>(ob) = pack2<DT == kBF16>(acc[0] * inv, acc[1] * inv);
+    } else {
+      ob[0] = static_cast<T>(acc[0] * inv);  // round to nearest even
     }
   };
-  if (n <= 8) {
+  if (DPL * 32 == D && n <= 8) {
     // Common case: every load of every piece issued in one round.
     float mj[8], lj[8], o[8][DPL];
 #pragma unroll
@@ -1198,13 +1224,7 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
       const float* r = rec_of(min(j, n - 1));
       mj[j] = __ldcg(r + mo);
       lj[j] = __ldcg(r + lo);
-      if constexpr (DPL == 4) {
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(r + oo));
-        o[j][0] = x.x; o[j][1] = x.y; o[j][2] = x.z; o[j][3] = x.w;
-      } else {
-        const float2 x = __ldcg(reinterpret_cast<const float2*>(r + oo));
-        o[j][0] = x.x; o[j][1] = x.y;
-      }
+      load_o(r, o[j]);
     }
     float M = -INFINITY;
 #pragma unroll
@@ -1224,8 +1244,6 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
     store(acc, L > 0.f ? 1.f / L : 0.f);
     return;
   }
-  // Scalars of pieces lane and lane + 32; pieces beyond 64 (rare) are folded
-  // in by a plain loop.
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   if (lane < n) {
     m0 = __ldcg(rec_of(lane) + mo);
@@ -1235,6 +1253,9 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
     m1 = __ldcg(rec_of(lane + 32) + mo);
     l1 = __ldcg(rec_of(lane + 32) + lo);
   }
+  float o[PB][DPL];
+#pragma unroll
+  for (int jj = 0; jj < PB; ++jj) load_o(rec_of(min(jj, n - 1)), o[jj]);
   float M = fmaxf(m0, m1);
   for (int j = 64 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(rec_of(j) + mo));
 #pragma unroll
@@ -1249,22 +1270,13 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
   float acc[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-  for (int j0 = 0; j0 < n; j0 += 8) {
-    float o[8][DPL];
+  for (int j0 = 0; j0 < n; j0 += PB) {
+    if (j0 > 0) {
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      const int j = min(j0 + jj, n - 1);
-      const float* r = rec_of(j) + oo;
-      if constexpr (DPL == 4) {
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(r));
-        o[jj][0] = x.x; o[jj][1] = x.y; o[jj][2] = x.z; o[jj][3] = x.w;
-      } else {
-        const float2 x = __ldcg(reinterpret_cast<const float2*>(r));
-        o[jj][0] = x.x; o[jj][1] = x.y;
-      }
+      for (int jj = 0; jj < PB; ++jj) load_o(rec_of(min(j0 + jj, n - 1)), o[jj]);
     }
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
+    for (int jj = 0; jj < PB; ++jj) {
       const int j = j0 + jj;
       float wj = __shfl_sync(0xffffffffu, (j & 32) ? w1 : w0, j & 31);
       if (j >= 64 && j < n) wj = exp2f(__ldcg(rec_of(j) + mo) - M);
@@ -1284,7 +1296,10 @@ __device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt
 // and zero-fills the rows of empty sequences.
 // kI8: the cache holds INT8 records (MmaConsumerI8).  kMQ: q_len > 1
 // queries per sequence (tensor-core consumer with per-row causal limits).
-template <int DT, int D, int GPAD, bool kI8, bool kMQ>
+// kFused: the launch first writes the new tokens of p.app into the cache
+// (paged_kv_append_and_decode); a separate instantiation, so that the plain
+// decode's register allocation does not carry the fused prologue.
+template <int DT, int D, int GPAD, bool kI8, bool kMQ, bool kFused = false>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     pkv_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeParams p) {
@@ -1337,6 +1352,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     tma_prefetch_desc(&tm_v);
   }
 
+  // Fused append: every thread of the grid writes its share of the new
+  // tokens' rows, then arrives on the grid barrier; the wait comes after the
+  // scan below, before any tile is read.  The proxy fence makes the rows,
+  // written through the generic proxy, visible to the TMA reads (async
+  // proxy) that follow the barrier.
+  constexpr bool fused_append = kFused;
+  [[maybe_unused]] unsigned int app_token = 0;
+  if constexpr (fused_append) {
+    append_range(p.app, blockIdx.x * static_cast<int64_t>(kDecodeThreads) + threadIdx.x,
+                 static_cast<int64_t>(gridDim.x) * kDecodeThreads);
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    app_token = cooperative_groups::this_grid().barrier_arrive();
+  }
+
   // Tiles per sequence -> exclusive prefix sums (block-wide scan).
   {
     const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
@@ -1367,7 +1396,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     if (threadIdx.x == kDecodeThreads - 1) prefix[B] = base + incl;
   }
-  __syncthreads();
+  if constexpr (fused_append)
+    cooperative_groups::this_grid().barrier_wait(static_cast<unsigned int&&>(app_token));  // ends with a CTA barrier
+  else
+    __syncthreads();
 
   const int T = prefix[B];
   const Sched sc = make_sched(T, p.num_units, p.sub_chunks, p.static_permille);
@@ -1385,6 +1417,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // is issued, and the claim of the next chunk is sent kClaimAhead tiles
     // before the current chunk's end and read at its last tile, so the warp
     // (whose lanes run in step) never waits on an L2 round trip.
+    if constexpr (fused_append) asm volatile("fence.proxy.async.global;" ::: "memory");
     const int u = blockIdx.x * kConsumerWarps + lane;
     // Test hook: the lane of the withheld unit never issues, so that its
     // consumer's bounded wait runs out (no copy is then in flight for it).
@@ -1631,25 +1664,42 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   {
     constexpr int kWarps = kConsumerWarps + 1;
     const int gw = blockIdx.x * kWarps + warp, n_warps = gridDim.x * kWarps;
-    const int items = n_chunks * p.rows;
     const int n_segs = B * p.ng;
+    // Long split contexts (many pieces per segment, few merges) are merged
+    // by D / 32 warps per query head, one dim per lane, so that more warps
+    // share the merge and each issues all its loads at once.  The choice is
+    // the same in every CTA (T and the schedule are).
+    // (T is re-read from shared memory so that it is not held in a register
+    // through phase 1.)
+    constexpr int kSlices = D / 32;
+    const int T2 = prefix[B];
+    const int Lq2 = T2 / max(1, min(p.num_units, T2));
+    const bool sliced = T2 > 0 && T2 / max(1, n_segs) >= 8 * max(1, Lq2) &&
+                        n_segs * p.rows * kSlices <= n_warps;
+    const int slices = sliced ? kSlices : 1;
+    const int per_chunk = p.rows * slices;
+    const int items = n_chunks * per_chunk;
     // Item metadata is loaded 32 items at a time, lane t for the round's
     // t-th item of this warp.
     for (int base = gw; base < items; base += 32 * n_warps) {
       int4 my_item = make_int4(-1, 0, 0, 0);
       const int i_lane = base + lane * n_warps;
-      if (i_lane < items) my_item = __ldcg(p.meta + i_lane / p.rows);
+      if (i_lane < items) my_item = __ldcg(p.meta + i_lane / per_chunk);
       for (int t = 0; t < 32 && base + t * n_warps < items; ++t) {
         const int i = base + t * n_warps;
-        const int c = i / p.rows;
+        const int c = i / per_chunk, rem = i - c * per_chunk;
         int4 mt;
         mt.x = __shfl_sync(0xffffffffu, my_item.x, t);
         mt.y = __shfl_sync(0xffffffffu, my_item.y, t);
         mt.z = __shfl_sync(0xffffffffu, my_item.z, t);
         // Entries of chunks that an aborted launch never reached may be
         // stale: only well-formed ones are merged.
-        if (mt.x >= 0 && mt.x < n_segs && mt.y > c && mt.y < n_chunks && (mt.z == 0 || mt.z == 1))
-          merge_head<DT, D>(p, c, mt, i % p.rows, lane);
+        if (mt.x >= 0 && mt.x < n_segs && mt.y > c && mt.y < n_chunks && (mt.z == 0 || mt.z == 1)) {
+          if (sliced)
+            merge_head<DT, D, 1>(p, c, mt, rem / kSlices, (rem % kSlices) * 32, lane);
+          else
+            merge_head<DT, D, D / 32>(p, c, mt, rem, 0, lane);
+        }
       }
     }
     // The claim counter must have seen every balancing chunk plus one failed

@@ -34,7 +34,7 @@ def test_header_declares_expected_entry_points():
             "paged_attention_workspace_size", "pkv_get_device_error", "pkv_status_string",
             "pkv_version", "paged_kv_copy_blocks", "paged_attention_workspace_size_ex", "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_hash_blocks",
             "pkv_bm_add_sequence", "pkv_bm_fork", "pkv_bm_append", "pkv_bm_free", "pkv_bm_get_tables",
-            "pkv_bm_stats", "pkv_bm_refcount"} <= names
+            "pkv_bm_stats", "pkv_bm_refcount", "paged_kv_append_and_decode"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -88,6 +88,24 @@ def test_decode_ex_rejects_bad_options(lib):
         st = lib.paged_attention_decode_ex(256, 256, 256, 256, 4, 256, 2, 8, 0.1, 8, 2, 128, 16, 256, 2,
                                            None, 0, None, ctypes.byref(opts))
         assert st == INVALID, bad
+
+
+def test_fused_append_and_decode_host_validation(lib):
+    f = lib.paged_kv_append_and_decode
+    ptr = 256
+
+    def call(q=ptr, k=ptr, v=ptr, sl=ptr, ntok=2, kc=ptr, vc=ptr, bt=ptr, maxb=4, cl=ptr, batch=2, nb=8,
+             scale=0.125, nq=8, nkv=2, d=128, bs=16, out=ptr, dtype=2):
+        return f(q, k, v, sl, ntok, kc, vc, bt, maxb, cl, batch, nb, scale, nq, nkv, d, bs, out, dtype, None, 0, None)
+
+    assert call(ntok=-1) == INVALID                      # the append's checks
+    assert call(k=None) == INVALID
+    assert call(sl=260) == INVALID                       # slot_mapping misaligned
+    assert call(bs=32) == UNSUPPORTED
+    assert call(nq=6, nkv=4) == INVALID                  # the decode's checks
+    assert call(q=8) == INVALID
+    assert call(d=96) == UNSUPPORTED
+    assert call(scale=float("nan")) == INVALID
 
 
 def test_append_host_validation(lib):
