@@ -157,6 +157,55 @@ pkv_status encode_cache_map_tile(CUtensorMap* map, const void* cache, pkv_dtype 
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// Encoded tensor maps, cached per (kind, base address, dtype, shape): a map
+// depends only on those, so a serving loop that calls with the same caches
+// every step pays the encode once.  A small table with least-recently-used
+// replacement, shared by every device and host thread.
+enum MapKind { kMapBox = 0, kMapTile = 1 };
+struct MapKey {
+  const void* base;
+  int kind, dtype, num_blocks, n_kv, head_dim;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && kind == o.kind && dtype == o.dtype && num_blocks == o.num_blocks && n_kv == o.n_kv &&
+           head_dim == o.head_dim;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  uint64_t last_use;  // 0: empty
+};
+constexpr int kMapCacheSize = 32;
+std::mutex g_map_mutex;
+MapEntry g_map_cache[kMapCacheSize];
+uint64_t g_map_clock = 0;
+
+pkv_status cached_map(MapKind kind, CUtensorMap* map, const void* cache, pkv_dtype dt, int num_blocks, int n_kv,
+                      int head_dim) {
+  const MapKey key = {cache, static_cast<int>(kind), static_cast<int>(dt), num_blocks, n_kv, head_dim};
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (MapEntry& e : g_map_cache) {
+      if (e.last_use != 0 && e.key == key) {
+        e.last_use = ++g_map_clock;
+        *map = e.map;
+        return PKV_OK;
+      }
+    }
+  }
+  const pkv_status st = kind == kMapTile ? encode_cache_map_tile(map, cache, dt, num_blocks, n_kv)
+                                         : encode_cache_map(map, cache, dt, num_blocks, n_kv, head_dim);
+  if (st != PKV_OK) return st;
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  MapEntry* victim = &g_map_cache[0];
+  for (MapEntry& e : g_map_cache)
+    if (e.last_use < victim->last_use) victim = &e;
+  victim->key = key;
+  victim->map = *map;
+  victim->last_use = ++g_map_clock;
+  return PKV_OK;
+}
+
 // The decode kernel is launched cooperatively: its CTAs (at most one per SM)
 // are guaranteed to be co-resident, which its grid-wide barrier needs.
 template <int DT, int D, int GPAD, bool kI8 = false, bool kMQ = false, bool kFused = false>
@@ -593,8 +642,8 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
 
   CUtensorMap mk = {}, mv = {};
   if (!i8) {
-    st = encode_cache_map(&mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
-    if (st == PKV_OK) st = encode_cache_map(&mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+    st = cached_map(kMapBox, &mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
+    if (st == PKV_OK) st = cached_map(kMapBox, &mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
   }
 
   DecodeParams p;
@@ -853,8 +902,8 @@ pkv_status paged_attention_decode_cascade_ex(const void* q, const void* k_cache,
   float* init = static_cast<float*>(ws);
 
   CUtensorMap mk, mv;
-  st = encode_cache_map(&mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
-  if (st == PKV_OK) st = encode_cache_map(&mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+  st = cached_map(kMapBox, &mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
+  if (st == PKV_OK) st = cached_map(kMapBox, &mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
   PrefixParams pp;
   pp.q = q;
   pp.prefix_tables = prefix_block_tables;
@@ -878,7 +927,7 @@ pkv_status paged_attention_decode_cascade_ex(const void* q, const void* k_cache,
   if (!tc && smem + 256 > static_cast<size_t>(di.smem_optin)) st = st == PKV_OK ? PKV_ERR_UNSUPPORTED : st;
   if (st == PKV_OK && tc) {
     CUtensorMap mv_tile;
-    st = encode_cache_map_tile(&mv_tile, v_cache, dtype, num_blocks, n_kv_heads);
+    st = cached_map(kMapTile, &mv_tile, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
     if (st == PKV_OK)
       st = dtype == PKV_F16
                ? launch_prefix_tc<kF16>(mk, mv_tile, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s)

@@ -327,3 +327,18 @@ def test_context_beyond_table_sets_flag():
     w.context_lens = torch.tensor([20, 33], dtype=torch.int32)   # table covers 32 tokens
     run_gpu(w, check_errors=False)
     assert pkv.pkv_get_device_error() & pkv.DEVERR_CONTEXT
+
+
+def test_tensor_map_cache_follows_reused_addresses_and_shapes():
+    # Encoded tensor maps are cached per (address, dtype, shape).  A cache
+    # freed and replaced by another at the same address -- with another
+    # shape, or the same shape and other contents -- must still decode right.
+    dev = torch.device("cuda")
+    for seed, nb_extra in ((71, 0), (72, 37), (73, 37)):
+        w = W.build_workload("mapcache", [40, 300, 129], 8, 2, 128, torch.bfloat16, seed=seed,
+                             pool_blocks=60 + nb_extra)
+        ref, _, _ = oracle.workload_decode(w)
+        out = run_gpu(w)
+        assert_close(out, ref, w.dtype, what=f"seed {seed} pool {w.num_blocks}")
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
