@@ -139,17 +139,23 @@ pkv_status encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dt, i
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
-// A block's whole K or V tile of one kv head as one TMA box (head dim 128,
-// 16-bit): dims {64 dims, 16 tokens, 2 halves of the head dim, kv head,
-// block}, box {64, 16, 2, 1, 1}, landing as [half][token][128 B] with the
-// 128-byte swizzle.
-pkv_status encode_cache_map_tile(CUtensorMap* map, const void* cache, pkv_dtype dt, int num_blocks, int n_kv) {
-  const CUtensorMapDataType ty = dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const cuuint64_t row = 128 * 2;
-  const cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(kBlockTokens), 2, static_cast<cuuint64_t>(n_kv),
+// A block's whole K or V tile of one kv head as one TMA box: dims {128
+// bytes of dims, 16 tokens, head_dim * es / 128 chunks, kv head, block}, box
+// {128 bytes, 16, chunks, 1, 1}, landing as [chunk][token][128 B] with the
+// 128-byte swizzle -- the layout of `chunks` separate 16-row boxes, in one
+// request.
+pkv_status encode_cache_map_tile(CUtensorMap* map, const void* cache, pkv_dtype dt, int num_blocks, int n_kv,
+                                 int head_dim) {
+  const int es = elem_bytes(dt);
+  const CUtensorMapDataType ty = dt == PKV_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * es;
+  const cuuint32_t x = static_cast<cuuint32_t>(128 / es), chunks = static_cast<cuuint32_t>(row / 128);
+  const cuuint64_t dims[5] = {x, static_cast<cuuint64_t>(kBlockTokens), chunks, static_cast<cuuint64_t>(n_kv),
                               static_cast<cuuint64_t>(num_blocks)};
   const cuuint64_t strides[4] = {row, 128, row * kBlockTokens, row * kBlockTokens * n_kv};
-  const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(kBlockTokens), 2, 1, 1};
+  const cuuint32_t box[5] = {x, static_cast<cuuint32_t>(kBlockTokens), chunks, 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUresult r = g_encode(map, ty, 5, const_cast<void*>(cache), dims, strides, box, estr,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -193,7 +199,7 @@ pkv_status cached_map(MapKind kind, CUtensorMap* map, const void* cache, pkv_dty
       }
     }
   }
-  const pkv_status st = kind == kMapTile ? encode_cache_map_tile(map, cache, dt, num_blocks, n_kv)
+  const pkv_status st = kind == kMapTile ? encode_cache_map_tile(map, cache, dt, num_blocks, n_kv, head_dim)
                                          : encode_cache_map(map, cache, dt, num_blocks, n_kv, head_dim);
   if (st != PKV_OK) return st;
   std::lock_guard<std::mutex> lock(g_map_mutex);
@@ -642,8 +648,8 @@ pkv_status decode_impl(const void* q, const void* k_cache, const void* v_cache, 
 
   CUtensorMap mk = {}, mv = {};
   if (!i8) {
-    st = cached_map(kMapBox, &mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
-    if (st == PKV_OK) st = cached_map(kMapBox, &mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+    st = cached_map(kMapTile, &mk, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
+    if (st == PKV_OK) st = cached_map(kMapTile, &mv, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
   }
 
   DecodeParams p;

@@ -1490,13 +1490,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             const size_t bh = static_cast<size_t>(ph) * p.n_kv_heads + t0.kvh;
             bulk_load(sk, p.kv_i8 + bh * kRingStride, kRingStride, &full_bar[slot]);
           } else {
+            // One request for the whole K tile and one for V: the number
+            // of requests per tile, not their bytes, sets the pace of the
+            // copy engine.
             mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
-#pragma unroll
-            for (int y = 0; y < Y; ++y)
-              tma_load_4d(sk + y * kBoxBytes, &tm_k, &full_bar[slot], y * X, 0, t0.kvh, ph);
-#pragma unroll
-            for (int y = 0; y < Y; ++y)
-              tma_load_4d(sk + kTileBytes + y * kBoxBytes, &tm_v, &full_bar[slot], y * X, 0, t0.kvh, ph);
+            tma_load_5d(sk, &tm_k, &full_bar[slot], 0, 0, 0, t0.kvh, ph);
+            tma_load_5d(sk + kTileBytes, &tm_v, &full_bar[slot], 0, 0, 0, t0.kvh, ph);
           }
           ++issued;
           if (++stage == p.stages) {

@@ -85,18 +85,6 @@ static_assert(kTcOutOffset + kTcRows * 512 <= kTcSmemBytes, "output rows fit in 
 constexpr int kTcBarBytes = (2 * kTcStages + 2 * kTcSBufs + 4) * 8 + 16;
 constexpr int kTcExchBytes = (4 * kTcRows + 2 * kTcRows + kTcRows) * 4;
 
-// 5-D tiled TMA load global -> this CTA's own shared memory: the
-// V tile of one block and kv head in one request, box {64 dims, 16 tokens,
-// 2 halves of the head dim} landing as [half][token][128 B].
-__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
-                                            int c2, int c3, int c4) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-      : "memory");
-}
-
 // Softmax arithmetic with fewer issue slots: two fp32 lanes per packed FMA /
 // add (sm_100), two new values per three-input max, and the hardware base-2
 // exponential with flush to zero (the probabilities become 16-bit anyway).
