@@ -114,6 +114,17 @@ __device__ __forceinline__ void append_range(const AppendParams& p, int64_t star
   }
 }
 
+// The fused append of the decode kernel's first phase: every thread writes its
+// share of the new rows, makes them visible to the TMA reads that follow the
+// grid barrier (fence.proxy.async: generic-proxy writes, async-proxy reads)
+// and arrives on that barrier.  Out of line, so that it stays out of the
+// decode loop's register allocation.
+__device__ __noinline__ unsigned int fused_append_arrive(const AppendParams& p, int64_t start, int64_t stride) {
+  append_range(p, start, stride);
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return cooperative_groups::this_grid().barrier_arrive();
+}
+
 __global__ void __launch_bounds__(256) pkv_append_kernel(const AppendParams p) {
   append_range(p, blockIdx.x * (int64_t)blockDim.x + threadIdx.x, (int64_t)gridDim.x * blockDim.x);
 }
@@ -1171,131 +1182,105 @@ __device__ __forceinline__ void q_fetch(uint8_t* qbuf, const DecodeParams& p, in
   cp_async_commit();
 }
 
-// Phase 2 of the decode kernel: one warp merges dims [d0, d0 + 32 DPL) of
-// query head g of the split segment whose first piece chunk u holds (mt =
-// meta[u]); the pieces are held by chunks u..u_hi (chunks are never empty)
-// and are combined in chunk (tile) order as
-//   M = max_i m_i,  w_i = 2^(m_i - M),  out = sum_i w_i O_i / sum_i w_i l_i.
-// Lane j holds the scalars of pieces j and j + 32 (pieces beyond 64 are
-// folded in by a plain loop); each lane owns DPL dims of the numerator.  The
-// records are read in batches of PB pieces, the first batch together with
-// the scalars, so that a merge of up to PB pieces costs one round trip to L2
-// (ld.global.cg: the records were written by other SMs before the grid
-// barrier).  With at most 8 pieces and DPL = D / 32 every load of every piece
-// goes out in one round without shuffles.
-template <int DT, int D, int DPL>
-__device__ __forceinline__ void merge_head(const DecodeParams& p, int u, int4 mt, int g, int d0, int lane) {
-  using T = typename DTypeInfo<DT>::T;
-  constexpr int PB = DPL >= 4 ? 8 : (DPL == 2 ? 12 : 24);  // pieces per batch: PB * DPL registers
-  const int seg = mt.x, b = seg / p.ng, hg = seg % p.ng, n = mt.y - u + 1;
-  const int mo = p.rows * D + g, lo = p.rows * D + p.rows + g, oo = g * D + d0 + lane * DPL;
-  auto rec_of = [&](int j) -> const float* {  // record of piece j (chunk u + j)
-    return p.records + (static_cast<size_t>(u + j) * 2 + (j == 0 ? mt.z : 0)) * p.rec_floats;
-  };
-  auto load_o = [&](const float* r, float (&x)[DPL]) {
-    if constexpr (DPL == 4) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(r + oo));
-      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-    } else if constexpr (DPL == 2) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(r + oo));
-      x[0] = v.x; x[1] = v.y;
-    } else {
-      x[0] = __ldcg(r + oo);
-    }
-  };
-  T* const ob = static_cast<T*>(p.out) + out_row(p, b, hg, g) * D + d0 + lane * DPL;
-  auto store = [&](const float (&acc)[DPL], float inv) {
-    if constexpr (DPL == 4) {
-      store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    } else if constexpr (DT == kF32) {
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) ob[i] = acc[i] * inv;
-    } else if constexpr (DPL == 2) {
-      *reinterpret_cast<uint32_t*>(ob) = pack2<DT == kBF16>(acc[0] * inv, acc[1] * inv);
-    } else {
-      ob[0] = static_cast<T>(acc[0] * inv);  // round to nearest even
-    }
-  };
-  if (DPL * 32 == D && n <= 8) {
-    // Common case: every load of every piece issued in one round.
-    float mj[8], lj[8], o[8][DPL];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float* r = rec_of(min(j, n - 1));
-      mj[j] = __ldcg(r + mo);
-      lj[j] = __ldcg(r + lo);
-      load_o(r, o[j]);
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < n) M = fmaxf(M, mj[j]);
-    float L = 0.f, acc[DPL];
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      // M is -inf only when every piece skipped all its tiles (bad block ids).
-      const float w = (j < n && M != -INFINITY) ? exp2f(mj[j] - M) : 0.f;
-      L = fmaf(w, lj[j], L);
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, o[j][i], acc[i]);
-    }
-    store(acc, L > 0.f ? 1.f / L : 0.f);
-    return;
-  }
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  if (lane < n) {
-    m0 = __ldcg(rec_of(lane) + mo);
-    l0 = __ldcg(rec_of(lane) + lo);
-  }
-  if (lane + 32 < n) {
-    m1 = __ldcg(rec_of(lane + 32) + mo);
-    l1 = __ldcg(rec_of(lane + 32) + lo);
-  }
-  float o[PB][DPL];
-#pragma unroll
-  for (int jj = 0; jj < PB; ++jj) load_o(rec_of(min(jj, n - 1)), o[jj]);
-  float M = fmaxf(m0, m1);
-  for (int j = 64 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(rec_of(j) + mo));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if (M == -INFINITY) M = 0.f;  // every piece empty (bad block ids): all weights 0, a zero row
-  const float w0 = exp2f(m0 - M), w1 = exp2f(m1 - M);
-  float L = w0 * l0 + w1 * l1;
-  for (int j = 64 + lane; j < n; j += 32) L = fmaf(exp2f(__ldcg(rec_of(j) + mo) - M), __ldcg(rec_of(j) + lo), L);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+// Where the partial records of one split segment are: piece 0 in chunk u1,
+// record slot z (0: the segment is the chunk's first, 1: its last); piece j
+// >= 1 in chunk base + j * step, slot 0 (the segment continues there from
+// the previous chunk).  n pieces in all.
+struct MergeSrc {
+  int u1, z, n, base, step;
+};
 
-  float acc[DPL];
+// Combines dims [d0, d0 + 32 DPL) of row g of segment (b, hg) from its
+// pieces, in piece order, as an online merge over batches of 8 pieces:
+//   M = max_i m_i,  w_i = 2^(m_i - M),  O = sum_i w_i O_i,  l = sum_i w_i l_i
+// (the running O and l are rescaled by 2^(M_old - M_new) when a batch raises
+// the maximum).  With to_rec null the result is normalised and written to
+// `out` (rounded to nearest even); otherwise the unnormalised state (O, M, l)
+// is written into the record `to_rec` (piece 0's own record: every load
+// comes before the stores).  Each lane owns DPL dims of O.  A batch's loads
+// (m, l and the lane's O slice of 8 pieces) go out together, in program order
+// (ld.global.cg: other SMs, or other warps of this CTA, wrote the records
+// before a barrier), so that a batch costs one round trip to L2.
+template <int DT, int D, int DPL>
+__device__ __forceinline__ void merge_rows(const DecodeParams& p, const MergeSrc& src, int b, int hg, int g, int d0,
+                                           int lane, float* to_rec) {
+  using T = typename DTypeInfo<DT>::T;
+  constexpr int kBatch = DPL == 1 ? 16 : 8;  // pieces per round: 3 kBatch + kBatch DPL registers
+  const int n = src.n;
+  const int mo = p.rows * D + g, lo = p.rows * D + p.rows + g, oo = g * D + d0 + lane * DPL;
+  float M = -INFINITY, L = 0.f, acc[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-  for (int j0 = 0; j0 < n; j0 += PB) {
-    if (j0 > 0) {
+  for (int j0 = 0; j0 < n; j0 += kBatch) {
+    float mj[kBatch], lj[kBatch], o[kBatch][DPL];
 #pragma unroll
-      for (int jj = 0; jj < PB; ++jj) load_o(rec_of(min(j0 + jj, n - 1)), o[jj]);
+    for (int jj = 0; jj < kBatch; ++jj) {
+      const int j = min(j0 + jj, n - 1);
+      const int chunk = j == 0 ? src.u1 : src.base + j * src.step;
+      const float* r = p.records + (static_cast<size_t>(chunk) * 2 + (j == 0 ? src.z : 0)) * p.rec_floats;
+      mj[jj] = ld_cg(r + mo);
+      lj[jj] = ld_cg(r + lo);
+      if constexpr (DPL == 4) {
+        const float4 v = ld_cg4(r + oo);
+        o[jj][0] = v.x; o[jj][1] = v.y; o[jj][2] = v.z; o[jj][3] = v.w;
+      } else if constexpr (DPL == 2) {
+        const float2 v = ld_cg2(r + oo);
+        o[jj][0] = v.x; o[jj][1] = v.y;
+      } else {
+        o[jj][0] = ld_cg(r + oo);
+      }
     }
+    float Mb = M;
 #pragma unroll
-    for (int jj = 0; jj < PB; ++jj) {
-      const int j = j0 + jj;
-      float wj = __shfl_sync(0xffffffffu, (j & 32) ? w1 : w0, j & 31);
-      if (j >= 64 && j < n) wj = exp2f(__ldcg(rec_of(j) + mo) - M);
-      if (j >= n) wj = 0.f;
+    for (int jj = 0; jj < kBatch; ++jj)
+      if (j0 + jj < n) Mb = fmaxf(Mb, mj[jj]);
+    // M (and Mb) stay -inf only while every piece so far skipped all its
+    // tiles (bad block ids): those weights are 0 and the state stays empty.
+    const float alpha = M == -INFINITY ? 0.f : exp2f(M - Mb);
+    L *= alpha;
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(wj, o[jj][i], acc[i]);
+    for (int i = 0; i < DPL; ++i) acc[i] *= alpha;
+#pragma unroll
+    for (int jj = 0; jj < kBatch; ++jj) {
+      const float w = (j0 + jj < n && Mb != -INFINITY) ? exp2f(mj[jj] - Mb) : 0.f;
+      L = fmaf(w, lj[jj], L);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, o[jj][i], acc[i]);
     }
+    M = Mb;
   }
-  store(acc, L > 0.f ? 1.f / L : 0.f);
+  if (to_rec != nullptr) {
+    float* ro = to_rec + oo;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) ro[i] = acc[i];
+    if (lane == 0 && d0 == 0) {
+      to_rec[mo] = M;
+      to_rec[lo] = L;
+    }
+    return;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;  // L is 0 only when every piece skipped all its tiles
+  T* const ob = static_cast<T*>(p.out) + out_row(p, b, hg, g) * D + d0 + lane * DPL;
+  if constexpr (DPL == 4) {
+    store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  } else if constexpr (DT == kF32) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) ob[i] = acc[i] * inv;
+  } else if constexpr (DPL == 2) {
+    *reinterpret_cast<uint32_t*>(ob) = pack2<DT == kBF16>(acc[0] * inv, acc[1] * inv);
+  } else {
+    ob[0] = static_cast<T>(acc[0] * inv);  // round to nearest even
+  }
 }
 
-// GPAD: 0 = CUDA-core consumer (gp == 1); 8 or 16 = tensor-core consumer.
-//
-// Launched cooperatively (all CTAs co-resident, one per SM): phase 1 runs the
-// producer/consumer pipeline; a grid-wide barrier follows (every wait before
-// it is bounded, so every thread reaches it); phase 2 merges split segments
-// and zero-fills the rows of empty sequences.
-// kI8: the cache holds INT8 records (MmaConsumerI8).  kMQ: q_len > 1
-// queries per sequence (tensor-core consumer with per-row causal limits).
+// Tile range [start, end) of segment (b, hg) from the block-wide prefix sums.
+__device__ __forceinline__ void segment_tiles(const int* prefix, const int* ctxs, int b, int hg, int& start,
+                                              int& end) {
+  const int nb = (ctxs[b] + kBlockTokens - 1) / kBlockTokens;
+  start = prefix[b] + hg * nb;
+  end = start + nb;
+}
+
 // kFused: the launch first writes the new tokens of p.app into the cache
 // (paged_kv_append_and_decode); a separate instantiation, so that the plain
 // decode's register allocation does not carry the fused prologue.
@@ -1360,10 +1345,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   constexpr bool fused_append = kFused;
   [[maybe_unused]] unsigned int app_token = 0;
   if constexpr (fused_append) {
-    append_range(p.app, blockIdx.x * static_cast<int64_t>(kDecodeThreads) + threadIdx.x,
-                 static_cast<int64_t>(gridDim.x) * kDecodeThreads);
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    app_token = cooperative_groups::this_grid().barrier_arrive();
+    app_token = fused_append_arrive(p.app, blockIdx.x * static_cast<int64_t>(kDecodeThreads) + threadIdx.x,
+                                    static_cast<int64_t>(gridDim.x) * kDecodeThreads);
   }
 
   // Tiles per sequence -> exclusive prefix sums (block-wide scan).
@@ -1418,6 +1401,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // before the current chunk's end and read at its last tile, so the warp
     // (whose lanes run in step) never waits on an L2 round trip.
     if constexpr (fused_append) asm volatile("fence.proxy.async.global;" ::: "memory");
+    const uint64_t kv_policy = l2_policy_evict_first();  // each K/V tile is read once
     const int u = blockIdx.x * kConsumerWarps + lane;
     // Test hook: the lane of the withheld unit never issues, so that its
     // consumer's bounded wait runs out (no copy is then in flight for it).
@@ -1488,14 +1472,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
             // The whole record in one contiguous request.
             const size_t bh = static_cast<size_t>(ph) * p.n_kv_heads + t0.kvh;
-            bulk_load(sk, p.kv_i8 + bh * kRingStride, kRingStride, &full_bar[slot]);
+            bulk_load_hint(sk, p.kv_i8 + bh * kRingStride, kRingStride, &full_bar[slot], kv_policy);
           } else {
             // One request for the whole K tile and one for V: the number
             // of requests per tile, not their bytes, sets the pace of the
             // copy engine.
             mbar_arrive_expect_tx(&full_bar[slot], kStageBytes);
-            tma_load_5d(sk, &tm_k, &full_bar[slot], 0, 0, 0, t0.kvh, ph);
-            tma_load_5d(sk + kTileBytes, &tm_v, &full_bar[slot], 0, 0, 0, t0.kvh, ph);
+            tma_load_5d_hint(sk, &tm_k, &full_bar[slot], t0.kvh, ph, kv_policy);
+            tma_load_5d_hint(sk + kTileBytes, &tm_v, &full_bar[slot], t0.kvh, ph, kv_policy);
           }
           ++issued;
           if (++stage == p.stages) {
@@ -1657,47 +1641,61 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 
   // ---------------- phase 2: merge split segments ----------------
-  // Every warp of the grid takes (chunk, query head) items; the items of
-  // chunks that hold the first piece of a split segment merge that head.
   cooperative_groups::this_grid().sync();
   {
     constexpr int kWarps = kConsumerWarps + 1;
     const int gw = blockIdx.x * kWarps + warp, n_warps = gridDim.x * kWarps;
     const int n_segs = B * p.ng;
-    // Long split contexts (many pieces per segment, few merges) are merged
-    // by D / 32 warps per query head, one dim per lane, so that more warps
-    // share the merge and each issues all its loads at once.  The choice is
-    // the same in every CTA (T and the schedule are).
-    // (T is re-read from shared memory so that it is not held in a register
-    // through phase 1.)
     constexpr int kSlices = D / 32;
-    const int T2 = prefix[B];
-    const int Lq2 = T2 / max(1, min(p.num_units, T2));
-    const bool sliced = T2 > 0 && T2 / max(1, n_segs) >= 8 * max(1, Lq2) &&
-                        n_segs * p.rows * kSlices <= n_warps;
-    const int slices = sliced ? kSlices : 1;
-    const int per_chunk = p.rows * slices;
-    const int items = n_chunks * per_chunk;
-    // Item metadata is loaded 32 items at a time, lane t for the round's
-    // t-th item of this warp.
-    for (int base = gw; base < items; base += 32 * n_warps) {
-      int4 my_item = make_int4(-1, 0, 0, 0);
-      const int i_lane = base + lane * n_warps;
-      if (i_lane < items) my_item = __ldcg(p.meta + i_lane / per_chunk);
-      for (int t = 0; t < 32 && base + t * n_warps < items; ++t) {
-        const int i = base + t * n_warps;
-        const int c = i / per_chunk, rem = i - c * per_chunk;
-        int4 mt;
-        mt.x = __shfl_sync(0xffffffffu, my_item.x, t);
-        mt.y = __shfl_sync(0xffffffffu, my_item.y, t);
-        mt.z = __shfl_sync(0xffffffffu, my_item.z, t);
-        // Entries of chunks that an aborted launch never reached may be
-        // stale: only well-formed ones are merged.
-        if (mt.x >= 0 && mt.x < n_segs && mt.y > c && mt.y < n_chunks && (mt.z == 0 || mt.z == 1)) {
-          if (sliced)
-            merge_head<DT, D, 1>(p, c, mt, rem / kSlices, (rem % kSlices) * 32, lane);
-          else
-            merge_head<DT, D, D / 32>(p, c, mt, rem, 0, lane);
+    if (M == 0) {
+      // Static schedule: every warp of the grid takes (segment, row[, dim
+      // slice]) items, so that the merges are spread evenly over the grid; a
+      // segment whose tiles span several units has one piece per unit (its
+      // record in the unit's chunk) and is merged here.  When the items are
+      // few, D / 32 warps share a row (one dim per lane), so that more warps
+      // take part.  (The schedule is recomputed from shared memory rather
+      // than held in registers through phase 1.)
+      const Sched s2 = make_sched(prefix[B], p.num_units, 0, p.static_permille);
+      const bool sliced = n_segs * p.rows * kSlices <= n_warps;
+      const int per_seg = sliced ? p.rows * kSlices : p.rows;
+      const int items = n_segs * per_seg;
+      for (int i = gw; i < items; i += n_warps) {
+        const int seg = i / per_seg, rem = i - seg * per_seg;
+        const int b = seg / p.ng, hg = seg - b * p.ng;
+        if (ctxs[b] == 0) continue;
+        int st, en;
+        segment_tiles(prefix, ctxs, b, hg, st, en);
+        const int u1 = unit_of_tile(s2, st), u2 = unit_of_tile(s2, en - 1);
+        if (u1 == u2) continue;  // the whole segment in one unit: written out in phase 1
+        const MergeSrc src = {u1, st == unit_begin(s2, u1) ? 0 : 1, u2 - u1 + 1, u1, 1};
+        if (sliced)
+          merge_rows<DT, D, 1>(p, src, b, hg, rem / kSlices, (rem % kSlices) * 32, lane, nullptr);
+        else
+          merge_rows<DT, D, D / 32>(p, src, b, hg, rem, 0, lane, nullptr);
+      }
+    } else {
+      // Balancing chunks: the chunk that holds a split segment's first piece
+      // publishes it in meta; every warp takes (chunk, row) items and merges
+      // the pieces of consecutive chunks.  Item metadata is loaded 32 items
+      // at a time, lane t for the round's t-th item of this warp.
+      const int items = n_chunks * p.rows;
+      for (int base = gw; base < items; base += 32 * n_warps) {
+        int4 my_item = make_int4(-1, 0, 0, 0);
+        const int i_lane = base + lane * n_warps;
+        if (i_lane < items) my_item = __ldcg(p.meta + i_lane / p.rows);
+        for (int t = 0; t < 32 && base + t * n_warps < items; ++t) {
+          const int i = base + t * n_warps;
+          const int c = i / p.rows;
+          int4 mt;
+          mt.x = __shfl_sync(0xffffffffu, my_item.x, t);
+          mt.y = __shfl_sync(0xffffffffu, my_item.y, t);
+          mt.z = __shfl_sync(0xffffffffu, my_item.z, t);
+          // Entries of chunks that an aborted launch never reached may be
+          // stale: only well-formed ones are merged.
+          if (mt.x >= 0 && mt.x < n_segs && mt.y > c && mt.y < n_chunks && (mt.z == 0 || mt.z == 1)) {
+            const MergeSrc src = {c, mt.z, mt.y - c + 1, c, 1};
+            merge_rows<DT, D, D / 32>(p, src, mt.x / p.ng, mt.x % p.ng, i - c * p.rows, 0, lane, nullptr);
+          }
         }
       }
     }
