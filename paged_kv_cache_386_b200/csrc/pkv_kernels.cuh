@@ -1344,18 +1344,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // proxy) that follow the barrier.
   constexpr bool fused_append = kFused;
   [[maybe_unused]] unsigned int app_token = 0;
+  const int scan_per = (B + kDecodeThreads - 1) / kDecodeThreads;
+  const int scan_lo = min(B, static_cast<int>(threadIdx.x) * scan_per), scan_hi = min(B, scan_lo + scan_per);
+  // Fused: this thread's first context length is read before the append, so
+  // that the two reads overlap.
+  [[maybe_unused]] int ctx_first = 0;
   if constexpr (fused_append) {
+    if (scan_lo < scan_hi) ctx_first = __ldg(p.context_lens + scan_lo);
     app_token = fused_append_arrive(p.app, blockIdx.x * static_cast<int64_t>(kDecodeThreads) + threadIdx.x,
                                     static_cast<int64_t>(gridDim.x) * kDecodeThreads);
   }
 
   // Tiles per sequence -> exclusive prefix sums (block-wide scan).
   {
-    const int per = (B + kDecodeThreads - 1) / kDecodeThreads;
-    const int lo = min(B, threadIdx.x * per), hi = min(B, lo + per);
+    const int lo = scan_lo, hi = scan_hi;
     int local = 0;
     for (int b = lo; b < hi; ++b) {
-      const int c0 = __ldg(p.context_lens + b);
+      int c0;
+      if constexpr (fused_append)
+        c0 = b == lo ? ctx_first : __ldg(p.context_lens + b);
+      else
+        c0 = __ldg(p.context_lens + b);
       int c = clamp_ctx(c0, max_ctx);
       if (c > 0 && c < p.q_len) c = 0;  // fewer tokens than queries: flagged, no output but zeros
       if (c != c0) flag_error(PKV_DEVERR_CONTEXT);
@@ -1648,26 +1657,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const int n_segs = B * p.ng;
     constexpr int kSlices = D / 32;
     if (M == 0) {
-      // Static schedule: every warp of the grid takes (segment, row[, dim
-      // slice]) items, so that the merges are spread evenly over the grid; a
-      // segment whose tiles span several units has one piece per unit (its
-      // record in the unit's chunk) and is merged here.  When the items are
-      // few, D / 32 warps share a row (one dim per lane), so that more warps
-      // take part.  (The schedule is recomputed from shared memory rather
-      // than held in registers through phase 1.)
-      const Sched s2 = make_sched(prefix[B], p.num_units, 0, p.static_permille);
-      const bool sliced = n_segs * p.rows * kSlices <= n_warps;
-      const int per_seg = sliced ? p.rows * kSlices : p.rows;
-      const int items = n_segs * per_seg;
+      // Static schedule.  A split segment is merged from its pieces, one
+      // record per unit it spans; its first piece lies in the unit where it
+      // starts, and a unit starts at most one segment that continues past its
+      // end (its last one).  The items are (segment, row[, dim slice]) or
+      // (unit, row[, dim slice]), whichever set is smaller -- every segment,
+      // and every unit, yields at most one merge per row -- taken by every
+      // warp of the grid in turn, so that the merges spread evenly.  When
+      // segments span many units (long contexts: few merges, many pieces),
+      // D / 32 warps share a row, one dim per lane, so that more warps take
+      // part.  (The schedule is recomputed from shared memory rather than
+      // held in registers through phase 1.)
+      const int T2 = prefix[B];
+      const Sched s2 = make_sched(T2, p.num_units, 0, p.static_permille);
+      const int n_units = T2 > 0 ? s2.U : 0;
+      const bool by_segment = n_segs <= n_units;
+      const bool sliced = T2 / max(1, n_segs) >= 8 * max(1, s2.Lq);
+      const int per_item = sliced ? p.rows * kSlices : p.rows;
+      const int items = (by_segment ? n_segs : n_units) * per_item;
       for (int i = gw; i < items; i += n_warps) {
-        const int seg = i / per_seg, rem = i - seg * per_seg;
-        const int b = seg / p.ng, hg = seg - b * p.ng;
-        if (ctxs[b] == 0) continue;
-        int st, en;
-        segment_tiles(prefix, ctxs, b, hg, st, en);
-        const int u1 = unit_of_tile(s2, st), u2 = unit_of_tile(s2, en - 1);
-        if (u1 == u2) continue;  // the whole segment in one unit: written out in phase 1
-        const MergeSrc src = {u1, st == unit_begin(s2, u1) ? 0 : 1, u2 - u1 + 1, u1, 1};
+        const int x = i / per_item, rem = i - x * per_item;
+        int b, hg, st, en, u1;
+        if (by_segment) {
+          b = x / p.ng;
+          hg = x - b * p.ng;
+          if (ctxs[b] == 0) continue;
+          segment_tiles(prefix, ctxs, b, hg, st, en);
+          u1 = unit_of_tile(s2, st);
+          if (en <= unit_begin(s2, u1 + 1)) continue;  // the whole segment in one unit: written in phase 1
+        } else {
+          u1 = x;
+          const int a = unit_begin(s2, u1), e = unit_begin(s2, u1 + 1);
+          Walk wl;
+          walk_begin(wl, prefix, ctxs, B, e - 1, e);  // the segment of the unit's last tile
+          b = wl.b;
+          hg = wl.hg;
+          segment_tiles(prefix, ctxs, b, hg, st, en);
+          if (st < a || en <= e) continue;  // started in an earlier unit, or ends in this one
+        }
+        const MergeSrc src = {u1, st == unit_begin(s2, u1) ? 0 : 1, unit_of_tile(s2, en - 1) - u1 + 1, u1, 1};
         if (sliced)
           merge_rows<DT, D, 1>(p, src, b, hg, rem / kSlices, (rem % kSlices) * 32, lane, nullptr);
         else
