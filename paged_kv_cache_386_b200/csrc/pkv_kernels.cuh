@@ -91,26 +91,41 @@ struct AppendParams {
 };
 
 // Chunks idx = start, start + stride, ... of the append: one 16-byte chunk
-// of one head row of one token per index.
+// of one head row of one token per index.  Four chunks' loads (slot, k, v)
+// go out before their stores, so that the loop does not wait for one load
+// round trip per chunk (the stores might alias the next loads otherwise).
 __device__ __forceinline__ void append_range(const AppendParams& p, int64_t start, int64_t stride) {
-  for (int64_t idx = start; idx < p.total; idx += stride) {
-    const int c = static_cast<int>(idx % p.row_chunks);
-    const int64_t th = idx / p.row_chunks;  // token * n_kv + head
-    const int h = static_cast<int>(th % p.n_kv_heads);
-    const int64_t i = th / p.n_kv_heads;
-    const int64_t s = __ldg(p.slot_mapping + i);
-    if (s < 0) continue;  // padding token
-    if (s >= p.num_slots) {
-      if (h == 0 && c == 0) flag_error(PKV_DEVERR_SLOT);
-      continue;
+  constexpr int kU = 4;
+  for (int64_t base = start; base < p.total; base += kU * stride) {
+    int4 kv[kU], vv[kU];
+    int64_t dst[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t idx = base + u * stride;
+      dst[u] = -1;
+      if (idx >= p.total) continue;
+      const int c = static_cast<int>(idx % p.row_chunks);
+      const int64_t th = idx / p.row_chunks;  // token * n_kv + head
+      const int h = static_cast<int>(th % p.n_kv_heads);
+      const int64_t i = th / p.n_kv_heads;
+      const int64_t sl = __ldg(p.slot_mapping + i);
+      const int64_t src = (th * p.row_chunks + c) * 16;
+      kv[u] = __ldg(reinterpret_cast<const int4*>(p.k + src));
+      vv[u] = __ldg(reinterpret_cast<const int4*>(p.v + src));
+      if (sl < 0) continue;  // padding token
+      if (sl >= p.num_slots) {
+        if (h == 0 && c == 0) flag_error(PKV_DEVERR_SLOT);
+        continue;
+      }
+      const int64_t blk = sl / kBlockTokens, off = sl % kBlockTokens;
+      dst[u] = (((blk * p.n_kv_heads + h) * kBlockTokens + off) * p.row_chunks + c) * 16;
     }
-    const int64_t blk = s / kBlockTokens, off = s % kBlockTokens;
-    const int64_t src = (th * p.row_chunks + c) * 16;
-    const int64_t dst = (((blk * p.n_kv_heads + h) * kBlockTokens + off) * p.row_chunks + c) * 16;
-    const int4 kv = __ldg(reinterpret_cast<const int4*>(p.k + src));
-    const int4 vv = __ldg(reinterpret_cast<const int4*>(p.v + src));
-    *reinterpret_cast<int4*>(p.k_cache + dst) = kv;
-    *reinterpret_cast<int4*>(p.v_cache + dst) = vv;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (dst[u] < 0) continue;
+      *reinterpret_cast<int4*>(p.k_cache + dst[u]) = kv[u];
+      *reinterpret_cast<int4*>(p.v_cache + dst[u]) = vv[u];
+    }
   }
 }
 
