@@ -181,3 +181,28 @@ def test_header_compiles_as_plain_c(tmp_path):
     r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
                         "-I", str(HEADER.parent), str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_binding_checks_dtypes_and_shapes_before_any_cuda_call(lib):
+    # The C layer sees raw pointers and q's dtype only; the binding refuses
+    # caches or outputs of another dtype or shape (CPU tensors suffice: the
+    # checks run before any pointer is taken).
+    import torch
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    kc = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16)
+    bt = torch.zeros(2, 2, dtype=torch.int32)
+    cl = torch.ones(2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="dtype"):
+        pkv.paged_attention_decode(q, kc.half(), kc.half(), bt, cl, 0.1)
+    with pytest.raises(ValueError, match="out"):
+        pkv.paged_attention_decode(q, kc, kc, bt, cl, 0.1, out=torch.zeros(2, 8, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="out"):
+        pkv.paged_attention_decode(q, kc, kc, bt, cl, 0.1, out=torch.zeros(2, 8, 128, dtype=torch.float16))
+    with pytest.raises(ValueError, match="out"):
+        pkv.paged_attention_decode_noalloc(q, kc, kc, bt, cl, 0.1, out=torch.zeros(3, 8, 128, dtype=torch.bfloat16))
+    k = torch.zeros(2, 2, 128, dtype=torch.bfloat16)
+    sl = torch.zeros(2, dtype=torch.int64)
+    with pytest.raises(ValueError):
+        pkv.paged_kv_append_and_decode(q, k.half(), k.half(), sl, kc, kc, bt, cl, 0.1)
+    with pytest.raises(ValueError):
+        pkv.paged_kv_append(k[:, :1], k[:, :1], sl, kc, kc)   # wrong kv-head count
