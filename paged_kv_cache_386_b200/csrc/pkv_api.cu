@@ -163,11 +163,31 @@ pkv_status encode_cache_map_tile(CUtensorMap* map, const void* cache, pkv_dtype 
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// K of a block for the tensor-memory prefix kernel (16-bit, head dim 128) as
+// one TMA box: dims {64 dims, 8 tokens, dim half, 8-token group, block x kv
+// head} (the cache's [block][kv head] pairs are 4 KiB apart), landing as
+// [token group][dim half][8 tokens][128 B] with the 128-byte swizzle, so that
+// the 8-token atoms of one dim half lie 2 KiB apart in shared memory.
+pkv_status encode_cache_map_kgroups(CUtensorMap* map, const void* cache, pkv_dtype dt, int num_blocks, int n_kv,
+                                    int head_dim) {
+  if (elem_bytes(dt) != 2 || head_dim != 128) return PKV_ERR_UNSUPPORTED;
+  const CUtensorMapDataType ty = dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint64_t row = 256;
+  const cuuint64_t dims[5] = {64, 8, 2, 2, static_cast<cuuint64_t>(num_blocks) * static_cast<cuuint64_t>(n_kv)};
+  const cuuint64_t strides[4] = {row, 128, 8 * row, kBlockTokens * row};
+  const cuuint32_t box[5] = {64, 8, 2, 2, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = g_encode(map, ty, 5, const_cast<void*>(cache), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
 // Encoded tensor maps, cached per (kind, base address, dtype, shape): a map
 // depends only on those, so a serving loop that calls with the same caches
 // every step pays the encode once.  A small table with least-recently-used
 // replacement, shared by every device and host thread.
-enum MapKind { kMapBox = 0, kMapTile = 1 };
+enum MapKind { kMapBox = 0, kMapTile = 1, kMapKGroups = 2 };
 struct MapKey {
   const void* base;
   int kind, dtype, num_blocks, n_kv, head_dim;
@@ -199,8 +219,9 @@ pkv_status cached_map(MapKind kind, CUtensorMap* map, const void* cache, pkv_dty
       }
     }
   }
-  const pkv_status st = kind == kMapTile ? encode_cache_map_tile(map, cache, dt, num_blocks, n_kv, head_dim)
-                                         : encode_cache_map(map, cache, dt, num_blocks, n_kv, head_dim);
+  const pkv_status st = kind == kMapTile      ? encode_cache_map_tile(map, cache, dt, num_blocks, n_kv, head_dim)
+                        : kind == kMapKGroups ? encode_cache_map_kgroups(map, cache, dt, num_blocks, n_kv, head_dim)
+                                              : encode_cache_map(map, cache, dt, num_blocks, n_kv, head_dim);
   if (st != PKV_OK) return st;
   std::lock_guard<std::mutex> lock(g_map_mutex);
   MapEntry* victim = &g_map_cache[0];
@@ -926,18 +947,21 @@ pkv_status paged_attention_decode_cascade_ex(const void* q, const void* k_cache,
   pp.scale_log2 = scale * 1.4426950408889634f;
   const size_t stage_bytes = static_cast<size_t>(2) * kPrefixBlocks * (head_dim * 2 / 128) * kBoxBytes;
   const size_t smem = 1024 + kPrefixStages * (stage_bytes + 2 * sizeof(uint64_t)) + 16 + static_cast<size_t>(batch) * 4;
-  // Head dim 128 runs on the tensor-memory kernel when its operands fit.
-  const bool tc_fits = head_dim == 128 && prefix_tc_smem(batch) + 256 <= static_cast<size_t>(di.smem_optin);
-  if (opt.prefix_kernel == 1 && !tc_fits) return PKV_ERR_UNSUPPORTED;
+  // Head dim 128 runs on the tensor-memory kernel when its operands fit (and
+  // its K map's block x kv-head coordinate fits 32 bits).
+  const bool tc_fits = head_dim == 128 && prefix_tc_smem(batch) + 256 <= static_cast<size_t>(di.smem_optin) &&
+                       static_cast<int64_t>(num_blocks) * n_kv_heads < (int64_t(1) << 31);
+  if (opt.prefix_kernel == 1 && !tc_fits && st == PKV_OK) st = PKV_ERR_UNSUPPORTED;  // the owned workspace is freed below
   const bool tc = tc_fits && opt.prefix_kernel != 2;
   if (!tc && smem + 256 > static_cast<size_t>(di.smem_optin)) st = st == PKV_OK ? PKV_ERR_UNSUPPORTED : st;
   if (st == PKV_OK && tc) {
-    CUtensorMap mv_tile;
-    st = cached_map(kMapTile, &mv_tile, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
+    CUtensorMap mk_groups, mv_tile;
+    st = cached_map(kMapKGroups, &mk_groups, k_cache, dtype, num_blocks, n_kv_heads, head_dim);
+    if (st == PKV_OK) st = cached_map(kMapTile, &mv_tile, v_cache, dtype, num_blocks, n_kv_heads, head_dim);
     if (st == PKV_OK)
       st = dtype == PKV_F16
-               ? launch_prefix_tc<kF16>(mk, mv_tile, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s)
-               : launch_prefix_tc<kBF16>(mk, mv_tile, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s);
+               ? launch_prefix_tc<kF16>(mk_groups, mv_tile, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s)
+               : launch_prefix_tc<kBF16>(mk_groups, mv_tile, pp, n_kv_heads, opt.prefix_splits, di.sm_count, s);
   } else if (st == PKV_OK) {
     if (dtype == PKV_F16)
       st = head_dim == 64 ? launch_prefix<kF16, 64>(mk, mv, pp, n_kv_heads, smem, s)

@@ -16,31 +16,34 @@
 // owner of a row group (rank lg * size / 4) reads the other shares through
 // distributed shared memory, weights each by 2^(m_k - max m), and writes the
 // row's state with coalesced stores.  320 threads:
-//   warps 0-7  softmax: warps lg and lg + 4 share rows 32 lg .. 32 lg + 31
-//              (tensor-memory lanes), each taking 32 of the 64 scores of a
-//              stage; they exchange row maxima through shared memory;
+//   warps 0-7  softmax, two sets of four: set t = warp / 4 takes the stages
+//              s = t, t + 2, t + 4, ... of this CTA's share, warp lg = warp % 4
+//              of a set the rows 32 lg .. 32 lg + 31 (its tensor-memory lanes)
+//              and all 64 scores of each of its stages;
 //   warp 8     producer: TMA loads of 64 prefix tokens (4 blocks) of K and V
 //              per stage into a 6-stage ring, from the kernel's start on;
-//   warp 9     allocates the tensor memory; its lane 0 issues every MMA.
-// Per stage s:  S_s = Q K_s^T (M 128, N 64 keys, K 128) into one of three S
-// buffers in tensor memory; the softmax warps read their S row, turn it into
-// probabilities P_s (16-bit, tensor memory) and the MMA thread accumulates
-// O += P_s V_s (M 128, N 128 dims, K 64 keys) in tensor memory.  S runs up to
-// two stages ahead of the softmax, so that the softmax of a stage never waits
-// for the tensor cores; P is double-buffered, so that the softmax of stage
-// s + 1 does not wait for O += P V of stage s.  The running maximum
-// is only moved (and O, l rescaled) when a row's maximum grows by more than
-// 2^8, so that O rarely makes a round trip through registers; P stays below
-// 2^8.
+//   warp 9     allocates the tensor memory and issues every MMA (the warp
+//              runs the issue loop converged, one elected lane issues).
+// Per stage s:  S_s = Q K_s^T (M 128, N 64 keys, K 128) into S buffer s % 3
+// of tensor memory; the softmax warps of set s % 2 read their S row, turn it
+// into probabilities P_s (16-bit, written over the first half of the same S
+// buffer) and the MMA thread accumulates O_t += P_s V_s (M 128, N 128 dims,
+// K 64 keys) into the set's own accumulator O_t.  The two sets keep separate
+// running maxima, sums and accumulators, so that the softmax of stage s + 1
+// runs while that of stage s is still in flight; they are combined, like the
+// shares of a cluster, after the last stage.  The running maximum is only
+// moved (and O_t, l rescaled) when a row's maximum grows by more than 2^8, so
+// that O_t rarely makes a round trip through registers; P stays below 2^8.
 //
 // Q and P, the A operands, live in tensor memory (lane = row).  The B
 // operands are in shared memory with the 128-byte swizzle (16-byte chunk c
 // of a 128-byte row r at chunk c ^ (r % 8)), in 1 KiB atoms of 8 rows:
-//   K     K-major B operand:  [64-dim block][64 tokens][128 B];
+//   K     K-major B operand:  [block][8-token group][64-dim half][8 tokens][128 B],
+//         so that the 8-token atoms of one dim half lie 2 KiB apart;
 //   V     MN-major B operand: [block][64-dim half][16 tokens][128 B].
-// K lands from the decode kernel's tensor map (one 16-row x 128-byte box per
-// block and 64-dim half), V from a 5-D map over the same cache whose box is a
-// block's whole tile.
+// Each lands as one TMA request per block: K through a 5-D map whose
+// dimensions are (64 dims, 8 tokens, dim half, token group, block x kv head),
+// V through a 5-D map whose box is a block's whole tile.
 #pragma once
 
 #include "pkv_prefix.cuh"
@@ -50,25 +53,25 @@ namespace pkv {
 constexpr int kTcRows = 128;                  // query rows per CTA (M)
 constexpr int kTcKeys = 64;                   // prefix tokens per stage (N of S, K of P V)
 constexpr int kTcBlocks = kTcKeys / kBlockTokens;
-constexpr int kTcSoftmaxWarps = 8;           // two per row group of 32: each takes 32 of the 64 scores
+constexpr int kTcSoftmaxWarps = 8;           // two sets of four: even and odd stages
+constexpr int kTcSetWarps = 4;
 constexpr int kTcProducerWarp = 8;
 constexpr int kTcMmaWarp = 9;
 constexpr int kTcThreads = 320;
 constexpr int kTcKVBytes = kTcKeys * 128 * 2;       // K (or V) of one stage: 64 tokens x 128 dims, 16 KiB
-constexpr int kTcKVHalf = kTcKVBytes / 2;           // one 64-dim block: 8 KiB
+constexpr int kTcBlockBytes = kTcKVBytes / kTcBlocks;  // one block's K (or V): 4 KiB
 constexpr int kTcStageBytes = 2 * kTcKVBytes;       // K and V of one stage
 constexpr int kTcStages = 6;
 constexpr int kTcSmemBytes = kTcStages * kTcStageBytes;  // the K/V ring, 192 KiB
-constexpr int kTcSBufs = 3;             // S buffers in tensor memory: S is issued two stages ahead
+constexpr int kTcSBufs = 3;             // S buffers in tensor memory (P of a stage overwrites its S)
 // Tensor-memory columns (one fp32 or one pair of 16-bit values each):
-// S0 [0,64), S1 [64,128), S2 [128,192), O [256,384), Q [384,448) and two P
-// buffers [448,480), [480,512).  Q and P are the A operands of the two MMAs,
-// read from tensor memory, so that the tensor cores fetch only K and V from
-// shared memory.
+// S0 [0,64), S1 [64,128), S2 [128,192), Q [192,256), O_0 [256,384) and
+// O_1 [384,512).  Q and P, the A operands of the two MMAs, are read from
+// tensor memory, so that the tensor cores fetch only K and V from shared
+// memory; P_s takes the first 32 columns of S buffer s % 3.
 constexpr uint32_t kTcTmemCols = 512;
-constexpr uint32_t kTcOCol = 256;
-constexpr uint32_t kTcQCol = 384;
-constexpr uint32_t kTcPCol = 448;
+constexpr uint32_t kTcQCol = 192;
+constexpr uint32_t kTcOCol = 256;       // O_t at kTcOCol + 128 t
 constexpr int kTcMaxSplit = 4;          // CTAs per cluster (prefix shares per tile)
 constexpr int kTcPartStride = 128 + 4;  // floats per row of a partial O in shared memory (float4 accesses
                                         // of 8 consecutive rows fall in distinct bank groups)
@@ -80,10 +83,12 @@ static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcStages * kTcSt
 constexpr int kTcOutOffset = 68 * 1024;
 static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcOutOffset, "partial state before the output rows");
 static_assert(kTcOutOffset + kTcRows * 512 <= kTcSmemBytes, "output rows fit in the drained ring");
-// Barriers, tensor-memory slot and abort flag, then the softmax exchange
-// arrays (pair maxima [2][2][128], pair sums [2][128], destination rows [128]).
-constexpr int kTcBarBytes = (2 * kTcStages + 2 * kTcSBufs + 4) * 8 + 16;
-constexpr int kTcExchBytes = (4 * kTcRows + 2 * kTcRows + kTcRows) * 4;
+// Barriers (K/V full and empty per ring slot; S full, S buffer free and P
+// full per S buffer; O_t updated per set; one to drain the MMAs on an abort),
+// the tensor-memory slot and the abort flag, then the exchange arrays of
+// the set merge (maxima [2][128], sums [2][128]) and the destination rows [128].
+constexpr int kTcBarBytes = (2 * kTcStages + 3 * kTcSBufs + 2 + 1) * 8 + 16;
+constexpr int kTcExchBytes = (2 * kTcRows + 2 * kTcRows + kTcRows) * 4;
 
 // Softmax arithmetic with fewer issue slots: two fp32 lanes per packed FMA /
 // add (sm_100), two new values per three-input max, and the hardware base-2
@@ -172,17 +177,24 @@ __host__ __device__ constexpr uint32_t tc_idesc(bool b_mn_major, uint32_t n) {
 // memory), A (M x 16, 16-bit) in tensor memory (lane = row, each 32-bit
 // column a pair of consecutive K elements), B from a shared-memory
 // descriptor.
+// Executed by a whole converged warp: the operands are the same in every
+// lane and one elected lane issues the MMA (so that the warp's control flow
+// and operand arithmetic stay uniform).
 __device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
                                           bool accumulate) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
       "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
+// The mbarrier tracks the completion of every MMA the elected lane (the
+// same lane as in tc_mma_ts) has issued; executed by the whole warp.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -231,27 +243,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                          const PrefixParams p) {
   constexpr bool kBf16 = (DT == kBF16);
   constexpr int D = 128;
-  constexpr int X = 64;  // 16-bit elements per 128-byte row
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* ring = base;                     // [stage]{K, V}: K [2][64 tokens][128 B], V [4 blocks][2][16][128 B]
+  uint8_t* ring = base;                     // [stage]{K, V}: K [4 blocks][2][2][8][128 B], V [4 blocks][2][16][128 B]
   uint8_t* out_s = ring + kTcOutOffset;     // after the last stage: the merged output rows, [128 rows][512 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kTcStages * kTcStageBytes);
   uint64_t* kv_full = bars;                // [kTcStages]
   uint64_t* kv_empty = bars + kTcStages;   // [kTcStages]
-  uint64_t* s_full = bars + 2 * kTcStages; // [kTcSBufs]
-  uint64_t* s_free = s_full + kTcSBufs;    // [kTcSBufs]
-  uint64_t* p_full = s_free + kTcSBufs;    // [2]: P of stages with that parity written
-  uint64_t* o_done = p_full + 2;           // [2]: P V of stages with that parity (P buffer free, O updated)
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(o_done + 2);
+  uint64_t* s_full = bars + 2 * kTcStages; // [kTcSBufs]: S written
+  uint64_t* s_free = s_full + kTcSBufs;    // [kTcSBufs]: P V of the buffer's stage done (buffer free)
+  uint64_t* p_full = s_free + kTcSBufs;    // [kTcSBufs]: P written by the four warps of the stage's set
+  uint64_t* o_done = p_full + kTcSBufs;    // [2]: a P V into O_t done
+  uint64_t* mma_drain = o_done + 2;        // every MMA issued done (abort path)
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red_max = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kTcBarBytes);  // [2][2][128]
-  float* red_l = red_max + 4 * kTcRows;                                                     // [2][128]
+  float* red_max = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kTcBarBytes);  // [2][128]
+  float* red_l = red_max + 2 * kTcRows;                                                     // [2][128]
   int* row_dst = reinterpret_cast<int*>(red_l + 2 * kTcRows);                               // [128]
   int* members = row_dst + kTcRows;                                                         // [batch]
   __shared__ int warp_counts[kTcThreads / 32];
+  __shared__ int set_ok[2][kTcSetWarps];
   __shared__ int n_members;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -266,12 +279,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < kTcSBufs; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kTcSoftmaxWarps);
+      mbar_init(&s_free[i], 1);
+      mbar_init(&p_full[i], kTcSetWarps);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&p_full[i], kTcSoftmaxWarps);
-      mbar_init(&o_done[i], 1);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -323,25 +335,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (plen_bad && threadIdx.x == 0) flag_error(PKV_DEVERR_CONTEXT);
 
-  // Softmax-warp geometry: row group lg (tensor-memory lanes 32 lg ..), half hf of the scores.
+  // Softmax-warp geometry: row group lg (tensor-memory lanes 32 lg ..) and
+  // set hf (stages of parity hf); after the last stage, warp (lg, hf) also
+  // takes the dims [64 hf, 64 hf + 64) of its rows.
   const int lg = warp & 3, hf = (warp >> 2) & 1;
   const int r = lg * 32 + lane;
   const uint32_t owner = static_cast<uint32_t>(lg) * csize / 4;  // cluster rank that writes these rows
   float m_ref = -INFINITY, l_row = 0.f;                           // the softmax thread's row state
+  float set_w[2] = {0.f, 0.f};                                    // weights of O_0, O_1 in the row's O
   bool ok = true;
   uint32_t tmem = 0;
+  // Columns [64 hf + 32 c, + 32) of this row's O, the two sets' accumulators
+  // combined (an accumulator of a set with no stage is never read).
+  auto load_o = [&](int c, float (&t)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) t[i] = 0.f;
+    if (!ok) return;
+    const uint32_t col = tmem + (static_cast<uint32_t>(lg * 32) << 16) + kTcOCol + hf * 64 + c * 32;
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+      if (n_stages > st) {
+        float u[32];
+        tmem_ld32(col + st * D, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) t[i] = fmaf(set_w[st], u[i], t[i]);
+      }
+    }
+  };
 
   if (warp == kTcProducerWarp) {
-    // ---------------- producer: 12 TMA requests per stage ----------------
-    // Lanes 0-7: K, block lane / 2, dim half lane % 2 (one 16-token x 64-dim
-    // box each); lanes 8-11: V of block lane - 8 (one 16-token x 128-dim box).
-    // Starts at once: the copies of the first stages overlap the Q load.
+    // ---------------- producer: 8 TMA requests per stage ----------------
+    // Lanes 0-3: K of block `lane`, lanes 4-7: V of block lane - 4, each one
+    // box of the block's whole 16-token x 128-dim tile.  Starts at once: the
+    // copies of the first stages overlap the Q load.
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
-    const bool is_k = lane < 2 * kTcBlocks, is_v = !is_k && lane < 3 * kTcBlocks;
-    const int blk = is_k ? lane >> 1 : is_v ? lane - 2 * kTcBlocks : 0, y = lane & 1;
+    const int n_kv = p.n_q_heads / G;
+    const bool is_k = lane < kTcBlocks, is_v = !is_k && lane < 2 * kTcBlocks;
+    const int blk = is_k ? lane : is_v ? lane - kTcBlocks : 0;
     int issued = 0;
     for (int s = 0; s < n_stages; ++s) {
       const int slot = s % kTcStages;
@@ -360,10 +394,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], kTcStageBytes);
       __syncwarp();
       uint8_t* stage = ring + slot * kTcStageBytes;
-      if (is_k) tma_load_4d(stage + y * kTcKVHalf + blk * (kBlockTokens * 128), &tm_k, &kv_full[slot], y * X, 0, kvh,
-                            phys);
-      if (is_v) tma_load_5d(stage + kTcKVBytes + blk * (2 * kBlockTokens * 128), &tm_v, &kv_full[slot], 0, 0, 0, kvh,
-                            phys);
+      if (is_k) tma_load_5d(stage + blk * kTcBlockBytes, &tm_k, &kv_full[slot], 0, 0, 0, 0, phys * n_kv + kvh);
+      if (is_v) tma_load_5d(stage + kTcKVBytes + blk * kTcBlockBytes, &tm_v, &kv_full[slot], 0, 0, 0, kvh, phys);
       ++issued;
     }
     // Do not leave while copies may still be landing.
@@ -421,147 +453,182 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
 
     if (warp == kTcMmaWarp) {
-      // ---------------- MMA issue (one thread) ----------------
+      // ---------------- MMA issue (the whole warp, one elected lane) ----------------
       // S of a stage is issued as soon as its K has landed and its S buffer
-      // is free (up to two stages ahead of the softmax), O += P V as soon as
-      // its P is written; the thread polls both and issues in stage order
-      // within each kind.
-      if (lane == 0 && n_stages > 0) {
+      // is free (P V of the stage three back done), O_t += P V as soon as
+      // its P is written; the warp polls both and issues in stage order
+      // within each kind.  Decisions are taken from lane 0, so that the
+      // warp stays converged.
+      if (n_stages > 0) {
         constexpr uint32_t kIdS = tc_idesc<kBf16>(false, kTcKeys), kIdPV = tc_idesc<kBf16>(true, D);
         const uint32_t ra = smem_u32(ring);
+        // Descriptors of ring slot 0's K (dims 0-15) and V (block 0); the
+        // other operands add a start-address offset (16-byte units).
+        const uint64_t dk0 = smem_desc_sw128(ra, 16, 2048);
+        const uint64_t dv0 = smem_desc_sw128(ra + kTcKVBytes, kBlockTokens * 128, 1024);
         int ns = 0, np = 0;  // next stage whose S, whose P V is to be issued
-        uint64_t t0 = global_timer_ns();
+        uint64_t t0 = 0;
+        uint32_t idle = 0;
         bool mok = true;
         while (np < n_stages) {
           bool progress = false;
-          if (ns < n_stages && mbar_test_wait(&kv_full[ns % kTcStages], (ns / kTcStages) & 1) &&
-              (ns < kTcSBufs || mbar_test_wait(&s_free[ns % kTcSBufs], ((ns - kTcSBufs) / kTcSBufs) & 1))) {
+          // The buffer's previous P V must have been issued before its
+          // barrier's parity says anything about it.
+          bool go = ns < n_stages && (ns < kTcSBufs || np > ns - kTcSBufs) &&
+                    mbar_test_wait(&kv_full[ns % kTcStages], (ns / kTcStages) & 1) &&
+                    (ns < kTcSBufs || mbar_test_wait(&s_free[ns % kTcSBufs], ((ns - kTcSBufs) / kTcSBufs) & 1));
+          if (__shfl_sync(0xffffffffu, go, 0)) {
             tc_fence_after();
-            const uint32_t ka = ra + (ns % kTcStages) * kTcStageBytes;
+            const uint64_t dk = dk0 + static_cast<uint64_t>(((ns % kTcStages) * kTcStageBytes) >> 4);
             const uint32_t d = tmem + (ns % kTcSBufs) * kTcKeys;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              tc_mma_ts(d, tmem + kTcQCol + kk * 8, smem_desc_sw128(ka + (kk >> 2) * kTcKVHalf + (kk & 3) * 32, 16, 1024),
+              // Dims 16 kk ..: dim half kk / 4, 32-byte step kk % 4 of its
+              // 128-byte rows; the 8-token atoms of the half lie 2 KiB apart.
+              tc_mma_ts(d, tmem + kTcQCol + kk * 8, dk + static_cast<uint64_t>(((kk >> 2) * 1024 + (kk & 3) * 32) >> 4),
                         kIdS, kk > 0);
             }
             tc_commit(&s_full[ns % kTcSBufs]);
             ++ns;
             progress = true;
           }
-          if (np < ns && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
+          go = np < ns && mbar_test_wait(&p_full[np % kTcSBufs], (np / kTcSBufs) & 1);
+          if (__shfl_sync(0xffffffffu, go, 0)) {
             tc_fence_after();
-            const uint32_t va = ra + (np % kTcStages) * kTcStageBytes + kTcKVBytes;
+            const uint64_t dv = dv0 + static_cast<uint64_t>(((np % kTcStages) * kTcStageBytes) >> 4);
+            const uint32_t pa = tmem + (np % kTcSBufs) * kTcKeys;
 #pragma unroll
             for (int kt = 0; kt < kTcKeys / 16; ++kt) {
               // V of block kt: [half][16 tokens][128 B], halves 2 KiB apart.
-              tc_mma_ts(tmem + kTcOCol, tmem + kTcPCol + (np & 1) * (kTcKeys / 2) + kt * 8,
-                        smem_desc_sw128(va + kt * 2 * kBlockTokens * 128, kBlockTokens * 128, 1024), kIdPV,
-                        np > 0 || kt > 0);
+              tc_mma_ts(tmem + kTcOCol + (np & 1) * D, pa + kt * 8,
+                        dv + static_cast<uint64_t>((kt * kTcBlockBytes) >> 4), kIdPV, np > 1 || kt > 0);
             }
             tc_commit(&o_done[np & 1]);
+            tc_commit(&s_free[np % kTcSBufs]);
             tc_commit(&kv_empty[np % kTcStages]);
             ++np;
             progress = true;
           }
+          int st = 0;  // 0 go on, 1 another warp gave up, 2 the limit passed
           if (progress) {
-            t0 = global_timer_ns();
-          } else if (*abort_flag) {
-            mok = false;
-            break;
-          } else if (global_timer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            flag_error(kDevErrTimeout);
+            idle = 0;
+          } else if ((++idle & 1023u) == 0) {
+            // The clock is read once per 1024 idle polls: the first read
+            // after progress starts the limit, later ones test it.
+            const uint64_t now = global_timer_ns();
+            if (idle == 1024u) t0 = now;
+            st = *abort_flag ? 1 : (now - t0 > kWaitLimitNs) ? 2 : 0;
+          }
+          st = __shfl_sync(0xffffffffu, st, 0);
+          if (st != 0) {
+            if (st == 2 && lane == 0) {
+              *abort_flag = 1;
+              flag_error(kDevErrTimeout);
+            }
             mok = false;
             break;
           }
         }
         // Before the tensor memory is freed, every MMA issued must have completed.
-        if (!mok && np > 0)
-          mbar_wait_bounded(&o_done[(np - 1) & 1], ((np - 1) >> 1) & 1, abort_flag, kWaitLimitNs);
+        if (!mok && ns > 0) {
+          tc_commit(mma_drain);
+          if (lane == 0) {
+            const uint64_t t1 = global_timer_ns();
+            while (!mbar_try_wait(mma_drain, 0) && global_timer_ns() - t1 < kWaitLimitNs) {
+            }
+          }
+          __syncwarp();
+        }
       }
     } else {
-      // ---------------- softmax: warps (lg, hf) share rows 32 lg .. 32 lg + 31 ----------------
+      // ---------------- softmax: set hf, rows 32 lg .. 32 lg + 31 ----------------
       // Every tensor-memory access is warp-converged (.sync.aligned): waits
-      // and decisions are made warp-uniform first.  The pair barrier is
-      // reached on every stage, also after a failed wait, so that the two
-      // warps of a pair never wait for each other in vain.
+      // and decisions are made warp-uniform first.  After a failed wait the
+      // warp still arrives on every P barrier, so that nothing waits for it
+      // in vain.
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(lg * 32) << 16);
+      const uint32_t o_col = kTcOCol + hf * D;
       const float sc = fabsf(p.scale_log2);
-      float l_half = 0.f;
-      // Block ids of this half's two blocks, read one stage ahead: a block
+      float l_set = 0.f;
+      // Block ids of a stage's four blocks, read one own stage ahead: a block
       // whose id is outside the pool contributes no key (its copy read block
       // 0, whose scores are masked here).
-      auto half_ids = [&](int s, int& a, int& b) {
-        const int j = (s_begin + s) * kTcBlocks + 2 * hf;
-        a = j < n_prefix_blocks ? __ldg(tab + j) : 0;
-        b = j + 1 < n_prefix_blocks ? __ldg(tab + j + 1) : 0;
+      auto bad_mask = [&](int s) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < kTcBlocks; ++i) {
+          const int j = (s_begin + s) * kTcBlocks + i;
+          const int id = j < n_prefix_blocks ? __ldg(tab + j) : 0;
+          if (id < 0 || id >= p.num_blocks) m |= 1u << i;
+        }
+        return m;
       };
-      int id_next0 = 0, id_next1 = 0;
-      if (n_stages > 0) half_ids(0, id_next0, id_next1);
-      for (int s = 0; s < n_stages; ++s) {
-        const int id0 = id_next0, id1 = id_next1;
-        if (s + 1 < n_stages) half_ids(s + 1, id_next0, id_next1);
+      uint32_t bad_next = hf < n_stages ? bad_mask(hf) : 0u;
+      int k = 0;  // this set's stage count so far
+      for (int s = hf; s < n_stages; s += 2, ++k) {
+        const uint32_t bad = bad_next;
+        if (s + 2 < n_stages) bad_next = bad_mask(s + 2);
         const int sb = s % kTcSBufs;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[sb], (s / kTcSBufs) & 1, abort_flag,
                                                                 kWaitLimitNs));
-        float x[32];
+        float x[64];
         if (ok) {
           tc_fence_after();
-          tmem_ld32(lane_base + sb * kTcKeys + hf * 32, x);
+          float xa[32], xb[32];
+          tmem_ld32(lane_base + sb * kTcKeys, xa);
+          tmem_ld32(lane_base + sb * kTcKeys + 32, xb);
           tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            x[i] = xa[i];
+            x[32 + i] = xb[i];
+          }
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = 0.f;
+          for (int i = 0; i < 64; ++i) x[i] = 0.f;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[sb]);
 
         // Scores past the prefix (only in the last stage) and those of a bad
-        // block are masked: bit i of `keep` is this half's score i.
-        const int live = min(kTcKeys, plen - (s_begin + s) * kTcKeys) - hf * 32;
-        uint32_t keep = live >= 32 ? 0xffffffffu : live <= 0 ? 0u : (1u << live) - 1u;
-        if (id0 < 0 || id0 >= p.num_blocks) keep &= 0xffff0000u;
-        if (id1 < 0 || id1 >= p.num_blocks) keep &= 0x0000ffffu;
-        if (keep != 0xffffffffu) {
+        // block are masked: bit i of keep[h] is score 32 h + i.
+        const int live = min(kTcKeys, plen - (s_begin + s) * kTcKeys);
+        uint32_t keep[2];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = ((keep >> i) & 1u) ? x[i] : -INFINITY;
+        for (int h = 0; h < 2; ++h) {
+          const int lv = live - 32 * h;
+          keep[h] = lv >= 32 ? 0xffffffffu : lv <= 0 ? 0u : (1u << lv) - 1u;
+          if (bad & (1u << (2 * h))) keep[h] &= 0xffff0000u;
+          if (bad & (2u << (2 * h))) keep[h] &= 0x0000ffffu;
+        }
+        const bool masked = (keep[0] & keep[1]) != 0xffffffffu;
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) x[i] = ((keep[i >> 5] >> (i & 31)) & 1u) ? x[i] : -INFINITY;
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], x[i], x[i + 1]);
+        for (int i = 0; i < 64; i += 2) mx4[(i >> 1) & 3] = max3f(mx4[(i >> 1) & 3], x[i], x[i + 1]);
         float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        mx = keep != 0u ? mx * sc : -INFINITY;  // the maximum of the scaled scores (sc >= 0)
-        red_max[((s & 1) * 2 + hf) * kTcRows + r] = mx;
-        named_bar_sync(2 + lg, 64);
-        mx = fmaxf(mx, red_max[((s & 1) * 2 + (hf ^ 1)) * kTcRows + r]);  // the row's maximum, same in both
-        // P buffer s % 2 is free once P V of stage s - 2 is done.
-        if (ok && s >= 2) {
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait_bounded(&o_done[s & 1], ((s - 2) >> 1) & 1, abort_flag, kWaitLimitNs));
-          if (ok) tc_fence_after();
-        }
+        mx = (keep[0] | keep[1]) != 0u ? mx * sc : -INFINITY;  // the maximum of the scaled scores (sc >= 0)
         // Move the reference maximum only when it grows by more than 2^8 (so
-        // that O rarely makes the round trip); when any row of the warp
-        // moves, the warp takes the round trip for its 64 columns of O, with
-        // factor 1 for the rows that stay.  O is stable once P V of stage
-        // s - 1 is done.  Both warps of a pair decide alike.
+        // that O_t rarely makes the round trip); when any row of the warp
+        // moves, the warp takes the round trip for its 128 columns of O_t,
+        // with factor 1 for the rows that stay.  O_t is stable once the set's
+        // previous P V is done.
         const bool move = mx > m_ref + 8.f;
-        if (ok && s > 0 && __any_sync(0xffffffffu, move)) {
-          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(s - 1) & 1], ((s - 1) >> 1) & 1, abort_flag,
-                                                         kWaitLimitNs));
+        if (ok && k > 0 && __any_sync(0xffffffffu, move)) {
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[hf], (k - 1) & 1, abort_flag, kWaitLimitNs));
           if (ok) {
             tc_fence_after();
             const float alpha = move ? exp2f(m_ref - mx) : 1.f;
-            l_half *= alpha;
+            l_set *= alpha;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
               float v[32];
-              tmem_ld32(lane_base + kTcOCol + hf * 64 + c * 32, v);
+              tmem_ld32(lane_base + o_col + c * 32, v);
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) v[i] *= alpha;
-              tmem_st32(lane_base + kTcOCol + hf * 64 + c * 32, v);
+              tmem_st32(lane_base + o_col + c * 32, v);
             }
             tmem_wait_st();
           }
@@ -570,42 +637,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         {
           const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) f2_unpack(f2_fma(f2_pack(x[i], x[i + 1]), sc2, nm2), x[i], x[i + 1]);
+          for (int i = 0; i < 64; i += 2) f2_unpack(f2_fma(f2_pack(x[i], x[i + 1]), sc2, nm2), x[i], x[i + 1]);
         }
-        if (keep != 0xffffffffu) {
+        if (masked) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = ((keep >> i) & 1u) ? x[i] : -INFINITY;
+          for (int i = 0; i < 64; ++i) x[i] = ((keep[i >> 5] >> (i & 31)) & 1u) ? x[i] : -INFINITY;
         }
         uint64_t sum2[2] = {0ull, 0ull};
-        uint32_t pw[16];  // this half's 32 probabilities as 16-bit pairs
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float a = ex2_ftz(x[2 * k]), b = ex2_ftz(x[2 * k + 1]);
-          sum2[k & 1] = f2_add(sum2[k & 1], f2_pack(a, b));
-          pw[k] = pack2<kBf16>(a, b);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pw[16];  // 32 probabilities as 16-bit pairs
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float a = ex2_ftz(x[32 * h + 2 * j]), b = ex2_ftz(x[32 * h + 2 * j + 1]);
+            sum2[j & 1] = f2_add(sum2[j & 1], f2_pack(a, b));
+            pw[j] = pack2<kBf16>(a, b);
+          }
+          // P over the first half of the stage's S buffer (its scores are in registers).
+          if (ok) tmem_st16(lane_base + sb * kTcKeys + h * 16, pw);
         }
-        if (ok) {
-          tmem_st16(lane_base + kTcPCol + (s & 1) * (kTcKeys / 2) + hf * 16, pw);
-          tmem_wait_st();
-        }
+        if (ok) tmem_wait_st();
         {
           float a0, a1, b0, b1;
           f2_unpack(sum2[0], a0, a1);
           f2_unpack(sum2[1], b0, b1);
-          l_half += (a0 + a1) + (b0 + b1);
+          l_set += (a0 + a1) + (b0 + b1);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[s & 1]);
+        if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      if (ok && n_stages > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(n_stages - 1) & 1], ((n_stages - 1) >> 1) & 1,
-                                                        abort_flag, kWaitLimitNs));
-      tc_fence_after();
-      // The row's sum over both halves; NaN marks a row whose pipeline failed.
-      red_l[hf * kTcRows + r] = ok ? l_half : __int_as_float(0x7fc00000);
+      // Both sets' accumulators are final once each set's last P V is done.
+      if (ok && k > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[hf], (k - 1) & 1, abort_flag, kWaitLimitNs));
+      // The two sets' states of each row, combined: weights 2^(m_t - max m),
+      // 0 for a set with no keys; NaN in the sum marks a row whose pipeline
+      // failed.
+      red_max[hf * kTcRows + r] = m_ref;
+      red_l[hf * kTcRows + r] = l_set;
+      if (lane == 0) set_ok[hf][lg] = ok ? 1 : 0;
+      tc_fence_before();
       named_bar_sync(2 + lg, 64);
-      l_row = red_l[hf * kTcRows + r] + red_l[(hf ^ 1) * kTcRows + r];
+      tc_fence_after();
+      ok = ok && set_ok[hf ^ 1][lg] != 0;  // warp-uniform
+      {
+        const float m_o = red_max[(hf ^ 1) * kTcRows + r], l_o = red_l[(hf ^ 1) * kTcRows + r];
+        const float m_c = fmaxf(m_ref, m_o);
+        const float a_me = m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_c);
+        const float a_o = m_o == -INFINITY ? 0.f : exp2f(m_o - m_c);
+        l_row = ok ? a_me * l_set + a_o * l_o : __int_as_float(0x7fc00000);
+        set_w[0] = hf == 0 ? a_me : a_o;  // selects, not a dynamic index (which would live on the stack)
+        set_w[1] = hf == 0 ? a_o : a_me;
+        m_ref = m_c;
+      }
       if (owner != crank) {
         // Partial state for the owner of these rows, in the drained ring
         // (every copy into it has been consumed by an MMA that has completed).
@@ -614,13 +698,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           float v[32];
-          if (ok && n_stages > 0) {
-            tmem_ld32(lane_base + kTcOCol + hf * 64 + c * 32, v);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
-          }
+          load_o(c, v);
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4*>(part_o + r * kTcPartStride + hf * 64 + c * 32 + i) =
@@ -640,7 +718,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // The row's state, merged over the cluster: O (unnormalised), m, l.
     const uint32_t part_o_addr = smem_u32(ring);
     const uint32_t part_ml_addr = part_o_addr + kTcRows * kTcPartStride * 4;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(lg * 32) << 16);
     float m_all = m_ref;
     float wk[kTcMaxSplit], lk[kTcMaxSplit];
     bool valid = !isnan(l_row);
@@ -679,13 +756,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       float t[32];
-      if (ok && n_stages > 0) {
-        tmem_ld32(lane_base + kTcOCol + hf * 64 + c * 32, t);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) t[i] = 0.f;
-      }
+      load_o(c, t);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int chunk = (hf * 16 + c * 8 + i) ^ (r & 7);
