@@ -21,10 +21,10 @@
 //              of a set the rows 32 lg .. 32 lg + 31 (its tensor-memory lanes)
 //              and all 64 scores of each of its stages;
 //   warp 8     producer: TMA loads of 64 prefix tokens (4 blocks) of K and V
-//              per stage into a 6-stage ring, from the kernel's start on;
+//              per stage into a 5-stage ring, from the kernel's start on;
 //   warp 9     allocates the tensor memory and issues every MMA (the warp
 //              runs the issue loop converged, one elected lane issues).
-// Per stage s:  S_s = Q K_s^T (M 128, N 64 keys, K 128) into S buffer s % 3
+// Per stage s:  S_s = Q K_s^T (M 128, N 64 keys, K 128) into S buffer s % 4
 // of tensor memory; the softmax warps of set s % 2 read their S row, turn it
 // into probabilities P_s (16-bit, written over the first half of the same S
 // buffer) and the MMA thread accumulates O_t += P_s V_s (M 128, N 128 dims,
@@ -35,9 +35,11 @@
 // moved (and O_t, l rescaled) when a row's maximum grows by more than 2^8, so
 // that O_t rarely makes a round trip through registers; P stays below 2^8.
 //
-// Q and P, the A operands, live in tensor memory (lane = row).  The B
-// operands are in shared memory with the 128-byte swizzle (16-byte chunk c
-// of a 128-byte row r at chunk c ^ (r % 8)), in 1 KiB atoms of 8 rows:
+// P, the A operand of P V, lives in tensor memory (lane = row).  Q, the A
+// operand of S, and the B operands are in shared memory with the 128-byte
+// swizzle (16-byte chunk c of a 128-byte row r at chunk c ^ (r % 8)), in 1 KiB
+// atoms of 8 rows:
+//   Q     K-major A operand:  [64-dim half][128 rows][128 B];
 //   K     K-major B operand:  [block][8-token group][64-dim half][8 tokens][128 B],
 //         so that the 8-token atoms of one dim half lie 2 KiB apart;
 //   V     MN-major B operand: [block][64-dim half][16 tokens][128 B].
@@ -61,33 +63,34 @@ constexpr int kTcThreads = 320;
 constexpr int kTcKVBytes = kTcKeys * 128 * 2;       // K (or V) of one stage: 64 tokens x 128 dims, 16 KiB
 constexpr int kTcBlockBytes = kTcKVBytes / kTcBlocks;  // one block's K (or V): 4 KiB
 constexpr int kTcStageBytes = 2 * kTcKVBytes;       // K and V of one stage
-constexpr int kTcStages = 6;
-constexpr int kTcSmemBytes = kTcStages * kTcStageBytes;  // the K/V ring, 192 KiB
-constexpr int kTcSBufs = 3;             // S buffers in tensor memory (P of a stage overwrites its S)
-// Tensor-memory columns (one fp32 or one pair of 16-bit values each):
-// S0 [0,64), S1 [64,128), S2 [128,192), Q [192,256), O_0 [256,384) and
-// O_1 [384,512).  Q and P, the A operands of the two MMAs, are read from
-// tensor memory, so that the tensor cores fetch only K and V from shared
-// memory; P_s takes the first 32 columns of S buffer s % 3.
+constexpr int kTcStages = 5;
+constexpr int kTcRingBytes = kTcStages * kTcStageBytes;  // the K/V ring, 160 KiB
+constexpr int kTcQBytes = kTcRows * 128 * 2;             // Q: [64-dim half][128 rows][128 B], 32 KiB
+constexpr int kTcSmemBytes = kTcRingBytes + kTcQBytes;
+constexpr int kTcSBufs = 4;             // S buffers in tensor memory (P of a stage overwrites its S)
+// Tensor-memory columns (one fp32 or one pair of 16-bit values each): S
+// buffer i at [64 i, 64 i + 64) for i < 4, O_0 [256,384) and O_1 [384,512).
+// P_s, the A operand of P V, takes the first 32 columns of S buffer s % 4;
+// Q, the A operand of S, is in shared memory.  S of stage s + 4 waits for P V
+// of stage s, so that the issuing warp rarely waits for a P V to complete.
 constexpr uint32_t kTcTmemCols = 512;
-constexpr uint32_t kTcQCol = 192;
 constexpr uint32_t kTcOCol = 256;       // O_t at kTcOCol + 128 t
 constexpr int kTcMaxSplit = 4;          // CTAs per cluster (prefix shares per tile)
 constexpr int kTcPartStride = 128 + 4;  // floats per row of a partial O in shared memory (float4 accesses
                                         // of 8 consecutive rows fall in distinct bank groups)
-static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcStages * kTcStageBytes,
+static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcRingBytes,
               "a partial state fits in the drained K/V ring");
 // After the last stage the drained ring holds a CTA's partial state for the
 // rows it does not own (from byte 0) and the output rows it owns (from
 // kTcOutOffset).
 constexpr int kTcOutOffset = 68 * 1024;
 static_assert(kTcRows * kTcPartStride * 4 + 2 * kTcRows * 4 <= kTcOutOffset, "partial state before the output rows");
-static_assert(kTcOutOffset + kTcRows * 512 <= kTcSmemBytes, "output rows fit in the drained ring");
+static_assert(kTcOutOffset + kTcRows * 512 <= kTcRingBytes, "output rows fit in the drained ring");
 // Barriers (K/V full and empty per ring slot; S full, S buffer free and P
-// full per S buffer; O_t updated per set; one to drain the MMAs on an abort),
-// the tensor-memory slot and the abort flag, then the exchange arrays of
-// the set merge (maxima [2][128], sums [2][128]) and the destination rows [128].
-constexpr int kTcBarBytes = (2 * kTcStages + 3 * kTcSBufs + 2 + 1) * 8 + 16;
+// full per S buffer; one to drain the MMAs on an abort), the tensor-memory
+// slot and the abort flag, then the exchange arrays of the set merge (maxima
+// [2][128], sums [2][128]) and the destination rows [128].
+constexpr int kTcBarBytes = (2 * kTcStages + 3 * kTcSBufs + 1) * 8 + 16;
 constexpr int kTcExchBytes = (2 * kTcRows + 2 * kTcRows + kTcRows) * 4;
 
 // Softmax arithmetic with fewer issue slots: two fp32 lanes per packed FMA /
@@ -188,6 +191,14 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint
       "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
+// The same with A from a shared-memory descriptor as well.
+__device__ __forceinline__ void tc_mma_ss(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
 // The mbarrier tracks the completion of every MMA the elected lane (the
 // same lane as in tc_mma_ts) has issued; executed by the whole warp.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -249,14 +260,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* ring = base;                     // [stage]{K, V}: K [4 blocks][2][2][8][128 B], V [4 blocks][2][16][128 B]
   uint8_t* out_s = ring + kTcOutOffset;     // after the last stage: the merged output rows, [128 rows][512 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kTcStages * kTcStageBytes);
+  uint8_t* q_s = ring + kTcRingBytes;     // Q, the K-major A operand of S: [half][128 rows][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(q_s + kTcQBytes);
   uint64_t* kv_full = bars;                // [kTcStages]
   uint64_t* kv_empty = bars + kTcStages;   // [kTcStages]
   uint64_t* s_full = bars + 2 * kTcStages; // [kTcSBufs]: S written
   uint64_t* s_free = s_full + kTcSBufs;    // [kTcSBufs]: P V of the buffer's stage done (buffer free)
   uint64_t* p_full = s_free + kTcSBufs;    // [kTcSBufs]: P written by the four warps of the stage's set
-  uint64_t* o_done = p_full + kTcSBufs;    // [2]: a P V into O_t done
-  uint64_t* mma_drain = o_done + 2;        // every MMA issued done (abort path)
+  uint64_t* mma_drain = p_full + kTcSBufs; // every MMA issued done (abort path)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red_max = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kTcBarBytes);  // [2][128]
@@ -282,7 +293,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&s_free[i], 1);
       mbar_init(&p_full[i], kTcSetWarps);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -411,15 +421,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   } else {
-    float qv[32];  // a softmax thread's 64 dims of its Q row, as 32 pairs
     if (warp == kTcMmaWarp) {
       asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                        smem_u32(const_cast<uint32_t*>(tmem_slot))),
                    "r"(kTcTmemCols));
       asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     } else {
-      // Q rows into tensor memory (zero rows past R): softmax warp (lg, hf)
-      // writes dims [64 hf, 64 hf + 64) of its 32 rows (lanes).
+      // Q rows into shared memory (zero rows past R): softmax warp (lg, hf)
+      // writes dims [64 hf, 64 hf + 64) of its 32 rows (lanes), 16-byte
+      // chunk c of row r at chunk c ^ (r % 8) (the 128-byte swizzle).
       // A negative scale is taken as |scale| on -Q (exact), so that the
       // softmax can take its maximum over the raw scores.
       const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
@@ -431,31 +441,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.q) +
                                              (static_cast<size_t>(b) * p.n_q_heads + h) * D * 2);
       }
+      uint4 v[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = src ? __ldg(src + c0 + c) : make_uint4(0u, 0u, 0u, 0u);
-        qv[4 * c] = __uint_as_float(v.x ^ flip);
-        qv[4 * c + 1] = __uint_as_float(v.y ^ flip);
-        qv[4 * c + 2] = __uint_as_float(v.z ^ flip);
-        qv[4 * c + 3] = __uint_as_float(v.w ^ flip);
-      }
+      for (int c = 0; c < 8; ++c) v[c] = src ? __ldg(src + c0 + c) : make_uint4(0u, 0u, 0u, 0u);
+      uint8_t* qrow = q_s + hf * (kTcRows * 128) + qr * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(qrow + ((c ^ (qr & 7)) * 16)) =
+            make_uint4(v[c].x ^ flip, v[c].y ^ flip, v[c].z ^ flip, v[c].w ^ flip);
+      // Generic-proxy writes, read by the tensor cores (async proxy).
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     tc_fence_before();
-    named_bar_sync(1, (kTcSoftmaxWarps + 1) * 32);  // softmax warps and the MMA warp: tensor memory allocated
+    named_bar_sync(1, (kTcSoftmaxWarps + 1) * 32);  // tensor memory allocated, Q in shared memory
     tc_fence_after();
     tmem = *tmem_slot;
-    if (warp != kTcMmaWarp) {
-      tmem_st32(tmem + (static_cast<uint32_t>(lg * 32) << 16) + kTcQCol + hf * 32, qv);
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    named_bar_sync(1, (kTcSoftmaxWarps + 1) * 32);  // Q is in tensor memory
-    tc_fence_after();
 
     if (warp == kTcMmaWarp) {
       // ---------------- MMA issue (the whole warp, one elected lane) ----------------
       // S of a stage is issued as soon as its K has landed and its S buffer
-      // is free (P V of the stage three back done), O_t += P V as soon as
+      // is free (P V of the stage four back done), O_t += P V as soon as
       // its P is written; the warp polls both and issues in stage order
       // within each kind.  Decisions are taken from lane 0, so that the
       // warp stays converged.
@@ -465,6 +470,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // Descriptors of ring slot 0's K (dims 0-15) and V (block 0); the
         // other operands add a start-address offset (16-byte units).
         const uint64_t dk0 = smem_desc_sw128(ra, 16, 2048);
+        const uint64_t dq0 = smem_desc_sw128(smem_u32(q_s), 16, 1024);
         const uint64_t dv0 = smem_desc_sw128(ra + kTcKVBytes, kBlockTokens * 128, 1024);
         int ns = 0, np = 0;  // next stage whose S, whose P V is to be issued
         uint64_t t0 = 0;
@@ -485,8 +491,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int kk = 0; kk < D / 16; ++kk) {
               // Dims 16 kk ..: dim half kk / 4, 32-byte step kk % 4 of its
               // 128-byte rows; the 8-token atoms of the half lie 2 KiB apart.
-              tc_mma_ts(d, tmem + kTcQCol + kk * 8, dk + static_cast<uint64_t>(((kk >> 2) * 1024 + (kk & 3) * 32) >> 4),
-                        kIdS, kk > 0);
+              tc_mma_ss(d, dq0 + static_cast<uint64_t>(((kk >> 2) * (kTcRows * 128) + (kk & 3) * 32) >> 4),
+                        dk + static_cast<uint64_t>(((kk >> 2) * 1024 + (kk & 3) * 32) >> 4), kIdS, kk > 0);
             }
             tc_commit(&s_full[ns % kTcSBufs]);
             ++ns;
@@ -503,7 +509,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tc_mma_ts(tmem + kTcOCol + (np & 1) * D, pa + kt * 8,
                         dv + static_cast<uint64_t>((kt * kTcBlockBytes) >> 4), kIdPV, np > 1 || kt > 0);
             }
-            tc_commit(&o_done[np & 1]);
             tc_commit(&s_free[np % kTcSBufs]);
             tc_commit(&kv_empty[np % kTcStages]);
             ++np;
@@ -613,10 +618,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // that O_t rarely makes the round trip); when any row of the warp
         // moves, the warp takes the round trip for its 128 columns of O_t,
         // with factor 1 for the rows that stay.  O_t is stable once the set's
-        // previous P V is done.
+        // previous P V (stage s - 2) is done: the free barrier of its S
+        // buffer, whose earlier use (stage s - 2 - kTcSBufs) completed before
+        // S of stage s - 2 was issued, so that its parity is unambiguous.
         const bool move = mx > m_ref + 8.f;
         if (ok && k > 0 && __any_sync(0xffffffffu, move)) {
-          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[hf], (k - 1) & 1, abort_flag, kWaitLimitNs));
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_free[(s - 2) % kTcSBufs], ((s - 2) / kTcSBufs) & 1,
+                                                         abort_flag, kWaitLimitNs));
           if (ok) {
             tc_fence_after();
             const float alpha = move ? exp2f(m_ref - mx) : 1.f;
@@ -667,9 +675,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      // Both sets' accumulators are final once each set's last P V is done.
-      if (ok && k > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[hf], (k - 1) & 1, abort_flag, kWaitLimitNs));
+      // Both sets' accumulators are final once each set's last P V is done
+      // (and with it every earlier MMA).  Its S buffer's free barrier is
+      // waited on, not a per-set counter: when the set's P V two stages
+      // back is still in flight, a per-set barrier would be two phases
+      // behind and its parity would read as done.
+      if (ok && k > 0) {
+        const int s_last = hf + 2 * (k - 1);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_free[s_last % kTcSBufs], (s_last / kTcSBufs) & 1,
+                                                        abort_flag, kWaitLimitNs));
+      }
       // The two sets' states of each row, combined: weights 2^(m_t - max m),
       // 0 for a set with no keys; NaN in the sum marks a row whose pipeline
       // failed.
