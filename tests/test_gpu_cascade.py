@@ -185,3 +185,32 @@ def test_cascade_bad_prefix_block_is_left_out(kernel, splits):
     out = run_cascade(w, cv, check_errors=False, prefix_kernel=kernel, prefix_splits=splits)
     assert pkv.pkv_get_device_error() & pkv.DEVERR_BLOCK_ID
     assert_close(out, ref, w.dtype, what=f"bad prefix blocks, kernel {kernel}")
+
+
+def test_cascade_repeated_full_size_runs_are_bit_identical():
+    # Every run of the same inputs gives the same bits.  A wait that passed
+    # before a set's last P V had finished once left about one full-size run
+    # in fifty with a wrong 128-row tile; sixty runs over three split counts
+    # catch such a race with high probability.  One run is also checked
+    # against the oracle on sampled rows.
+    w = W.shared_prefix(seed=3)
+    dev = torch.device("cuda")
+    kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
+    pkv.paged_kv_append(w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev), kc, vc)
+    cv = W.cascade_view(w)
+    args = [t.to(dev) for t in (cv.prefix_block_tables, cv.prefix_lens, cv.seq_group, cv.block_tables,
+                                cv.context_lens)]
+    q = w.q.to(dev)
+    rows = sample_rows(w, 48)
+    ref, _, _ = oracle.workload_decode(w, rows=rows)
+    for splits in (0, 2, 4):
+        first = None
+        for _ in range(20):
+            out = pkv.paged_attention_decode_cascade(q, kc, vc, *args, w.scale, prefix_splits=splits)
+            if first is None:
+                first = out.clone()
+            else:
+                assert torch.equal(bits(out), bits(first)), f"splits={splits}: runs differ"
+        torch.cuda.synchronize()
+        assert pkv.pkv_get_device_error() == 0
+        assert_close(first.cpu(), ref, w.dtype, rows=rows, what=f"repeated runs, splits={splits}")
