@@ -1235,7 +1235,11 @@ __device__ __forceinline__ void merge_rows(const DecodeParams& p, const MergeSrc
       const float* r = p.records + (static_cast<size_t>(chunk) * 2 + (j == 0 ? src.z : 0)) * p.rec_floats;
       mj[jj] = ld_cg(r + mo);
       lj[jj] = ld_cg(r + lo);
-      if constexpr (DPL == 4) {
+      if constexpr (DPL == 8) {
+        const float4 v = ld_cg4(r + oo), w = ld_cg4(r + oo + 4);
+        o[jj][0] = v.x; o[jj][1] = v.y; o[jj][2] = v.z; o[jj][3] = v.w;
+        o[jj][4] = w.x; o[jj][5] = w.y; o[jj][6] = w.z; o[jj][7] = w.w;
+      } else if constexpr (DPL == 4) {
         const float4 v = ld_cg4(r + oo);
         o[jj][0] = v.x; o[jj][1] = v.y; o[jj][2] = v.z; o[jj][3] = v.w;
       } else if constexpr (DPL == 2) {
@@ -1276,7 +1280,10 @@ __device__ __forceinline__ void merge_rows(const DecodeParams& p, const MergeSrc
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;  // L is 0 only when every piece skipped all its tiles
   T* const ob = static_cast<T*>(p.out) + out_row(p, b, hg, g) * D + d0 + lane * DPL;
-  if constexpr (DPL == 4) {
+  if constexpr (DPL == 8) {
+    store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    store4<DT>(ob + 4, acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  } else if constexpr (DPL == 4) {
     store4<DT>(ob, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
   } else if constexpr (DT == kF32) {
 #pragma unroll
@@ -1690,16 +1697,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const bool sliced = T2 / max(1, n_segs) >= 8 * max(1, s2.Lq);
       const int per_item = sliced ? p.rows * kSlices : p.rows;
       const int items = (by_segment ? n_segs : n_units) * per_item;
-      for (int i = gw; i < items; i += n_warps) {
-        const int x = i / per_item, rem = i - x * per_item;
-        int b, hg, st, en, u1;
+      // Item i's segment (b, hg), row and source pieces; false when it needs
+      // no merge (written in phase 1, or taken from another item).
+      auto item = [&](int i, int& b, int& hg, int& rem, MergeSrc& src) {
+        const int x = i / per_item;
+        rem = i - x * per_item;
+        int st, en, u1;
         if (by_segment) {
           b = x / p.ng;
           hg = x - b * p.ng;
-          if (ctxs[b] == 0) continue;
+          if (ctxs[b] == 0) return false;
           segment_tiles(prefix, ctxs, b, hg, st, en);
           u1 = unit_of_tile(s2, st);
-          if (en <= unit_begin(s2, u1 + 1)) continue;  // the whole segment in one unit: written in phase 1
+          if (en <= unit_begin(s2, u1 + 1)) return false;  // the whole segment in one unit: written in phase 1
         } else {
           u1 = x;
           const int a = unit_begin(s2, u1), e = unit_begin(s2, u1 + 1);
@@ -1708,13 +1718,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           b = wl.b;
           hg = wl.hg;
           segment_tiles(prefix, ctxs, b, hg, st, en);
-          if (st < a || en <= e) continue;  // started in an earlier unit, or ends in this one
+          if (st < a || en <= e) return false;  // started in an earlier unit, or ends in this one
         }
-        const MergeSrc src = {u1, st == unit_begin(s2, u1) ? 0 : 1, unit_of_tile(s2, en - 1) - u1 + 1, u1, 1};
-        if (sliced)
-          merge_rows<DT, D, 1>(p, src, b, hg, rem / kSlices, (rem % kSlices) * 32, lane, nullptr);
-        else
-          merge_rows<DT, D, D / 32>(p, src, b, hg, rem, 0, lane, nullptr);
+        src = {u1, st == unit_begin(s2, u1) ? 0 : 1, unit_of_tile(s2, en - 1) - u1 + 1, u1, 1};
+        return true;
+      };
+      if (sliced) {
+        for (int i = gw; i < items; i += n_warps) {
+          int b, hg, rem;
+          MergeSrc src;
+          if (item(i, b, hg, rem, src))
+            merge_rows<DT, D, 1>(p, src, b, hg, rem / kSlices, (rem % kSlices) * 32, lane, nullptr);
+        }
+      } else {
+        // Each half-warp takes items of its own (16 lanes, D / 16 dims per
+        // lane): a merge is a round trip or two of loads, so that two in
+        // flight per warp halve the rounds of phase 2.
+        const int half = lane >> 4;
+        for (int i = 2 * gw + half; i < items; i += 2 * n_warps) {
+          int b, hg, rem;
+          MergeSrc src;
+          if (item(i, b, hg, rem, src)) merge_rows<DT, D, D / 16>(p, src, b, hg, rem, 0, lane & 15, nullptr);
+        }
       }
     } else {
       // Balancing chunks: the chunk that holds a split segment's first piece
