@@ -1000,17 +1000,27 @@ struct MmaConsumerI8 : MmaConsumer<DT, 128, GPAD> {
                    : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
                    : "r"(kbase + row * 128 + (((2 * t + 1) ^ (row & 7)) << 4)));
       const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+      if constexpr (GPAD == 16) {
+        int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        // With at most 8 rows, rows 8..15 of A are zero (literal zeros: no registers held).
-        const uint32_t h1 = GPAD == 16 ? qa[kk][1] : 0u, h3 = GPAD == 16 ? qa[kk][3] : 0u;
-        const uint32_t l1 = GPAD == 16 ? qa[4 + kk][1] : 0u, l3 = GPAD == 16 ? qa[4 + kk][3] : 0u;
-        mma_16832_s8(ah, qa[kk][0], h1, qa[kk][2], h3, w[2 * kk], w[2 * kk + 1]);
-        mma_16832_s8(al, qa[4 + kk][0], l1, qa[4 + kk][2], l3, w[2 * kk], w[2 * kk + 1]);
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_16832_s8(ah, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], w[2 * kk], w[2 * kk + 1]);
+          mma_16832_s8(al, qa[4 + kk][0], qa[4 + kk][1], qa[4 + kk][2], qa[4 + kk][3], w[2 * kk], w[2 * kk + 1]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = static_cast<float>(ah[e] * 128 + al[e]);
+      } else {
+        // At most 8 rows: the high parts of Q go in A's rows 0-7 and the low
+        // parts in rows 8-15, so that one MMA per k-step gives both dot
+        // products, in the same lane (c0, c1: high; c2, c3: low).
+        int a[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_16832_s8(a, qa[kk][0], qa[4 + kk][0], qa[kk][2], qa[4 + kk][2], w[2 * kk], w[2 * kk + 1]);
+        s[nt][0] = static_cast<float>(a[0] * 128 + a[2]);
+        s[nt][1] = static_cast<float>(a[1] * 128 + a[3]);
+        s[nt][2] = s[nt][3] = 0.f;  // rows 8-15: none
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] = static_cast<float>(ah[e] * 128 + al[e]);
     }
     // Scales: the row's grid step and the K scale of this lane's columns
     // (tokens 2t, 2t + 1 and 2t + 8, 2t + 9).
