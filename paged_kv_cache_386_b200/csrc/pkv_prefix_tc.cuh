@@ -89,9 +89,9 @@ static_assert(kTcOutOffset + kTcRows * 512 <= kTcRingBytes, "output rows fit in 
 // Barriers (K/V full and empty per ring slot; S full, S buffer free and P
 // full per S buffer; one to drain the MMAs on an abort), the tensor-memory
 // slot and the abort flag, then the exchange arrays of the set merge (maxima
-// [2][128], sums [2][128]) and the destination rows [128].
+// [2][128], sums [2][128]).
 constexpr int kTcBarBytes = (2 * kTcStages + 3 * kTcSBufs + 1) * 8 + 16;
-constexpr int kTcExchBytes = (2 * kTcRows + 2 * kTcRows + kTcRows) * 4;
+constexpr int kTcExchBytes = (2 * kTcRows + 2 * kTcRows) * 4;
 
 // Softmax arithmetic with fewer issue slots: two fp32 lanes per packed FMA /
 // add (sm_100), two new values per three-input max, and the hardware base-2
@@ -272,8 +272,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red_max = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kTcBarBytes);  // [2][128]
   float* red_l = red_max + 2 * kTcRows;                                                     // [2][128]
-  int* row_dst = reinterpret_cast<int*>(red_l + 2 * kTcRows);                               // [128]
-  int* members = row_dst + kTcRows;                                                         // [batch]
+  int* members = reinterpret_cast<int*>(red_l + 2 * kTcRows);                               // [batch]
   __shared__ int warp_counts[kTcThreads / 32];
   __shared__ int set_ok[2][kTcSetWarps];
   __shared__ int n_members;
@@ -723,16 +722,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           part_ml[r] = m_ref;
           part_ml[kTcRows + r] = l_row;
         }
+      } else {
+        // This warp's 64 columns of its own share of O, not yet weighted, into
+        // [128 rows][512 B] (16-byte chunk c of row r at c ^ (r % 8)); done
+        // before the cluster barrier, so that it overlaps the other CTAs'
+        // partial writes.
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float t[32];
+          load_o(c, t);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int chunk = (hf * 16 + c * 8 + i) ^ (r & 7);
+            *reinterpret_cast<float4*>(out_s + r * 512 + chunk * 16) =
+                make_float4(t[4 * i], t[4 * i + 1], t[4 * i + 2], t[4 * i + 3]);
+          }
+        }
       }
     }
   }
   tc_fence_before();
-  cluster_sync();  // partial states written
+  cluster_sync();  // partial states and own shares written
   tc_fence_after();
   if (warp < kTcSoftmaxWarps && owner == crank) {
     // The row's state, merged over the cluster: O (unnormalised), m, l.
+    // Rows out, coalesced: warp (lg, hf) takes rows 32 lg + 16 hf .. + 15,
+    // lane l the 16-byte chunk l of each; the other shares of the same chunk
+    // come from their CTAs' shared memory, one 512-byte row per warp-wide
+    // load, weighted with the factors of the lane that holds the row's state
+    // (lane 16 hf + j for row 32 lg + 16 hf + j).  The first other share's
+    // rows are requested together with every share's m and l.
     const uint32_t part_o_addr = smem_u32(ring);
     const uint32_t part_ml_addr = part_o_addr + kTcRows * kTcPartStride * 4;
+    const int rbase = lg * 32 + hf * 16;
+    const uint32_t first = crank == 0 ? 1u : 0u;  // the first other CTA of the cluster
     float m_all = m_ref;
     float wk[kTcMaxSplit], lk[kTcMaxSplit];
     bool valid = !isnan(l_row);
@@ -743,6 +766,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (k < static_cast<int>(csize) && k != static_cast<int>(crank)) {
         wk[k] = ld_cluster(cluster_map(part_ml_addr + r * 4, k));
         lk[k] = ld_cluster(cluster_map(part_ml_addr + (kTcRows + r) * 4, k));
+      }
+    }
+    float4 t[16];
+    if (csize > 1) {
+      const uint32_t src = cluster_map(part_o_addr + (rbase * kTcPartStride + lane * 4) * 4, first);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) t[j] = ld_cluster4(src + j * kTcPartStride * 4);
+    }
+    float4 o[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int rr = rbase + j;
+      o[j] = *reinterpret_cast<const float4*>(out_s + rr * 512 + ((lane ^ (rr & 7)) * 16));
+    }
+#pragma unroll
+    for (int k = 0; k < kTcMaxSplit; ++k) {
+      if (k < static_cast<int>(csize) && k != static_cast<int>(crank)) {
         valid = valid && !isnan(lk[k]);
         m_all = fmaxf(m_all, wk[k]);
       }
@@ -756,47 +796,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       l_all += wk[k] * lk[k];
     }
     const int row = row0 + r;
-    if (hf == 0) {
-      int dst = -1;
-      if (row < R && valid) {
-        dst = members[row / G] * p.n_q_heads + kvh * G + row % G;
+    int dst = -1;  // this lane's row's destination (-1: none)
+    if (row < R && valid) {
+      dst = members[row / G] * p.n_q_heads + kvh * G + row % G;
+      if (hf == 0) {
         const size_t nqb = static_cast<size_t>(p.batch) * p.n_q_heads;
         p.init[nqb * D + dst] = m_all;
         p.init[nqb * D + nqb + dst] = l_all;
       }
-      row_dst[r] = dst;
     }
-    // This warp's 64 columns of its own share of O, weighted, into
-    // [128 rows][512 B] (16-byte chunk c of row r at c ^ (r % 8)).
+    float w_first = 0.f;
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      float t[32];
-      load_o(c, t);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int chunk = (hf * 16 + c * 8 + i) ^ (r & 7);
-        *reinterpret_cast<float4*>(out_s + r * 512 + chunk * 16) =
-            make_float4(t[4 * i] * a_self, t[4 * i + 1] * a_self, t[4 * i + 2] * a_self, t[4 * i + 3] * a_self);
-      }
-    }
-    named_bar_sync(2 + lg, 64);
-    // Rows out, coalesced: warp (lg, hf) takes rows 32 lg + 16 hf .. + 15,
-    // lane l the 16-byte chunk l of each.  The other shares of the same
-    // chunk are added from their CTAs' shared memory, one 512-byte row per
-    // warp-wide load, with the row's weight from the lane that owns the row.
-    const int rbase = lg * 32 + hf * 16;
-    const int dst_l = row_dst[rbase + (lane & 15)];
-    float4 o[16];
+    for (int k = 0; k < kTcMaxSplit; ++k) w_first = k == static_cast<int>(first) ? wk[k] : w_first;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const int rr = rbase + j;
-      o[j] = *reinterpret_cast<const float4*>(out_s + rr * 512 + ((lane ^ (rr & 7)) * 16));
+      const float ws = __shfl_sync(0xffffffffu, a_self, hf * 16 + j);
+      o[j].x *= ws;
+      o[j].y *= ws;
+      o[j].z *= ws;
+      o[j].w *= ws;
+    }
+    if (csize > 1) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float w = __shfl_sync(0xffffffffu, w_first, hf * 16 + j);
+        o[j].x += w * t[j].x;
+        o[j].y += w * t[j].y;
+        o[j].z += w * t[j].z;
+        o[j].w += w * t[j].w;
+      }
     }
 #pragma unroll
     for (int k = 0; k < kTcMaxSplit; ++k) {
-      if (k < static_cast<int>(csize) && k != static_cast<int>(crank)) {
+      if (k < static_cast<int>(csize) && k != static_cast<int>(crank) && k != static_cast<int>(first)) {
         const uint32_t src = cluster_map(part_o_addr + (rbase * kTcPartStride + lane * 4) * 4, k);
-        float4 t[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) t[j] = ld_cluster4(src + j * kTcPartStride * 4);
 #pragma unroll
@@ -811,8 +844,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const int dst = __shfl_sync(0xffffffffu, dst_l, j);
-      if (dst >= 0) *reinterpret_cast<float4*>(p.init + static_cast<size_t>(dst) * D + lane * 4) = o[j];
+      const int d = __shfl_sync(0xffffffffu, dst, hf * 16 + j);
+      if (d >= 0) *reinterpret_cast<float4*>(p.init + static_cast<size_t>(d) * D + lane * 4) = o[j];
     }
   }
   tc_fence_before();
